@@ -1,1 +1,11 @@
-"""B200-native exact attention forward (sm_100a, tcgen05/TMEM/TMA)."""
+"""B200-native exact attention forward (sm_100a: tcgen05 / TMEM / TMA).
+
+The compute path is libfa.so (C ABI in include/fa.h); this package holds its
+sources (csrc/), its build step (build.py), the ctypes binding (binding.py)
+and the seeded input generator (inputs.py).
+"""
+from .binding import (FA_BF16, FA_F16, FaError, fa_fwd, fa_get_device_status,
+                      fa_version, flash_fwd, load, status_string)
+
+__all__ = ["FA_BF16", "FA_F16", "FaError", "fa_fwd", "fa_get_device_status",
+           "fa_version", "flash_fwd", "load", "status_string"]

@@ -1,0 +1,130 @@
+"""Python binding of the C ABI in include/fa.h (argument marshalling only).
+
+``fa_fwd`` mirrors the C entry point one to one (raw pointers and sizes).
+``flash_fwd`` is the convenience call for torch tensors: it checks shapes,
+allocates ``out`` / ``lse`` with torch and passes the current stream; every
+step of the attention itself runs in libfa.so's kernels.  There is no CPU or
+eager fallback: if libfa.so cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "lib", "libfa.so")
+
+FA_F16, FA_BF16 = 0, 1
+FA_OK = 0
+STATUS = {
+    0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_SHAPE", -3: "FA_ERR_HEADDIM",
+    -4: "FA_ERR_DTYPE", -5: "FA_ERR_ALIGN", -6: "FA_ERR_ARG", -7: "FA_ERR_CUDA",
+    -8: "FA_ERR_TIMEOUT",
+}
+EXPORTS = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FaError(RuntimeError):
+    """A non-zero status from libfa.so."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} "
+                         f"({status_string(status) if _lib is not None else ''})")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfa.so (in-tree build) and declare the C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"libfa.so not found at {path}; build it with "
+                "`python -m exact_attention_113_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(path)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
+                               i, i, i, i, vp]
+        lib.fa_fwd.restype = i
+        lib.fa_get_device_status.argtypes = [vp]
+        lib.fa_get_device_status.restype = i
+        lib.fa_status_string.argtypes = [i]
+        lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_version.argtypes = []
+        lib.fa_version.restype = i
+        _lib = lib
+        return lib
+
+
+# ------------------------------------------------------------ raw C calls
+def fa_fwd(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
+           window_left, window_right, dtype, stream) -> int:
+    """The C entry point, unchanged: pointers as ints, returns the status."""
+    return load().fa_fwd(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D,
+                         float(scale), int(causal), int(window_left),
+                         int(window_right), int(dtype), stream)
+
+
+def fa_get_device_status(stream=None) -> int:
+    return load().fa_get_device_status(stream)
+
+
+def status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def fa_version() -> int:
+    return load().fa_version()
+
+
+# ------------------------------------------------------------ torch call
+def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
+              return_lse=True, out=None, lse=None, stream=None):
+    """Exact attention forward on CUDA tensors.
+
+    q: [B, H, L_q, D]; k, v: [B, H_kv, L_k, D]; fp16 or bf16, contiguous, on
+    one CUDA device.  ``scale`` defaults to 1/sqrt(D).  Returns ``(out, lse)``
+    (``lse`` is None unless ``return_lse``).  Launches asynchronously on
+    ``stream`` (default: torch's current stream).
+    """
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, H, L, D]")
+    B, H, L_q, D = q.shape
+    Bk, H_kv, L_k, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
+        raise ValueError("k, v must be [B, H_kv, L_k, D] with q's B and D")
+    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype \
+            or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share dtype float16 or bfloat16")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+    dtype = FA_F16 if q.dtype == torch.float16 else FA_BF16
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, L_q), dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                    lse.data_ptr() if lse is not None else None,
+                    B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                    window_right, dtype, stream.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd")
+    return out, lse

@@ -1,0 +1,100 @@
+"""Build libfa.so (the C ABI of include/fa.h) for sm_100a with nvcc.
+
+The library is built in-tree, at exact_attention_113_b200/lib/libfa.so, and
+links the CUDA runtime statically; it reaches the driver's tensor-map encoder
+through cudaGetDriverEntryPoint, so it loads on a machine without a GPU.
+
+    python -m exact_attention_113_b200.build [--verbose]
+"""
+from __future__ import annotations
+
+import os
+import re
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB_DIR = os.path.join(PKG, "lib")
+LIB_PATH = os.path.join(LIB_DIR, "libfa.so")
+SOURCES = [os.path.join(CSRC, "fa_api.cu")]
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "fa_fwd_kernel.cuh")] + [
+    os.path.join(INCLUDE, "fa.h")]
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC", "-shared",
+    "-cudart", "static",
+]
+
+
+def nvcc() -> str:
+    cand = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def is_stale() -> bool:
+    if not os.path.exists(LIB_PATH):
+        return True
+    t = os.path.getmtime(LIB_PATH)
+    return any(os.path.getmtime(p) > t for p in DEPENDS)
+
+
+# The attention kernel launches 384 threads and re-splits its registers with
+# setmaxnreg (2 warpgroups x 216 + 1 x 64 <= 384 x 168).  That split is only
+# valid when every instance is compiled at exactly this many registers.
+LAUNCH_REGS = 168
+KERNEL_TAG = "fa_fwd_kernel"
+
+
+def check_register_counts(ptxas_log: str) -> dict:
+    """Parse `ptxas -v` output; require LAUNCH_REGS for every kernel instance."""
+    counts, current = {}, None
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Function properties for (\S+)", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Compiling entry function '(\S+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current and KERNEL_TAG in current:
+            counts[current] = int(m.group(1))
+    if not counts:
+        raise RuntimeError("no register counts found for the attention kernel")
+    bad = {k: v for k, v in counts.items() if v != LAUNCH_REGS}
+    if bad:
+        raise RuntimeError(f"attention kernel register count != {LAUNCH_REGS}: {bad}; "
+                           "the setmaxnreg split would not match the launch")
+    return counts
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not is_stale():
+        return LIB_PATH
+    os.makedirs(LIB_DIR, exist_ok=True)
+    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    cmd = [nvcc(), "-Xptxas=-v", *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
+           *SOURCES]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building libfa.so")
+    if verbose:
+        sys.stderr.write(res.stdout + res.stderr)
+    try:
+        check_register_counts(res.stdout + res.stderr)
+    except RuntimeError:
+        os.remove(tmp)
+        raise
+    os.replace(tmp, LIB_PATH)
+    return LIB_PATH
+
+
+if __name__ == "__main__":
+    print(build(force=True, verbose="--verbose" in sys.argv))

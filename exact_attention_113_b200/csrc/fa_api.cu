@@ -1,0 +1,209 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, TMA
+// tensor-map encoding, kernel selection and launch, device status.
+//
+// Operator statement followed ("FlashAttention算法原理与性能优化实战" section
+// 2.2): 4-D [B, H, S, D] query/key/value, an output shaped like the query,
+// fp32 softmax statistics of shape [B, H, S]; scale, pre_tokens and
+// next_tokens as attributes.  The statistics here are one log-sum-exp per row
+// (Triton FA2 walkthrough: the logsumexp kept for the backward pass).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kMaxSeq = 1 << 30;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A rank-3 tensor map over a contiguous [n_heads, L, D] array with a box of
+// [1, 128, box_cols] and the swizzle that matches `box_cols` 16-bit elements.
+bool encode_map(CUtensorMap *map, const void *base, int dtype, int n_heads, int L, int D,
+                int box_cols) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType dt =
+      dtype == FA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(n_heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(L) * D * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const int sw_bytes = box_cols * 2;
+  const CUtensorMapSwizzle sw = sw_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : sw_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+__global__ void fill_kernel(float *p, size_t n, float value) {
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (; i < n; i += stride) p[i] = value;
+}
+
+template <int D, int DT>
+int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
+  using G = Geo<D>;
+  auto kern = fa_fwd_kernel<D, DT>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  static bool configured[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    if (!configured[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               G::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+      configured[dev] = true;
+    }
+  }
+  dim3 grid(static_cast<unsigned>(prm.n_qpairs) * static_cast<unsigned>(B * H), 1, 1);
+  kern<<<grid, kThreads, G::kSmemBytes, stream>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                      int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                      int causal, int window_left, int window_right, int dtype,
+                      cudaStream_t stream) {
+  // ---------------------------------------------------------------- checks
+  if (!q || !k || !v || !out) return FA_ERR_NULL;
+  if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
+  if (H % H_kv != 0) return FA_ERR_SHAPE;
+  if (L_q > kMaxSeq || L_k > kMaxSeq) return FA_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * H * ((static_cast<int64_t>(L_q) + 255) / 256) >
+      (1ll << 31) - 1)
+    return FA_ERR_SHAPE;                   // one CTA per (head, 256 query rows)
+  if (D != 16 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return FA_ERR_ALIGN;
+  if (lse && !aligned(lse, 4)) return FA_ERR_ALIGN;
+  if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+
+  // ---------------------------------------------------------------- edges
+  if (L_q == 0) return FA_OK;
+  if (L_k == 0) {
+    // no key is visible: O = 0, lse = -inf
+    const size_t n_out = static_cast<size_t>(B) * H * L_q * D * 2;
+    if (cudaMemsetAsync(out, 0, n_out, stream) != cudaSuccess) return FA_ERR_CUDA;
+    if (lse) {
+      const size_t n = static_cast<size_t>(B) * H * L_q;
+      fill_kernel<<<148, 256, 0, stream>>>(lse, n, -INFINITY);
+      if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
+  }
+
+  // ---------------------------------------------------------------- params
+  FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  int wl = window_left < 0 ? -1 : window_left;
+  int wr = window_right < 0 ? -1 : window_right;
+  if (causal) wr = 0;                      // causal => wr := min(wr, 0)
+  if (wl >= L_q) wl = -1;                  // no constraint left of row 0
+  if (wr >= L_k) wr = -1;                  // no constraint right of L_k - 1
+  prm.lse = lse;
+  prm.H = H;
+  prm.H_kv = H_kv;
+  prm.L_q = L_q;
+  prm.L_k = L_k;
+  prm.group = H / H_kv;
+  prm.n_qpairs = (L_q + 2 * kBM - 1) / (2 * kBM);
+  prm.wl = wl;
+  prm.wr = wr;
+  prm.reverse = (wr >= 0) ? 1 : 0;         // later query tiles see more keys
+  {
+    float sl2 = scale * 1.4426950408889634f;
+    prm.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;
+  }
+  const int box_cols = D * 2 >= 128 ? 64 : D;
+  if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
+      !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
+      !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
+      !encode_map(&prm.tm_o, out, dtype, B * H, L_q, D, box_cols))
+    return FA_ERR_CUDA;
+
+  switch (D * 2 + dtype) {
+    case 32: return launch<16, 0>(prm, B, H, stream);
+    case 33: return launch<16, 1>(prm, B, H, stream);
+    case 64: return launch<32, 0>(prm, B, H, stream);
+    case 65: return launch<32, 1>(prm, B, H, stream);
+    case 128: return launch<64, 0>(prm, B, H, stream);
+    case 129: return launch<64, 1>(prm, B, H, stream);
+    case 256: return launch<128, 0>(prm, B, H, stream);
+    case 257: return launch<128, 1>(prm, B, H, stream);
+  }
+  return FA_ERR_HEADDIM;
+}
+
+extern "C" int fa_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int st = 0;
+  if (cudaMemcpyFromSymbol(&st, g_fa_status, sizeof(st)) != cudaSuccess) return FA_ERR_CUDA;
+  if (st != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(zero)) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+extern "C" const char *fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+    case FA_ERR_SHAPE: return "FA_ERR_SHAPE: bad sizes (B,H,H_kv>=1, L>=0, H%H_kv==0)";
+    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: D must be 16, 32, 64 or 128";
+    case FA_ERR_DTYPE: return "FA_ERR_DTYPE: dtype must be FA_F16 or FA_BF16";
+    case FA_ERR_ALIGN: return "FA_ERR_ALIGN: q/k/v/out need 16-byte, lse 4-byte alignment";
+    case FA_ERR_ARG: return "FA_ERR_ARG: scale must be finite and >= 0";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "unknown fa status";
+}
+
+extern "C" int fa_version(void) { return kVersion; }

@@ -1,0 +1,538 @@
+// fa_fwd_kernel.cuh -- exact attention forward for sm_100a.
+//
+// What it computes (per (batch, head), query row i):
+//   O_i = sum_j softmax_j(scale * q_i . k_j | visible) v_j,
+//   lse_i = ln sum_j exp(scale * q_i . k_j) over visible j,
+// with the online softmax of "Flash Attention是怎么做到又快又省显存的？"
+// (running max m and normaliser d', rescaled when the max grows), in the FA2
+// loop order of the Triton FA2 walkthrough (outer loop over query tiles, one
+// per CTA slot; inner loop over K/V blocks; division by the normaliser moved
+// to the end) and never writing the score matrix to global memory.
+//
+// CTA layout (384 threads = 3 warpgroups, one CTA per SM):
+//   warps 0-3   softmax warpgroup for query tile 0 (rows q0 .. q0+127)
+//   warps 4-7   softmax warpgroup for query tile 1 (rows q0+128 .. q0+255)
+//   warp  8     MMA issuer (one thread) and TMEM owner
+//   warp  9     TMA producer (one thread)
+//   warps 10-11 idle
+// Each softmax thread owns one query row, which is one TMEM lane.
+// Registers: launched at kLaunchRegs per thread; the third warpgroup gives
+// back down to kSmallRegs and the two softmax warpgroups grow to kBigRegs:
+//   2*128*kBigRegs + 128*kSmallRegs <= 384*kLaunchRegs (63488 <= 64512).
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
+// O1 [256+D, 256+2D).  P_t (fp16/bf16, two per 32-bit column) is written over
+// the first 64 columns of S_t and read by the PV MMA straight from TMEM.
+//
+// MMA issue order per K/V block j (the ping-pong of the two query tiles):
+//   S0(j), PV1(j-1), S1(j), PV0(j)
+// so that while softmax warpgroup 0 works on S0(j), the tensor pipe runs
+// PV1(j-1) and S1(j), and the other way round.  S_t(j+1) is issued after
+// PV_t(j), which reads P_t from the same TMEM columns; tcgen05 MMAs issued by
+// one thread execute in issue order.
+//
+// Shared memory: Q tile 0, Q tile 1, then a ring of kSlots K/V tiles loaded in
+// the order K_lo, V_lo, K_lo+1, V_lo+1, ...  Tiles are stored as TMA writes
+// them (rows of `kSwBytes`, swizzled), which is the canonical K-major layout
+// for Q and K and the canonical MN-major layout for V.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;        // query rows per tile = TMEM lanes
+constexpr int kBN = 128;        // keys per K/V block
+constexpr int kThreads = 384;
+constexpr uint32_t kLaunchRegs = 168;   // 65536 / 384, rounded down to 8
+constexpr uint32_t kBigRegs = 216;
+constexpr uint32_t kSmallRegs = 64;
+static_assert(2 * 128 * kBigRegs + 128 * kSmallRegs <= kThreads * kLaunchRegs,
+              "register split must fit in the launch allocation");
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
+
+struct FwdParams {
+  CUtensorMap tm_q;   // [B*H,    L_q, D]
+  CUtensorMap tm_k;   // [B*H_kv, L_k, D]
+  CUtensorMap tm_v;   // [B*H_kv, L_k, D]
+  CUtensorMap tm_o;   // [B*H,    L_q, D]
+  float *lse;         // [B*H, L_q] or nullptr
+  int H, H_kv, L_q, L_k;
+  int group;          // H / H_kv
+  int n_qpairs;       // ceil(L_q / 256)
+  int wl, wr;         // visible iff i - wl <= j <= i + wr; -1 = unbounded
+  int reverse;        // process query pairs last-first (causal: heavy first)
+  float scale_log2;   // scale * log2(e), clamped to >= 1e-30
+};
+
+template <int D>
+struct Geo {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kSwBytes = kRowBytes >= 128 ? 128 : kRowBytes;  // swizzle span
+  static constexpr int kBoxCols = kSwBytes / 2;                       // elements per box row
+  static constexpr int kNumBox = kRowBytes / kSwBytes;                 // column boxes per tile
+  static constexpr int kBoxBytes = kBM * kSwBytes;
+  static constexpr int kTileBytes = kBM * kRowBytes;
+  static constexpr int kSlots = D == 128 ? 5 : (D == 64 ? 8 : 16);
+  static constexpr uint32_t kLayout = kSwBytes == 128 ? 2u : (kSwBytes == 64 ? 4u : 6u);
+  static constexpr int kUnitsPerBoxRow = kSwBytes / 16;
+  // shared memory map (offsets from a 1024-byte aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kUsed = kOffBar + kBarBytes;
+  // at least ~116 KB so that only one CTA (and one 512-column TMEM
+  // allocation) fits on an SM
+  static constexpr int kSmemBytes = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(256 + 2 * D <= 512, "TMEM budget");
+};
+
+// Barrier block inside shared memory.
+template <int kSlots>
+struct Bars {
+  uint64_t q_full[2];
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Key range [lo, hi) in blocks for query rows [first, last] of one tile.
+struct BlockRange {
+  int lo, hi;
+};
+
+__device__ __forceinline__ BlockRange tile_block_range(int first, int last, int L_k, int wl,
+                                                       int wr) {
+  int klo = wl < 0 ? 0 : max(0, first - wl);
+  int khi = wr < 0 ? L_k - 1 : min(L_k - 1, last + wr);
+  BlockRange r;
+  if (khi < klo) {
+    r.lo = 0;
+    r.hi = 0;
+  } else {
+    r.lo = klo / kBN;
+    r.hi = khi / kBN + 1;
+  }
+  return r;
+}
+
+template <int D, int DT>
+__global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using G = Geo<D>;
+  constexpr int kSlots = G::kSlots;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Bars<kSlots> *bars = reinterpret_cast<Bars<kSlots> *>(smem + G::kOffBar);
+  volatile int *abort_flag = &bars->abort_flag;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // ---- work item: (batch*head, pair of query tiles); consecutive CTAs take
+  // consecutive query pairs of one head, so a head's K/V stays hot in L2.
+  const int bh = static_cast<int>(blockIdx.x) / p.n_qpairs;
+  const int qp_idx = static_cast<int>(blockIdx.x) - bh * p.n_qpairs;
+  const int qpair = p.reverse ? (p.n_qpairs - 1 - qp_idx) : qp_idx;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+  const int bh_kv = b * p.H_kv + h / p.group;   // GQA: contiguous head groups
+
+  int q0[2], rows[2];
+  BlockRange rng[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    q0[t] = qpair * 2 * kBM + t * kBM;
+    rows[t] = max(0, min(kBM, p.L_q - q0[t]));
+    if (rows[t] > 0) {
+      rng[t] = tile_block_range(q0[t], q0[t] + rows[t] - 1, p.L_k, p.wl, p.wr);
+    } else {
+      rng[t].lo = 0;
+      rng[t].hi = 0;
+    }
+  }
+  const bool act0 = rng[0].hi > rng[0].lo, act1 = rng[1].hi > rng[1].lo;
+  const int lo = act0 ? (act1 ? min(rng[0].lo, rng[1].lo) : rng[0].lo) : rng[1].lo;
+  const int hi = act0 ? (act1 ? max(rng[0].hi, rng[1].hi) : rng[0].hi) : rng[1].hi;
+  const bool any_work = act0 || act1;
+
+  // ---- setup
+  if (tid == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&bars->q_full[t]), 1);
+      mbar_init(smem_u32(&bars->s_full[t]), 1);
+      mbar_init(smem_u32(&bars->p_full[t]), kBM);
+      mbar_init(smem_u32(&bars->pv_done[t]), 1);
+    }
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(smem_u32(&bars->full[s]), 1);
+      mbar_init(smem_u32(&bars->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->mma_done), 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_k);
+    prefetch_tensormap(&p.tm_v);
+    prefetch_tensormap(&p.tm_o);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  const uint32_t sQ = smem_u32(smem + G::kOffQ);
+  const uint32_t sRing = smem_u32(smem + G::kOffRing);
+
+  if (warp >= 8) {
+  // ===================================================== warpgroup 2
+  regs_dec<kSmallRegs>();
+  if (warp == kLoadWarp) {
+    // =================================================== TMA producer
+    if (lane == 0 && any_work) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (rng[t].hi <= rng[t].lo) continue;
+        const uint32_t bar = smem_u32(&bars->q_full[t]);
+        mbar_arrive_expect_tx(bar, G::kTileBytes);
+        for (int bx = 0; bx < G::kNumBox; ++bx)
+          tma_load_3d(sQ + t * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, bar,
+                      bx * G::kBoxCols, q0[t], bh, pol_stream);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int j = lo; j < hi && ok; ++j) {
+        for (int which = 0; which < 2; ++which, ++it) {
+          const int slot = it % kSlots;
+          if (it >= kSlots) {
+            ok = mbar_wait(smem_u32(&bars->empty[slot]), ((it / kSlots) - 1) & 1, abort_flag);
+            if (!ok) break;
+          }
+          const uint32_t bar = smem_u32(&bars->full[slot]);
+          mbar_arrive_expect_tx(bar, G::kTileBytes);
+          const CUtensorMap *map = which == 0 ? &p.tm_k : &p.tm_v;
+          for (int bx = 0; bx < G::kNumBox; ++bx)
+            tma_load_3d(sRing + slot * G::kTileBytes + bx * G::kBoxBytes, map, bar,
+                        bx * G::kBoxCols, j * kBN, bh_kv, pol_keep);
+        }
+      }
+      if (!ok) {
+        // drain: let the copies already issued land before the CTA exits
+        for (int k = max(0, it - kSlots); k < it; ++k)
+          mbar_wait_slow(smem_u32(&bars->full[k % kSlots]), (k / kSlots) & 1, abort_flag,
+                         false);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // =================================================== MMA issuer
+    if (lane == 0 && any_work) {
+      constexpr uint32_t kIdescS = make_idesc_f16(kBM, kBN, DT, 0, 0);
+      constexpr uint32_t kIdescPV = make_idesc_f16(kBM, D, DT, 0, 1);
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      bool ok = true;
+      if (act0) ok = mbar_wait(smem_u32(&bars->q_full[0]), 0, abort_flag);
+      if (act1 && ok) ok = mbar_wait(smem_u32(&bars->q_full[1]), 0, abort_flag);
+      int npv[2] = {0, 0};
+
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = sQ + t * G::kTileBytes;
+        const uint32_t ka = sRing + slot * G::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int byte = kk * 32;
+          const uint32_t off = (byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes);
+          const uint64_t ad = smem_desc(qa + off, 16, 8 * G::kSwBytes, G::kLayout);
+          const uint64_t bd = smem_desc(ka + off, 16, 8 * G::kSwBytes, G::kLayout);
+          mma_ss(tS[t], ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&bars->s_full[t]));
+      };
+      auto issue_pv = [&](int t, int slot) {
+        const uint32_t va = sRing + slot * G::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd =
+              smem_desc(va + kk * 16 * G::kSwBytes, G::kBoxBytes, 8 * G::kSwBytes, G::kLayout);
+          mma_ts(tO[t], tS[t] + kk * 8, bd, kIdescPV, (npv[t] > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&bars->pv_done[t]));
+        ++npv[t];
+      };
+      auto in = [&](int t, int j) { return j >= rng[t].lo && j < rng[t].hi; };
+      auto slot_of = [&](int idx) { return idx % kSlots; };
+      auto par_of = [&](int idx) { return static_cast<uint32_t>((idx / kSlots) & 1); };
+
+      for (int j = lo; j < hi && ok; ++j) {
+        const int ik = 2 * (j - lo), iv = ik + 1;
+        ok = mbar_wait(smem_u32(&bars->full[slot_of(ik)]), par_of(ik), abort_flag);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (in(0, j)) issue_s(0, slot_of(ik));
+        if (j > lo) {
+          if (in(1, j - 1)) {
+            ok = mbar_wait(smem_u32(&bars->full[slot_of(iv - 2)]), par_of(iv - 2), abort_flag) &&
+                 mbar_wait(smem_u32(&bars->p_full[1]), npv[1] & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_pv(1, slot_of(iv - 2));
+          }
+          tc_commit(smem_u32(&bars->empty[slot_of(iv - 2)]));
+        }
+        if (in(1, j)) issue_s(1, slot_of(ik));
+        tc_commit(smem_u32(&bars->empty[slot_of(ik)]));
+        if (in(0, j)) {
+          ok = mbar_wait(smem_u32(&bars->full[slot_of(iv)]), par_of(iv), abort_flag) &&
+               mbar_wait(smem_u32(&bars->p_full[0]), npv[0] & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_pv(0, slot_of(iv));
+        }
+      }
+      if (ok) {
+        const int iv = 2 * (hi - 1 - lo) + 1;
+        if (in(1, hi - 1)) {
+          ok = mbar_wait(smem_u32(&bars->full[slot_of(iv)]), par_of(iv), abort_flag) &&
+               mbar_wait(smem_u32(&bars->p_full[1]), npv[1] & 1, abort_flag);
+          if (ok) {
+            tc_fence_after_sync();
+            issue_pv(1, slot_of(iv));
+          }
+        }
+        tc_commit(smem_u32(&bars->empty[slot_of(iv)]));
+      }
+      tc_commit(smem_u32(&bars->mma_done));
+    } else if (lane == 0) {
+      tc_commit(smem_u32(&bars->mma_done));
+    }
+  }
+  } else {
+    // =================================================== softmax / epilogue
+    regs_inc<kBigRegs>();
+    const int t = warp >> 2;             // query tile of this warpgroup
+    const int r = tid & 127;             // row within the tile = TMEM lane
+    // this tile's scalars (selected, so that nothing is indexed at run time)
+    const int tq0 = t ? q0[1] : q0[0];
+    const int trows = t ? rows[1] : rows[0];
+    const int tlo = t ? rng[1].lo : rng[0].lo;
+    const int n_blocks = t ? rng[1].hi - rng[1].lo : rng[0].hi - rng[0].lo;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * 128u;
+    const uint32_t tO = tmem + lane_base + 256u + t * D;
+    const int i = tq0 + r;               // query index of this row
+    const int row_lo = p.wl < 0 ? 0 : i - p.wl;
+    const int row_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, i + p.wr);
+    const int first = tq0, last = tq0 + trows - 1;
+    const int full_lo = p.wl < 0 ? 0 : last - p.wl;               // block start bound
+    const int full_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, first + p.wr);
+    const float sl2 = p.scale_log2;
+
+    float m_use = -INFINITY;   // running max (log2 units of scaled scores)
+    float l = 0.0f;            // running normaliser, relative to m_use
+    bool ok = true;
+
+    if (trows > 0) {
+      for (int n = 0; n < n_blocks; ++n) {
+        const int j = tlo + n;
+        ok = mbar_wait_warp(smem_u32(&bars->s_full[t]), n & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after_sync();
+
+        uint32_t sr[4][32];
+        tmem_ld_x32(tS + 0, sr[0]);
+        tmem_ld_x32(tS + 32, sr[1]);
+        tmem_ld_x32(tS + 64, sr[2]);
+        tmem_ld_x32(tS + 96, sr[3]);
+        tmem_wait_ld();
+        reg_dep(sr[0]);
+        reg_dep(sr[1]);
+        reg_dep(sr[2]);
+        reg_dep(sr[3]);
+        float s[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+
+        const bool full = (j * kBN >= full_lo) && (j * kBN + kBN - 1 <= full_hi);
+        if (!full) {
+          const int lo_c = row_lo - j * kBN;
+          const int hi_c = row_hi - j * kBN;
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c < lo_c || c > hi_c) s[c] = -INFINITY;
+        }
+        // row max of this block
+        float mx[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = s[u];
+#pragma unroll
+        for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
+        float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
+
+        // conditional rescale: only when some row's max grew by > 2^8
+        const bool need = m_new > m_use + kRescaleThreshold;
+        float alpha = 1.0f;
+        const bool warp_rescale = __any_sync(0xffffffffu, need);
+        if (warp_rescale) {
+          const float m_upd = fmaxf(m_use, m_new);
+          alpha = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
+          m_use = m_upd;
+          l *= alpha;
+        }
+        const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
+
+        // P = 2^(s*scale*log2e - m), packed two per 32-bit TMEM column
+        // P overwrites S columns [0, 64): all of S is already in registers.
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < kBN / 2; c += 2) {
+            const float p0 = ex2(fmaf(s[half * 64 + c], sl2, -m_sub));
+            const float p1 = ex2(fmaf(s[half * 64 + c + 1], sl2, -m_sub));
+            ls[(c >> 1) & 3] += p0 + p1;
+            pk[c >> 1] = pack2<DT>(p0, p1);
+          }
+          tmem_st_x32(tS + half * 32, pk);
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+
+        if (warp_rescale && n > 0) {
+          // O_t was completed up to block j-1 (PV_t(j-1) finished before
+          // S_t(j) was issued); scale it by alpha row by row.
+          if constexpr (D >= 32) {
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              tmem_ld_x32(tO + c, o);
+              tmem_wait_ld();
+              reg_dep(o);
+#pragma unroll
+              for (int u = 0; u < 32; ++u)
+                o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+              tmem_st_x32(tO + c, o);
+            }
+          } else {
+            uint32_t o[16];
+            tmem_ld_x16(tO, o);
+            tmem_wait_ld();
+            reg_dep(o);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+            tmem_st_x16(tO, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(smem_u32(&bars->p_full[t]));
+      }
+
+      // ---------------------------------------------- epilogue: O / l, lse
+      if (ok && n_blocks > 0) {
+        ok = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n_blocks - 1) & 1, abort_flag);
+        if (ok) tc_fence_after_sync();
+      }
+      const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+      uint8_t *stage = smem + G::kOffQ + t * G::kTileBytes;   // Q_t is free now
+      const int sw = ((r * G::kSwBytes) >> 7) & (G::kUnitsPerBoxRow - 1);
+      auto put_units = [&](int c0, const uint32_t *w, int nunits) {
+        // c0: first column of this chunk; w: packed pairs, 4 words per unit
+#pragma unroll
+        for (int u = 0; u < nunits; ++u) {
+          const int unit = (c0 * 2) / 16 + u;
+          const int box = unit / G::kUnitsPerBoxRow;
+          const int cc = unit % G::kUnitsPerBoxRow;
+          uint4 *dst = reinterpret_cast<uint4 *>(stage + box * G::kBoxBytes + r * G::kSwBytes +
+                                                 ((cc ^ sw) << 4));
+          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      };
+      if (ok) {
+        if constexpr (D >= 32) {
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            if (n_blocks > 0) {
+              tmem_ld_x32(tO + c, o);
+              tmem_wait_ld();
+              reg_dep(o);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) o[u] = 0u;
+            }
+            uint32_t w[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+              w[u] = pack2<DT>(__uint_as_float(o[2 * u]) * inv_l,
+                               __uint_as_float(o[2 * u + 1]) * inv_l);
+            put_units(c, w, 4);
+          }
+        } else {
+          uint32_t o[16];
+          if (n_blocks > 0) {
+            tmem_ld_x16(tO, o);
+            tmem_wait_ld();
+            reg_dep(o);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) o[u] = 0u;
+          }
+          uint32_t w[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            w[u] = pack2<DT>(__uint_as_float(o[2 * u]) * inv_l,
+                             __uint_as_float(o[2 * u + 1]) * inv_l);
+          put_units(0, w, 2);
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1 + t, kBM);
+      if (r == 0 && !*abort_flag) {
+        for (int bx = 0; bx < G::kNumBox; ++bx)
+          tma_store_3d(&p.tm_o, smem_u32(stage + bx * G::kBoxBytes), bx * G::kBoxCols, tq0,
+                       bh);
+        bulk_commit_group();
+        bulk_wait_group_all();
+      }
+      if (ok && p.lse != nullptr && r < trows) {
+        const float lse = l > 0.0f ? (m_use + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+        p.lse[static_cast<size_t>(bh) * p.L_q + i] = lse;
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after_sync();
+    mbar_wait_slow(smem_u32(&bars->mma_done), 0, abort_flag, false);
+    __syncwarp();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace fa

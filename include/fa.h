@@ -1,0 +1,107 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention forward library
+ *         (libfa.so).
+ *
+ * The operation: O = softmax(scale * Q K^T + mask) V for every (batch, head),
+ * computed tile by tile with the online softmax, never writing the L_q x L_k
+ * score matrix to memory, plus the per-row log-sum-exp of the scaled, masked
+ * scores.
+ *   - formulas: "PyTorch Transformer Flash Attention机制" section 1;
+ *     "FlashAttention算法原理与性能优化实战" section 1.1;
+ *   - online softmax: "Flash Attention是怎么做到又快又省显存的？" (Online
+ *     normalizer derivation) and "FlashAttention算法原理与性能优化实战"
+ *     section 1.2.2;
+ *   - operator statement (4-D [B,H,S,D] inputs, output shaped like the query,
+ *     fp32 softmax statistics of shape [B,H,S], scale_value, pre_tokens /
+ *     next_tokens window): "FlashAttention算法原理与性能优化实战" section 2.2;
+ *   - logsumexp kept for the backward pass: Triton FA2 walkthrough;
+ *   - MQA/GQA and the causal mask: "FlashAttention算法原理与性能优化实战"
+ *     section 1.3.
+ *
+ * All functions return 0 (FA_OK) or a negative fa_status; none aborts.
+ * Every pointer argument marked "device" must point to memory the current
+ * CUDA device can read/write; the library allocates no memory and keeps no
+ * state between calls other than one device-side status word.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_F16 = 0,  /* IEEE binary16 */
+    FA_BF16 = 1  /* bfloat16 */
+} fa_dtype;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,     /* q, k, v or out is NULL */
+    FA_ERR_SHAPE = -2,    /* B, H, H_kv < 1; L_q, L_k < 0; H % H_kv != 0;
+                             or a size whose byte extent overflows */
+    FA_ERR_HEADDIM = -3,  /* D not in {16, 32, 64, 128} */
+    FA_ERR_DTYPE = -4,    /* dtype not FA_F16 / FA_BF16 */
+    FA_ERR_ALIGN = -5,    /* q, k, v, out not 16-byte aligned, or lse not
+                             4-byte aligned */
+    FA_ERR_ARG = -6,      /* scale is negative, NaN or infinite */
+    FA_ERR_CUDA = -7,     /* a CUDA runtime/driver call failed (launch,
+                             tensor-map encoding, device query) */
+    FA_ERR_TIMEOUT = -8   /* a device-side wait gave up (watchdog); the
+                             outputs of that launch are not valid */
+} fa_status;
+
+/*
+ * fa_fwd -- exact attention forward on `stream` (asynchronous).
+ *
+ *   q     device, [B, H,    L_q, D] contiguous, element type `dtype`
+ *   k, v  device, [B, H_kv, L_k, D] contiguous, element type `dtype`
+ *   out   device, [B, H,    L_q, D] contiguous, element type `dtype`
+ *         (written; RNE rounding of the fp32 result)
+ *   lse   device, [B, H, L_q] contiguous fp32, or NULL to skip it.
+ *         lse = ln(sum_j exp(scale * q_i . k_j)) over the visible keys j;
+ *         -inf for a row with no visible key (whose out row is 0).
+ *   scale finite, >= 0 (the pages use 1/sqrt(D); this ABI has no default).
+ *   causal, window_left, window_right:
+ *         key j is visible from query i iff j < L_k and
+ *         (window_left  < 0 or j >= i - window_left) and
+ *         (window_right < 0 or j <= i + window_right) and
+ *         (causal == 0 or j <= i).  Indices are raw positions (row i of Q
+ *         and row j of K), so causal == 1 equals window_right = 0.
+ *         A negative window means unbounded (the pages' INT_MAX default).
+ *   GQA / MQA: query head h reads key/value head h / (H / H_kv).
+ *   L_q == 0 is a no-op; L_k == 0 writes out = 0 and lse = -inf.
+ *
+ * Buffers are owned by the caller and must not overlap out/lse with inputs.
+ * The call only enqueues work: argument errors are returned before anything
+ * is enqueued; device-side watchdog errors are reported by
+ * fa_get_device_status().
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+           int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+           int causal, int window_left, int window_right, int dtype,
+           cudaStream_t stream);
+
+/*
+ * fa_get_device_status -- synchronise `stream`, then read and clear the
+ * device status word that the kernels set when a bounded wait gives up.
+ * Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA if the synchronisation or
+ * the read failed.
+ */
+int fa_get_device_status(cudaStream_t stream);
+
+/* fa_status_string -- a static, human-readable name for a status code. */
+const char *fa_status_string(int status);
+
+/*
+ * fa_version -- library version as major*10000 + minor*100 + patch.
+ */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

@@ -1,0 +1,100 @@
+"""Shared helpers for the GPU-vs-oracle parity tests.
+
+Gate (from the target tolerances, widened by the output rounding the target
+cannot avoid): |O_gpu - O_oracle| <= 3e-3 + ulp_dtype(O_oracle)/2 element by
+element, |lse_gpu - lse_oracle| <= 1e-3, and -inf lse exactly where the
+oracle has it.  The half-ulp term is the RNE rounding of the fp32 result to
+fp16/bf16: bf16's half ulp is 3.9e-3 for |O| in [1, 2)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from exact_attention_113_b200.inputs import BF16, F16, Workload, make_qkv, to_bits
+
+O_TOL = 3e-3
+LSE_TOL = 1e-3
+
+
+def half_ulp(x: np.ndarray, dtype: int) -> np.ndarray:
+    mbits, emin = (10, -14) if dtype == F16 else (7, -126)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, emin)
+    return 0.5 * np.exp2(e - mbits)
+
+
+def compare(out_gpu: np.ndarray, lse_gpu: np.ndarray | None, out_ref: np.ndarray,
+            lse_ref: np.ndarray | None, dtype: int, where: str = "") -> dict:
+    """Assert the gate; return max errors for reporting."""
+    out_gpu = np.asarray(out_gpu, dtype=np.float64)
+    assert out_gpu.shape == out_ref.shape, (out_gpu.shape, out_ref.shape)
+    assert np.all(np.isfinite(out_gpu)), f"{where}: non-finite output"
+    err = np.abs(out_gpu - out_ref)
+    bound = O_TOL + half_ulp(out_ref, dtype)
+    bad = err > bound
+    stats = {"o_max_abs": float(err.max(initial=0.0)),
+             "o_worst_excess": float((err - bound).max(initial=-1.0))}
+    assert not bad.any(), (f"{where}: {int(bad.sum())} outputs beyond tolerance; "
+                           f"max err {err.max():.3g} at {np.unravel_index(err.argmax(), err.shape)}")
+    if lse_ref is not None:
+        lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+        inf_ref = np.isneginf(lse_ref)
+        assert np.array_equal(np.isneginf(lse_gpu), inf_ref), f"{where}: -inf lse mismatch"
+        fin = ~inf_ref
+        lerr = np.abs(lse_gpu[fin] - lse_ref[fin])
+        stats["lse_max_abs"] = float(lerr.max(initial=0.0))
+        assert np.all(np.isfinite(lse_gpu[fin])), f"{where}: non-finite lse"
+        assert (lerr <= LSE_TOL).all(), f"{where}: lse err {lerr.max():.3g}"
+    return stats
+
+
+def run_gpu(q, k, v, w: Workload, with_lse: bool = True):
+    """Run the CUDA path; outputs pre-filled with NaN so unwritten rows show."""
+    import exact_attention_113_b200 as fa
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.full_like(qd, float("nan"))
+    lse = torch.full((w.B, w.H, w.L_q), float("nan"), dtype=torch.float32,
+                     device="cuda") if with_lse else None
+    fa.flash_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal,
+                 window_left=w.window_left, window_right=w.window_right,
+                 return_lse=with_lse, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0, "device watchdog fired"
+    return out, lse
+
+
+def check_full(w: Workload, with_lse: bool = True) -> dict:
+    """Every row against the oracle."""
+    q, k, v = make_qkv(w)
+    out, lse = run_gpu(q, k, v, w, with_lse)
+    ref, ref_lse = oracle.attention(to_bits(q), to_bits(k), to_bits(v), w.dtype,
+                                    w.softmax_scale, w.causal, w.window_left,
+                                    w.window_right)
+    return compare(out.float().cpu().numpy(), lse.cpu().numpy() if with_lse else None,
+                   ref, ref_lse if with_lse else None, w.dtype, w.name)
+
+
+_cache = {}
+
+
+def cached_qkv(w: Workload):
+    """make_qkv with a one-entry cache: variants of one shape share inputs."""
+    key = (w.B, w.H, w.H_kv, w.L_q, w.L_k, w.D, w.dtype, w.std, w.seed)
+    if key not in _cache:
+        _cache.clear()
+        _cache[key] = make_qkv(w)
+    return _cache[key]
+
+
+def check_rows(w: Workload, rows: np.ndarray, inputs=None) -> dict:
+    """Sampled rows (flattened ids (b*H+h)*L_q+i) against the oracle."""
+    q, k, v = inputs if inputs is not None else cached_qkv(w)
+    out, lse = run_gpu(q, k, v, w, True)
+    ref, ref_lse, _ = oracle.attention_rows(to_bits(q), to_bits(k), to_bits(v), w.dtype,
+                                            w.softmax_scale, w.causal, w.window_left,
+                                            w.window_right, rows=rows)
+    o = out.reshape(-1, w.D)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    lz = lse.reshape(-1)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    return compare(o, lz, ref, ref_lse, w.dtype, w.name)

@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI (CPU only: no kernel is launched).
+
+The library must load without a GPU, export every function include/fa.h
+declares, and reject bad arguments with the documented status codes before
+any CUDA call is made."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import exact_attention_113_b200 as fa
+from exact_attention_113_b200 import binding
+from exact_attention_113_b200.build import build, LIB_PATH
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return fa.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    assert _declared() == sorted(binding.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)$", out, re.M))
+    assert set(_declared()) <= exported
+
+
+def test_status_strings_and_version(lib):
+    assert fa.fa_version() >= 10000
+    for code, name in binding.STATUS.items():
+        assert fa.status_string(code).startswith(name)
+    assert fa.status_string(12345) == "unknown fa status"
+
+
+GOOD = dict(q=16, k=16, v=16, out=16, lse=0, B=1, H=4, H_kv=2, L_q=8, L_k=8, D=64,
+            scale=0.125, causal=0, wl=-1, wr=-1, dtype=0)
+
+
+def _call(**kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"], a["H_kv"],
+                     a["L_q"], a["L_k"], a["D"], a["scale"], a["causal"], a["wl"], a["wr"],
+                     a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(k=0), -1), (dict(v=0), -1), (dict(out=0), -1),
+    (dict(B=0), -2), (dict(H=0), -2), (dict(H_kv=0), -2), (dict(H=4, H_kv=3), -2),
+    (dict(L_q=-1), -2), (dict(L_k=-5), -2), (dict(L_q=(1 << 30) + 1), -2),
+    (dict(B=1 << 16, H=1 << 15, L_q=1 << 10), -2),
+    (dict(D=0), -3), (dict(D=48), -3), (dict(D=96), -3), (dict(D=256), -3),
+    (dict(dtype=2), -4), (dict(dtype=-1), -4),
+    (dict(q=24), -5), (dict(out=8), -5), (dict(v=4), -5), (dict(lse=2), -5),
+    (dict(scale=-0.5), -6), (dict(scale=float("nan")), -6), (dict(scale=float("inf")), -6),
+])
+def test_argument_errors(lib, kw, code):
+    assert _call(**kw) == code
+
+
+def test_empty_query_is_a_no_op(lib):
+    # L_q == 0 returns before touching the device (pointers are never read)
+    assert _call(L_q=0) == 0
+
+
+def test_flash_fwd_rejects_bad_tensors(lib):
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        fa.flash_fwd(q, q, q)                       # CPU tensors
+    with pytest.raises(ValueError):
+        fa.flash_fwd(q[0], q, q)                    # not 4-D
+    with pytest.raises(TypeError):
+        fa.flash_fwd(q.float(), q.float(), q.float())
+    with pytest.raises(ValueError):
+        fa.flash_fwd(q, q[:, :, :, :32], q)         # D mismatch
