@@ -1,0 +1,471 @@
+"""Benchmark of the exact attention forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--skip-cpu-baseline] [--skip-e2e]
+
+A step is one forward (one fa_fwd launch) over the whole workload; the
+default workload is the non-causal B=4, H=48, L=8192, D=128 fp16 forward.
+The metric is forward TFLOPS with the pages' convention 4*B*H*L_q*L_k*D
+(halved when causal).  Timing: W untimed warm-up steps, then K steps timed
+with CUDA events on the launching stream, bracketed by a barrier and a
+device synchronise; the slowest rank's time counts.  The inputs (1.2 GB) are
+larger than the 126 MB L2, so no flush is needed between steps.
+
+N > 1 (torchrun, one process per GPU, NCCL for the barrier and the max):
+every rank runs the same-sized problem on its own inputs (weak scaling; the
+path has no exchange step), and the value is all ranks' FLOPs over the
+slowest rank's time.
+
+--impl reference runs the fp64 CPU oracle (the only other implementation
+this path has) on the host cores, over a bounded sample of query rows of the
+same workload per step, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_attention_113_b200 import inputs as W  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (and % of B200 fp16 tensor peak) vs seq len"
+UNIT = "TFLOPS"
+DEFAULT_WORKLOAD = W.ROOFLINE.name
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fa_fwd_roofline_b4h48l8192d128_ncu.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_113_b200", "csrc", f)
+                  for f in ("fa_fwd_kernel.cuh", "sm100.cuh", "fa_api.cu")]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ FLOPs
+def visible_pairs_per_head(w: W.Workload) -> int:
+    """(query, key) pairs that pass the mask in one head."""
+    wr = 0 if w.causal else w.window_right
+    i = np.arange(w.L_q, dtype=np.int64)
+    lo = np.zeros_like(i) if w.window_left < 0 else np.maximum(i - w.window_left, 0)
+    hi = np.full_like(i, w.L_k - 1) if wr < 0 else np.minimum(i + wr, w.L_k - 1)
+    return int(np.clip(hi - lo + 1, 0, None).sum())
+
+
+def metric_flops(w: W.Workload) -> float:
+    """The pages' convention: 4*B*H*L_q*L_k*D, halved when causal."""
+    f = 4.0 * w.B * w.H * w.L_q * w.L_k * w.D
+    return f / 2 if w.causal else f
+
+
+def algorithmic_flops(w: W.Workload) -> float:
+    """Two length-D dot products (4*D FLOP) per visible (query, key) pair."""
+    return 4.0 * w.D * w.B * w.H * visible_pairs_per_head(w)
+
+
+def row_flops(w: W.Workload, rows: np.ndarray) -> float:
+    """Algorithmic FLOPs of the given flattened query rows."""
+    i = rows % w.L_q
+    wr = 0 if w.causal else w.window_right
+    lo = np.zeros_like(i) if w.window_left < 0 else np.maximum(i - w.window_left, 0)
+    hi = np.full_like(i, w.L_k - 1) if wr < 0 else np.minimum(i + wr, w.L_k - 1)
+    return float(4.0 * w.D * np.clip(hi - lo + 1, 0, None).sum())
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def whole_job_value(flops_per_rank_step: float, world: int, steps: int,
+                    max_seconds: float) -> float:
+    """All ranks' FLOPs over the slowest rank's time, in TFLOPS."""
+    return flops_per_rank_step * world * steps / max_seconds / 1e12
+
+
+# ------------------------------------------------------------------ peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel sources as they are now (else None)."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    text = open(PROFILE_SUMMARY).read()
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+# ------------------------------------------------------------------ clocks
+def physical_gpu_index(cuda_index: int) -> int:
+    """nvidia-smi's index of torch's cuda:<cuda_index>."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [t.strip() for t in vis.split(",") if t.strip()]
+        if cuda_index < len(ids) and ids[cuda_index].isdigit():
+            return int(ids[cuda_index])
+    return cuda_index
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=5)
+
+    def summary(self):
+        """Median SM clock and active throttle reasons over the samples that
+        arrived inside the marked (timed) window."""
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        t0, t1 = getattr(self, "t0", -1e30), getattr(self, "t1", 1e30)
+        for ts, line in self.lines:
+            if not t0 <= ts <= t1 + 0.25:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_oracle_sample(w: W.Workload, q, k, v, target_seconds: float, seed: int = 0):
+    """Time the oracle on a seeded sample of query rows sized to about
+    ``target_seconds`` of CPU work.  Returns (TFLOPS, threads, description)."""
+    import oracle
+    from exact_attention_113_b200.inputs import to_bits
+    qb, kb, vb = to_bits(q), to_bits(k), to_bits(v)
+    rng = np.random.default_rng(seed)
+    n_total = w.B * w.H * w.L_q
+    # calibrate on a few rows, then size the sample
+    probe = rng.integers(0, n_total, size=64)
+    t0 = time.perf_counter()
+    oracle.attention_rows(qb, kb, vb, w.dtype, w.softmax_scale, w.causal, w.window_left,
+                          w.window_right, rows=probe)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(n_total, max(64, 64 * target_seconds / dt)))
+    rows = np.sort(rng.choice(n_total, size=n, replace=False))
+    t0 = time.perf_counter()
+    _, _, used = oracle.attention_rows(qb, kb, vb, w.dtype, w.softmax_scale, w.causal,
+                                       w.window_left, w.window_right, rows=rows)
+    dt = time.perf_counter() - t0
+    tflops = row_flops(w, rows) / dt / 1e12
+    desc = (f"{n} of {n_total} query rows ({n / n_total:.3%}), seeded uniform sample, "
+            f"fp64 oracle, {dt:.1f} s")
+    return tflops, used, desc
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w: W.Workload):
+    import torch
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import exact_attention_113_b200 as fa
+
+    # per-rank problem: same shape, its own seed (weak scaling)
+    w_rank = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    q_cpu, k_cpu, v_cpu = W.make_qkv(w_rank)
+    q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.L_q), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
+                     window_left=w.window_left, window_right=w.window_right,
+                     out=out, lse=lse, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device watchdog fired during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(physical_gpu_index(dev.index)) as clk:
+        time.sleep(0.5)                    # let the sampler start
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        clk.mark_start()
+        with torch.cuda.stream(stream):
+            for s in range(args.steps):
+                starts[s].record(stream)
+                step()
+                ends[s].record(stream)
+        torch.cuda.synchronize(dev)
+        clk.mark_end()
+        barrier(world, dev)
+    launch_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_s = starts[0].elapsed_time(ends[-1]) / 1e3
+    if fa.fa_get_device_status(stream.cuda_stream) != 0:
+        raise RuntimeError("device watchdog fired during the timed steps")
+    max_total = max_over_ranks(total_s, world, dev)
+    value = whole_job_value(metric_flops(w), world, args.steps, max_total)
+    avg_launch_s = sum(launch_ms) / len(launch_ms) / 1e3
+
+    # ---- roofline of the (only) kernel
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = algorithmic_flops(w) / avg_launch_s / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": profiled_traffic(),
+                "peak_source": f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)",
+                "algorithmic_flop_per_launch": algorithmic_flops(w),
+                "min_hbm_bytes_per_launch": min_hbm_bytes(w)}
+
+    # ---- end to end through host buffers (pinned), rank-local
+    e2e = None
+    if not args.skip_e2e:
+        hq, hk, hv = (t.pin_memory() for t in (q_cpu, k_cpu, v_cpu))
+        hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        n_e2e = max(3, min(args.steps, 10))
+        with torch.cuda.stream(stream):
+            e2e_step()
+            torch.cuda.synchronize(dev)
+            barrier(world, dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+        e2e = {"value": round(whole_job_value(metric_flops(w), world, n_e2e, e2e_s), 2),
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": n_e2e, "ms_per_step": round(e2e_s / n_e2e * 1e3, 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        tf, cores, desc = cpu_oracle_sample(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
+        cpu = {"value": round(tf, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": desc, "host_nproc": os.cpu_count()}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(max_total / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16" if w.dtype == W.F16 else "bf16",
+        "data": "synthetic (seeded N(0,%g) inputs, per-rank seeds)" % w.std,
+        "config": workload_config(w, world),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "clocks": clk.summary(), "gpu_launches": args.steps,
+        "pct_of_tensor_peak": round(100.0 * value / world / peak, 2),
+        "launch_ms": {"min": round(min(launch_ms), 4), "median": round(statistics.median(launch_ms), 4),
+                      "max": round(max(launch_ms), 4)},
+    }
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def min_hbm_bytes(w: W.Workload) -> int:
+    """Q, K, V read once, O written once (2 B/elem), lse written (4 B/row)."""
+    qo = 2 * w.B * w.H * w.L_q * w.D * 2
+    kv = 2 * w.B * w.H_kv * w.L_k * w.D * 2
+    return qo + kv + 4 * w.B * w.H * w.L_q
+
+
+def workload_config(w: W.Workload, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "L_q": w.L_q,
+            "L_k": w.L_k, "D": w.D, "causal": w.causal, "window_left": w.window_left,
+            "window_right": w.window_right, "scale": w.softmax_scale,
+            "input_dtype": W.DTYPE_NAME[w.dtype], "accumulate": "fp32",
+            "l2": "inputs larger than L2 (no flush between steps)",
+            "parallelism": f"{world} independent replica(s), one per GPU"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, w: W.Workload):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return                       # rank 0 alone runs the CPU oracle
+    q, k, v = W.make_qkv(w)
+    import oracle
+    from exact_attention_113_b200.inputs import to_bits
+    qb, kb, vb = to_bits(q), to_bits(k), to_bits(v)
+    n_total = w.B * w.H * w.L_q
+    rng = np.random.default_rng(1)
+    # size one step to ~target seconds of CPU work from a short calibration
+    probe = rng.integers(0, n_total, size=32)
+    t0 = time.perf_counter()
+    oracle.attention_rows(qb, kb, vb, w.dtype, w.softmax_scale, w.causal, w.window_left,
+                          w.window_right, rows=probe)
+    per_row = max(time.perf_counter() - t0, 1e-6) / 32
+    n = int(max(32, min(n_total, args.ref_step_seconds / per_row)))
+    times, flops, used = [], 0.0, 0
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(n_total, size=n, replace=False))
+        t0 = time.perf_counter()
+        _, _, used = oracle.attention_rows(qb, kb, vb, w.dtype, w.softmax_scale, w.causal,
+                                           w.window_left, w.window_right, rows=rows)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            flops += row_flops(w, rows)
+    total = sum(times)
+    value = flops / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,%g) inputs)" % w.std,
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": used,
+                         "kind": "oracle",
+                         "sample": f"{n} of {n_total} query rows per step, seeded uniform "
+                                   f"samples, fp64 oracle on the host cores"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.ALL))
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU work in the cpu_baseline sample")
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0,
+                    help="CPU work per step of --impl reference")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
+    args.steps = max(1, args.steps)
+    w = W.ALL[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -413,6 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           for (int c = 0; c < kBN / 2; c += 2) {
             const float p0 = ex2(fmaf(s[half * 64 + c], sl2, -m_sub));
             const float p1 = ex2(fmaf(s[half * 64 + c + 1], sl2, -m_sub));
+            // l sums the unrounded fp32 weights: lse = m + ln(l) then keeps
+            // fp32 accuracy whatever the input type
             ls[(c >> 1) & 3] += p0 + p1;
             pk[c >> 1] = pack2<DT>(p0, p1);
           }

@@ -111,4 +111,9 @@ GQA_WINDOW = _c("gqa_window_l16384", B=2, H=32, H_kv=8, L_q=16384, L_k=16384, D=
 ROOFLINE = _c("roofline_b4h48l8192d128", B=4, H=48, H_kv=48, L_q=8192, L_k=8192,
               D=128, dtype=F16, causal=False, seed=1014)
 
-ALL = {w.name: w for w in TINY + [GPT2] + MEMTABLE + SWEEP + [GQA_WINDOW, ROOFLINE]}
+# a smaller case of the roofline kernel for detailed profiles (400 MB of
+# inputs and outputs: larger than L2, a few hundred MB on the device)
+PROFILE = _c("profile_b4h48l2048d128", B=4, H=48, H_kv=48, L_q=2048, L_k=2048, D=128,
+             dtype=F16, causal=False, seed=1015)
+
+ALL = {w.name: w for w in TINY + [GPT2] + MEMTABLE + SWEEP + [GQA_WINDOW, ROOFLINE, PROFILE]}

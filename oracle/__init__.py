@@ -95,7 +95,7 @@ class Oracle:
             fn.restype = None
         lib.oracle_attention_rows.argtypes = [
             u16p, u16p, u16p, ctypes.c_int, i64, i64, i64, i64, i64, i64,
-            ctypes.c_double, ctypes.c_int, i64, i64, i64p, i64, dp, dp,
+            ctypes.c_double, ctypes.c_int, i64, i64, i64p, i64, dp, dp, dp,
             ctypes.c_int]
         lib.oracle_attention_rows.restype = ctypes.c_int
         lib.oracle_attention_rows_online.argtypes = [
@@ -155,9 +155,10 @@ class Oracle:
     # ------------------------------------------------------------- attention
     def attention_rows(self, q, k, v, dtype, scale, causal=False,
                        window_left=-1, window_right=-1, rows=None,
-                       n_threads=0):
+                       n_threads=0, with_wabs=False):
         """Exact attention for flattened row ids r = (b*H + h)*L_q + i
-        (None = every row).  Returns (out [n, D], lse [n], threads_used)."""
+        (None = every row).  Returns (out [n, D], lse [n], threads_used), or
+        (out, lse, threads_used, wabs [n, D]) with ``with_wabs``."""
         q, k, v, B, H, H_kv, L_q, L_k, D = _shape_args(q, k, v)
         if rows is None:
             n, rows_p = B * H * L_q, None
@@ -166,14 +167,18 @@ class Oracle:
             n, rows_p = rows.size, _ptr(rows, ctypes.c_int64)
         out = np.zeros((n, D), dtype=np.float64)
         lse = np.zeros((n,), dtype=np.float64)
+        wabs = np.zeros((n, D), dtype=np.float64) if with_wabs else None
         used = self.lib.oracle_attention_rows(
             _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
             _ptr(v, ctypes.c_uint16), int(dtype), B, H, H_kv, L_q, L_k, D,
             float(scale), int(bool(causal)), int(window_left),
             int(window_right), rows_p, n, _ptr(out, ctypes.c_double),
-            _ptr(lse, ctypes.c_double), int(n_threads))
+            _ptr(lse, ctypes.c_double),
+            _ptr(wabs, ctypes.c_double) if with_wabs else None, int(n_threads))
         if used < 0:
             raise ValueError("oracle rejected the arguments")
+        if with_wabs:
+            return out, lse, used, wabs
         return out, lse, used
 
     def attention(self, q, k, v, dtype, scale, causal=False, window_left=-1,

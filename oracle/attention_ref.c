@@ -184,6 +184,11 @@ static void build_decode_table(int dtype, double *tab)
  *   k, v : [B, H_kv, L_k, D]
  *   rows : flattened row ids r = (b*H + h)*L_q + i, or NULL for all rows
  *   out  : [n_rows, D] fp64;  lse : [n_rows] fp64 (may be NULL)
+ *   wabs : [n_rows, D] fp64 (may be NULL): sum_j p_j |v_j[d]|, the softmax-
+ *          weighted mean magnitude of V.  Not part of the attention result:
+ *          it is the scale of the error that rounding the weights p_j to a
+ *          t-bit format causes in O (at most 2^-t * wabs per element, first
+ *          order), which the parity tests use in their tolerance.
  * Returns the number of threads used, or a negative value on bad input.
  */
 int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
@@ -192,7 +197,7 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
                           double scale, int causal, int64_t window_left,
                           int64_t window_right, const int64_t *rows,
                           int64_t n_rows, double *out, double *lse,
-                          int n_threads)
+                          double *wabs, int n_threads)
 {
     if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1)
         return -1;
@@ -252,6 +257,16 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
             }
             if (lse)
                 lse[t] = (m == -INFINITY) ? -INFINITY : m + log(den);
+            if (wabs) {
+                double *w = wabs + t * D;
+                for (int64_t d = 0; d < D; d++)
+                    w[d] = 0.0;
+                for (int64_t j = 0; j < L_k; j++) {
+                    if (p[j] == 0.0) continue;
+                    for (int64_t d = 0; d < D; d++)
+                        w[d] += p[j] * fabs(tab[vp[j * D + d]]);
+                }
+            }
         }
         free(qrow);
         free(s);

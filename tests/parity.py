@@ -1,10 +1,20 @@
 """Shared helpers for the GPU-vs-oracle parity tests.
 
-Gate (from the target tolerances, widened by the output rounding the target
-cannot avoid): |O_gpu - O_oracle| <= 3e-3 + ulp_dtype(O_oracle)/2 element by
-element, |lse_gpu - lse_oracle| <= 1e-3, and -inf lse exactly where the
-oracle has it.  The half-ulp term is the RNE rounding of the fp32 result to
-fp16/bf16: bf16's half ulp is 3.9e-3 for |O| in [1, 2)."""
+Gate on the named workloads (the target tolerances, widened by the output
+rounding the target cannot avoid): |O_gpu - O_oracle| <= 3e-3 +
+ulp_dtype(O_oracle)/2 element by element, |lse_gpu - lse_oracle| <= 1e-3,
+and -inf lse exactly where the oracle has it.  The half-ulp term is the RNE
+rounding of the fp32 result to fp16/bf16: bf16's half ulp is 3.9e-3 for |O|
+in [1, 2).
+
+Derived gate for the extra edge-case shapes (rows that see a handful of
+keys): the PV product takes P rounded to the input type, so each weight p_j
+carries a relative error up to u = 2^-8 (bf16) or 2^-11 (fp16), while the
+normaliser l sums the unrounded fp32 weights.  That moves O[d] by at most
+u * sum_j w_j |v_j[d]| = u * wabs[d] (wabs from the oracle).  With a row of
+two keys this term alone exceeds 3e-3 for bf16, whatever the implementation,
+so the derived gate adds it, doubled for the second-order terms and the fp32
+rounding of the accumulation: 3e-3 + ulp/2 + 2u * wabs."""
 from __future__ import annotations
 
 import numpy as np
@@ -15,6 +25,7 @@ from exact_attention_113_b200.inputs import BF16, F16, Workload, make_qkv, to_bi
 
 O_TOL = 3e-3
 LSE_TOL = 1e-3
+P_UNIT_ROUNDOFF = {F16: 2.0 ** -11, BF16: 2.0 ** -8}
 
 
 def half_ulp(x: np.ndarray, dtype: int) -> np.ndarray:
@@ -26,13 +37,17 @@ def half_ulp(x: np.ndarray, dtype: int) -> np.ndarray:
 
 
 def compare(out_gpu: np.ndarray, lse_gpu: np.ndarray | None, out_ref: np.ndarray,
-            lse_ref: np.ndarray | None, dtype: int, where: str = "") -> dict:
-    """Assert the gate; return max errors for reporting."""
+            lse_ref: np.ndarray | None, dtype: int, where: str = "",
+            wabs: np.ndarray | None = None) -> dict:
+    """Assert the gate (the derived one when ``wabs`` is given); return max
+    errors for reporting."""
     out_gpu = np.asarray(out_gpu, dtype=np.float64)
     assert out_gpu.shape == out_ref.shape, (out_gpu.shape, out_ref.shape)
     assert np.all(np.isfinite(out_gpu)), f"{where}: non-finite output"
     err = np.abs(out_gpu - out_ref)
     bound = O_TOL + half_ulp(out_ref, dtype)
+    if wabs is not None:
+        bound = bound + 2.0 * P_UNIT_ROUNDOFF[dtype] * wabs.reshape(out_ref.shape)
     bad = err > bound
     stats = {"o_max_abs": float(err.max(initial=0.0)),
              "o_worst_excess": float((err - bound).max(initial=-1.0))}
@@ -65,15 +80,18 @@ def run_gpu(q, k, v, w: Workload, with_lse: bool = True):
     return out, lse
 
 
-def check_full(w: Workload, with_lse: bool = True) -> dict:
-    """Every row against the oracle."""
+def check_full(w: Workload, with_lse: bool = True, derived: bool = False) -> dict:
+    """Every row against the oracle (``derived``: the edge-case gate)."""
     q, k, v = make_qkv(w)
     out, lse = run_gpu(q, k, v, w, with_lse)
-    ref, ref_lse = oracle.attention(to_bits(q), to_bits(k), to_bits(v), w.dtype,
-                                    w.softmax_scale, w.causal, w.window_left,
-                                    w.window_right)
+    ref, ref_lse, _, wabs = oracle.attention_rows(
+        to_bits(q), to_bits(k), to_bits(v), w.dtype, w.softmax_scale, w.causal,
+        w.window_left, w.window_right, with_wabs=True)
+    ref = ref.reshape(w.B, w.H, w.L_q, w.D)
+    ref_lse = ref_lse.reshape(w.B, w.H, w.L_q)
     return compare(out.float().cpu().numpy(), lse.cpu().numpy() if with_lse else None,
-                   ref, ref_lse if with_lse else None, w.dtype, w.name)
+                   ref, ref_lse if with_lse else None, w.dtype, w.name,
+                   wabs if derived else None)
 
 
 _cache = {}

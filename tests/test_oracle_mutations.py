@@ -35,6 +35,8 @@ MUTATIONS = {
                   "v = ldexp((double)(128 + m), e - 133);"),
     "round_half_away": ("double r = nearbyint(ldexp(a, -q_exp));",
                         "double r = round(ldexp(a, -q_exp));"),
+    "wabs_signed": ("w[d] += p[j] * fabs(tab[vp[j * D + d]]);",
+                    "w[d] += p[j] * tab[vp[j * D + d]];"),
     "online_stale_max": ("d = d * exp(m - m_new) + exp(x[i] - m_new);",
                          "d = d + exp(x[i] - m_new);"),
 }
@@ -57,6 +59,7 @@ def _battery(orc):
     yield lambda: pins.test_gqa_equals_mha_with_repeated_heads(orc)
     yield lambda: pins.test_shifting_every_key(orc)
     yield lambda: pins.test_fully_masked_rows(orc)
+    yield lambda: pins.test_weighted_abs_value_closed_forms(orc)
 
 
 def _first_failure(orc):

@@ -171,6 +171,7 @@ def _brute(qf, kf, vf, scale, causal, wl, wr):
     grp = H // H_kv
     out = np.zeros((B, H, L_q, D))
     lse = np.zeros((B, H, L_q))
+    wabs = np.zeros((B, H, L_q, D))
     for b in range(B):
         for h in range(H):
             g = h // grp
@@ -190,8 +191,11 @@ def _brute(qf, kf, vf, scale, causal, wl, wr):
                     out[b, h, i, d] = math.fsum(
                         math.exp(t - m) / den * float(vf[b, g, j, d])
                         for j, t in s)
+                    wabs[b, h, i, d] = math.fsum(
+                        math.exp(t - m) / den * abs(float(vf[b, g, j, d]))
+                        for j, t in s)
                 lse[b, h, i] = m + math.log(den)
-    return out, lse
+    return out, lse, wabs
 
 
 BRUTE_CASES = [
@@ -215,9 +219,12 @@ def test_matches_brute_force(orc, case):
     v = _rand_bits((B, H_kv, L_k, D), dtype, 13)
     scale = 1.0 / math.sqrt(D)
     out, lse = orc.attention(q, k, v, dtype, scale, causal, wl, wr)
-    ro, rl = _brute(_lib_decode(q, dtype), _lib_decode(k, dtype),
-                    _lib_decode(v, dtype), scale, causal, wl, wr)
+    ro, rl, rw = _brute(_lib_decode(q, dtype), _lib_decode(k, dtype),
+                        _lib_decode(v, dtype), scale, causal, wl, wr)
     assert np.allclose(out, ro, rtol=0, atol=1e-12)
+    _, _, _, wabs = orc.attention_rows(q, k, v, dtype, scale, causal, wl, wr,
+                                       with_wabs=True)
+    assert np.allclose(wabs, rw.reshape(wabs.shape), rtol=0, atol=1e-12)
     inf = np.isinf(rl)
     assert np.array_equal(np.isinf(lse), inf)
     assert np.allclose(lse[~inf], rl[~inf], rtol=0, atol=1e-12)
@@ -288,6 +295,21 @@ def test_causal_row_zero_is_v0(orc):
         for h in range(H):
             dot = math.fsum(qf[b, h, 0, d] * kf[b, h, 0, d] for d in range(D))
             assert abs(lse[b, h, 0] - scale * dot) < 1e-13
+
+
+def test_weighted_abs_value_closed_forms(orc):
+    # constant V rows = c  =>  sum_j p_j |c| = |c|;  one key  =>  |v_0|
+    B, H, L, D = 1, 2, 9, 4
+    q = _rand_bits((B, H, L, D), F16, 141)
+    k = _rand_bits((B, H, L, D), F16, 142)
+    row = _rand_bits((D,), F16, 143)
+    v = np.broadcast_to(row, (B, H, L, D)).copy()
+    _, _, _, w = orc.attention_rows(q, k, v, F16, 0.3, True, with_wabs=True)
+    assert np.allclose(w, np.abs(_lib_decode(row, F16)), rtol=1e-14, atol=0)
+    k1, v1 = k[:, :, :1], _rand_bits((B, H, 1, D), F16, 144)
+    _, _, _, w1 = orc.attention_rows(q, k1, v1, F16, 0.3, False, with_wabs=True)
+    assert np.array_equal(w1.reshape(B, H, L, D),
+                          np.broadcast_to(np.abs(_lib_decode(v1, F16)), (B, H, L, D)))
 
 
 def test_single_key_is_v0(orc):

@@ -1,6 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle,
 element by element on the same seeded inputs.  Small and medium workloads are
-compared in full; the full-size workloads on a deterministic row sample."""
+compared in full; the full-size workloads on a deterministic row sample.
+Named workloads use the target gate; the extra edge-case shapes use the
+derived gate of tests/parity.py (P rounded to the input type)."""
 import dataclasses
 import math
 
@@ -46,7 +48,7 @@ EDGE_L = [1, 17, 127, 128, 129, 255, 256, 300, 513]
 @pytest.mark.parametrize("causal", [False, True])
 def test_ragged_lengths(D, L, causal):
     dtype = BF16 if (L + D) % 2 else F16
-    check_full(_w(L_q=L, L_k=L, D=D, dtype=dtype, causal=causal, seed=L * 7 + D))
+    check_full(_w(L_q=L, L_k=L, D=D, dtype=dtype, causal=causal, seed=L * 7 + D), derived=True)
 
 
 @pytest.mark.parametrize("L_q,L_k", [(1, 300), (300, 1), (129, 700), (700, 129),
@@ -54,7 +56,7 @@ def test_ragged_lengths(D, L, causal):
 @pytest.mark.parametrize("causal", [False, True])
 def test_unequal_lengths(L_q, L_k, causal):
     # rows past the last key under causal/top-left alignment are fully masked
-    check_full(_w(L_q=L_q, L_k=L_k, D=64, causal=causal, seed=L_q + 3 * L_k))
+    check_full(_w(L_q=L_q, L_k=L_k, D=64, causal=causal, seed=L_q + 3 * L_k), derived=True)
 
 
 @pytest.mark.parametrize("wl,wr,causal", [(0, -1, True), (1, -1, True), (127, -1, True),
@@ -64,17 +66,18 @@ def test_unequal_lengths(L_q, L_k, causal):
 @pytest.mark.parametrize("D", [32, 128])
 def test_windows(wl, wr, causal, D):
     check_full(_w(B=2, H=2, H_kv=1, L_q=777, L_k=777, D=D, causal=causal, window_left=wl,
-                  window_right=wr, dtype=BF16 if D == 128 else F16, seed=wl + 11 * wr + D))
+                  window_right=wr, dtype=BF16 if D == 128 else F16, seed=wl + 11 * wr + D),
+               derived=True)
 
 
 @pytest.mark.parametrize("H,H_kv", [(8, 1), (8, 2), (6, 3), (4, 4)])
 def test_gqa_mqa(H, H_kv):
-    check_full(_w(B=2, H=H, H_kv=H_kv, L_q=333, L_k=333, D=128, causal=True, seed=H * 10 + H_kv))
+    check_full(_w(B=2, H=H, H_kv=H_kv, L_q=333, L_k=333, D=128, causal=True, seed=H * 10 + H_kv), derived=True)
 
 
 def test_fully_masked_rows_give_zero_and_neg_inf():
     w = _w(L_q=600, L_k=200, D=64, causal=True, window_left=0)
-    stats = check_full(w)
+    stats = check_full(w, derived=True)
     q, k, v = make_qkv(w)
     out, lse = run_gpu(q, k, v, w)
     assert torch.all(out[:, :, 200:] == 0)
