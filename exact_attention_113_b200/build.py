@@ -44,7 +44,7 @@ def is_stale() -> bool:
 
 
 # The attention kernel launches 384 threads and re-splits its registers with
-# setmaxnreg (2 warpgroups x 216 + 1 x 64 <= 384 x 168).  That split is only
+# setmaxnreg (2 warpgroups x 224 + 1 x 56 = 384 x 168).  That split is only
 # valid when every instance is compiled at exactly this many registers.
 LAUNCH_REGS = 168
 KERNEL_TAG = "fa_fwd_kernel"

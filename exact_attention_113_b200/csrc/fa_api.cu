@@ -108,8 +108,9 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
                       int causal, int window_left, int window_right, int dtype,
                       cudaStream_t stream) {
   // ---------------------------------------------------------------- checks
-  if (!q || !k || !v || !out) return FA_ERR_NULL;
   if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
+  // a pointer may be NULL only when its tensor has no elements
+  if ((L_q > 0 && (!q || !out)) || (L_k > 0 && (!k || !v))) return FA_ERR_NULL;
   if (H % H_kv != 0) return FA_ERR_SHAPE;
   if (L_q > kMaxSeq || L_k > kMaxSeq) return FA_ERR_SHAPE;
   if (static_cast<int64_t>(B) * H * ((static_cast<int64_t>(L_q) + 255) / 256) >

@@ -12,13 +12,14 @@
 // CTA layout (384 threads = 3 warpgroups, one CTA per SM):
 //   warps 0-3   softmax warpgroup for query tile 0 (rows q0 .. q0+127)
 //   warps 4-7   softmax warpgroup for query tile 1 (rows q0+128 .. q0+255)
-//   warp  8     MMA issuer (one thread) and TMEM owner
-//   warp  9     TMA producer (one thread)
-//   warps 10-11 idle
+//   warp  8     MMA issuer (one elected thread) and TMEM owner
+//   warp  9     TMA producer of Q and K (one elected thread)
+//   warp  10    TMA producer of V (one elected thread)
+//   warp  11    idle
 // Each softmax thread owns one query row, which is one TMEM lane.
 // Registers: launched at kLaunchRegs per thread; the third warpgroup gives
 // back down to kSmallRegs and the two softmax warpgroups grow to kBigRegs:
-//   2*128*kBigRegs + 128*kSmallRegs <= 384*kLaunchRegs (63488 <= 64512).
+//   2*128*kBigRegs + 128*kSmallRegs <= 384*kLaunchRegs (64512 <= 64512).
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D).  P_t (fp16/bf16, two per 32-bit column) is written over
@@ -31,11 +32,15 @@
 // PV_t(j), which reads P_t from the same TMEM columns; tcgen05 MMAs issued by
 // one thread execute in issue order.
 //
-// Shared memory: Q tile 0, Q tile 1, then a ring of kSlots K/V tiles loaded in
-// the order K_lo, V_lo, K_lo+1, V_lo+1, ...  Tiles are stored as TMA writes
+// Shared memory: Q tile 0, Q tile 1, a ring of kSlotsK K tiles and a ring of
+// kSlotsV V tiles.  K_j is needed half a block before V_j, so K gets the
+// deeper ring; each ring has its own producer warp so that neither waits
+// behind the other's free slot.  Tiles are stored as TMA writes
 // them (rows of `kSwBytes`, swizzled), which is the canonical K-major layout
 // for Q and K and the canonical MN-major layout for V.
 #pragma once
+
+#include <type_traits>
 
 #include "sm100.cuh"
 
@@ -45,12 +50,13 @@ constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kBN = 128;        // keys per K/V block
 constexpr int kThreads = 384;
 constexpr uint32_t kLaunchRegs = 168;   // 65536 / 384, rounded down to 8
-constexpr uint32_t kBigRegs = 216;
-constexpr uint32_t kSmallRegs = 64;
+constexpr uint32_t kBigRegs = 224;
+constexpr uint32_t kSmallRegs = 56;
 static_assert(2 * 128 * kBigRegs + 128 * kSmallRegs <= kThreads * kLaunchRegs,
               "register split must fit in the launch allocation");
 constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kLoadWarp = 9;     // Q and K
+constexpr int kLoadWarpV = 10;   // V
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 
@@ -76,9 +82,15 @@ struct Geo {
   static constexpr int kNumBox = kRowBytes / kSwBytes;                 // column boxes per tile
   static constexpr int kBoxBytes = kBM * kSwBytes;
   static constexpr int kTileBytes = kBM * kRowBytes;
-  static constexpr int kSlots = D == 128 ? 5 : (D == 64 ? 8 : 16);
+  static constexpr int kSlotsK = D == 128 ? 3 : (D == 64 ? 4 : 8);
+  static constexpr int kSlotsV = D == 128 ? 2 : (D == 64 ? 4 : 8);
+  static constexpr int kSlots = kSlotsK + kSlotsV;
   static constexpr uint32_t kLayout = kSwBytes == 128 ? 2u : (kSwBytes == 64 ? 4u : 6u);
   static constexpr int kUnitsPerBoxRow = kSwBytes / 16;
+  // In unmasked blocks one column pair in kPolyPeriod takes 2^x from the FMA
+  // pipe (exp2_poly2) instead of MUFU: the MUFU rate (16/clk/SM) alone needs
+  // as many cycles per block as the D=128 tensor work.
+  static constexpr int kPolyPeriod = 1 << 20;  // (tuned below)
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kTileBytes;
@@ -204,126 +216,156 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   if (warp >= 8) {
   // ===================================================== warpgroup 2
   regs_dec<kSmallRegs>();
-  if (warp == kLoadWarp) {
-    // =================================================== TMA producer
-    if (lane == 0 && any_work) {
+  if (warp == kLoadWarp || warp == kLoadWarpV) {
+    // =================================================== TMA producers
+    // Warp 9 loads Q and the K ring, warp 10 the V ring.  The whole warp
+    // walks the schedule (its operands stay warp-uniform); one elected lane
+    // issues each copy.
+    if (any_work) {
+      const bool is_k = warp == kLoadWarp;
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
+      if (is_k) {
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (rng[t].hi <= rng[t].lo) continue;
-        const uint32_t bar = smem_u32(&bars->q_full[t]);
-        mbar_arrive_expect_tx(bar, G::kTileBytes);
-        for (int bx = 0; bx < G::kNumBox; ++bx)
-          tma_load_3d(sQ + t * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, bar,
-                      bx * G::kBoxCols, q0[t], bh, pol_stream);
-      }
-      int it = 0;
-      bool ok = true;
-      for (int j = lo; j < hi && ok; ++j) {
-        for (int which = 0; which < 2; ++which, ++it) {
-          const int slot = it % kSlots;
-          if (it >= kSlots) {
-            ok = mbar_wait(smem_u32(&bars->empty[slot]), ((it / kSlots) - 1) & 1, abort_flag);
-            if (!ok) break;
+        for (int t = 0; t < 2; ++t) {
+          if (rng[t].hi <= rng[t].lo) continue;
+          const uint32_t bar = smem_u32(&bars->q_full[t]);
+          if (elect_one()) {
+            mbar_arrive_expect_tx(bar, G::kTileBytes);
+#pragma unroll
+            for (int bx = 0; bx < G::kNumBox; ++bx)
+              tma_load_3d(sQ + t * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, bar,
+                          bx * G::kBoxCols, q0[t], bh, pol_stream);
           }
-          const uint32_t bar = smem_u32(&bars->full[slot]);
+          __syncwarp();
+        }
+      }
+      const int nslot = is_k ? G::kSlotsK : G::kSlotsV;
+      const int base = is_k ? 0 : G::kSlotsK;           // first slot of this ring
+      const CUtensorMap *map = is_k ? &p.tm_k : &p.tm_v;
+      int q = 0;
+      bool ok = true;
+      for (int j = lo; j < hi; ++j, ++q) {
+        const int slot = base + q % nslot;
+        if (q >= nslot) {
+          ok = mbar_wait_warp(smem_u32(&bars->empty[slot]), ((q / nslot) - 1) & 1, abort_flag);
+          if (!ok) break;
+        }
+        const uint32_t bar = smem_u32(&bars->full[slot]);
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar, G::kTileBytes);
-          const CUtensorMap *map = which == 0 ? &p.tm_k : &p.tm_v;
+#pragma unroll
           for (int bx = 0; bx < G::kNumBox; ++bx)
             tma_load_3d(sRing + slot * G::kTileBytes + bx * G::kBoxBytes, map, bar,
                         bx * G::kBoxCols, j * kBN, bh_kv, pol_keep);
         }
+        __syncwarp();
       }
       if (!ok) {
         // drain: let the copies already issued land before the CTA exits
-        for (int k = max(0, it - kSlots); k < it; ++k)
-          mbar_wait_slow(smem_u32(&bars->full[k % kSlots]), (k / kSlots) & 1, abort_flag,
+        for (int k = max(0, q - nslot); k < q; ++k)
+          mbar_wait_slow(smem_u32(&bars->full[base + k % nslot]), (k / nslot) & 1, abort_flag,
                          false);
       }
     }
   } else if (warp == kMmaWarp) {
     // =================================================== MMA issuer
-    if (lane == 0 && any_work) {
-      constexpr uint32_t kIdescS = make_idesc_f16(kBM, kBN, DT, 0, 0);
-      constexpr uint32_t kIdescPV = make_idesc_f16(kBM, D, DT, 0, 1);
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+    // The whole warp runs the loop; one elected lane (always the same one,
+    // so that its commits track its own MMAs) issues the tcgen05 ops.
+    constexpr uint32_t kIdescS = make_idesc_f16(kBM, kBN, DT, 0, 0);
+    constexpr uint32_t kIdescPV = make_idesc_f16(kBM, D, DT, 0, 1);
+    constexpr uint32_t kHi = desc_hi(8 * G::kSwBytes, G::kLayout);   // K- and MN-major
+    if (any_work) {
       bool ok = true;
-      if (act0) ok = mbar_wait(smem_u32(&bars->q_full[0]), 0, abort_flag);
-      if (act1 && ok) ok = mbar_wait(smem_u32(&bars->q_full[1]), 0, abort_flag);
-      int npv[2] = {0, 0};
+      if (act0) ok = mbar_wait_warp(smem_u32(&bars->q_full[0]), 0, abort_flag);
+      if (act1 && ok) ok = mbar_wait_warp(smem_u32(&bars->q_full[1]), 0, abort_flag);
+      int npv0 = 0, npv1 = 0;
+      const uint32_t q_lo0 = desc_lo(sQ, 16), q_lo1 = desc_lo(sQ + G::kTileBytes, 16);
 
       auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = sQ + t * G::kTileBytes;
-        const uint32_t ka = sRing + slot * G::kTileBytes;
+        const uint32_t qlo = t ? q_lo1 : q_lo0;
+        const uint32_t klo = desc_lo(sRing + slot * G::kTileBytes, 16);
+        const uint32_t d_tmem = tmem + (t ? 128u : 0u);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int byte = kk * 32;
-          const uint32_t off = (byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes);
-          const uint64_t ad = smem_desc(qa + off, 16, 8 * G::kSwBytes, G::kLayout);
-          const uint64_t bd = smem_desc(ka + off, 16, 8 * G::kSwBytes, G::kLayout);
-          mma_ss(tS[t], ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int byte = kk * 32;
+            const uint32_t off = ((byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes)) >> 4;
+            mma_ss(d_tmem, desc_join(qlo + off, kHi), desc_join(klo + off, kHi), kIdescS,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&bars->s_full[t]));
         }
-        tc_commit(smem_u32(&bars->s_full[t]));
+        __syncwarp();
       };
       auto issue_pv = [&](int t, int slot) {
-        const uint32_t va = sRing + slot * G::kTileBytes;
+        const uint32_t vlo = desc_lo(sRing + slot * G::kTileBytes, G::kBoxBytes);
+        const uint32_t a_tmem = tmem + (t ? 128u : 0u);
+        const uint32_t d_tmem = tmem + 256u + (t ? D : 0u);
+        const bool first = (t ? npv1 : npv0) == 0;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd =
-              smem_desc(va + kk * 16 * G::kSwBytes, G::kBoxBytes, 8 * G::kSwBytes, G::kLayout);
-          mma_ts(tO[t], tS[t] + kk * 8, bd, kIdescPV, (npv[t] > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(d_tmem, a_tmem + kk * 8, desc_join(vlo + ((kk * 16 * G::kSwBytes) >> 4), kHi),
+                   kIdescPV, (!first || kk > 0) ? 1u : 0u);
+          tc_commit(smem_u32(&bars->pv_done[t]));
         }
-        tc_commit(smem_u32(&bars->pv_done[t]));
-        ++npv[t];
+        __syncwarp();
+        if (t) ++npv1; else ++npv0;
+      };
+      auto commit = [&](uint32_t bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
       };
       auto in = [&](int t, int j) { return j >= rng[t].lo && j < rng[t].hi; };
-      auto slot_of = [&](int idx) { return idx % kSlots; };
-      auto par_of = [&](int idx) { return static_cast<uint32_t>((idx / kSlots) & 1); };
+      // ring slots of K_j / V_j (q = j - lo) and the parity of their fill
+      auto kslot = [&](int q) { return q % G::kSlotsK; };
+      auto vslot = [&](int q) { return G::kSlotsK + q % G::kSlotsV; };
+      auto kpar = [&](int q) { return static_cast<uint32_t>((q / G::kSlotsK) & 1); };
+      auto vpar = [&](int q) { return static_cast<uint32_t>((q / G::kSlotsV) & 1); };
 
       for (int j = lo; j < hi && ok; ++j) {
-        const int ik = 2 * (j - lo), iv = ik + 1;
-        ok = mbar_wait(smem_u32(&bars->full[slot_of(ik)]), par_of(ik), abort_flag);
+        const int q = j - lo;
+        ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
-        if (in(0, j)) issue_s(0, slot_of(ik));
+        if (in(0, j)) issue_s(0, kslot(q));
         if (j > lo) {
           if (in(1, j - 1)) {
-            ok = mbar_wait(smem_u32(&bars->full[slot_of(iv - 2)]), par_of(iv - 2), abort_flag) &&
-                 mbar_wait(smem_u32(&bars->p_full[1]), npv[1] & 1, abort_flag);
+            ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q - 1)]), vpar(q - 1),
+                                abort_flag) &&
+                 mbar_wait_warp(smem_u32(&bars->p_full[1]), npv1 & 1, abort_flag);
             if (!ok) break;
             tc_fence_after_sync();
-            issue_pv(1, slot_of(iv - 2));
+            issue_pv(1, vslot(q - 1));
           }
-          tc_commit(smem_u32(&bars->empty[slot_of(iv - 2)]));
+          commit(smem_u32(&bars->empty[vslot(q - 1)]));
         }
-        if (in(1, j)) issue_s(1, slot_of(ik));
-        tc_commit(smem_u32(&bars->empty[slot_of(ik)]));
+        if (in(1, j)) issue_s(1, kslot(q));
+        commit(smem_u32(&bars->empty[kslot(q)]));
         if (in(0, j)) {
-          ok = mbar_wait(smem_u32(&bars->full[slot_of(iv)]), par_of(iv), abort_flag) &&
-               mbar_wait(smem_u32(&bars->p_full[0]), npv[0] & 1, abort_flag);
+          ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q)]), vpar(q), abort_flag) &&
+               mbar_wait_warp(smem_u32(&bars->p_full[0]), npv0 & 1, abort_flag);
           if (!ok) break;
           tc_fence_after_sync();
-          issue_pv(0, slot_of(iv));
+          issue_pv(0, vslot(q));
         }
       }
       if (ok) {
-        const int iv = 2 * (hi - 1 - lo) + 1;
+        const int q = hi - 1 - lo;
         if (in(1, hi - 1)) {
-          ok = mbar_wait(smem_u32(&bars->full[slot_of(iv)]), par_of(iv), abort_flag) &&
-               mbar_wait(smem_u32(&bars->p_full[1]), npv[1] & 1, abort_flag);
+          ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q)]), vpar(q), abort_flag) &&
+               mbar_wait_warp(smem_u32(&bars->p_full[1]), npv1 & 1, abort_flag);
           if (ok) {
             tc_fence_after_sync();
-            issue_pv(1, slot_of(iv));
+            issue_pv(1, vslot(q));
           }
         }
-        tc_commit(smem_u32(&bars->empty[slot_of(iv)]));
+        commit(smem_u32(&bars->empty[vslot(q)]));
       }
-      tc_commit(smem_u32(&bars->mma_done));
-    } else if (lane == 0) {
-      tc_commit(smem_u32(&bars->mma_done));
     }
+    if (elect_one()) tc_commit(smem_u32(&bars->mma_done));
+    __syncwarp();
   }
   } else {
     // =================================================== softmax / epilogue
@@ -357,95 +399,159 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         if (!ok) break;
         tc_fence_after_sync();
 
-        uint32_t sr[4][32];
-        tmem_ld_x32(tS + 0, sr[0]);
-        tmem_ld_x32(tS + 32, sr[1]);
-        tmem_ld_x32(tS + 64, sr[2]);
-        tmem_ld_x32(tS + 96, sr[3]);
-        tmem_wait_ld();
-        reg_dep(sr[0]);
-        reg_dep(sr[1]);
-        reg_dep(sr[2]);
-        reg_dep(sr[3]);
-        float s[kBN];
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
-
         const bool full = (j * kBN >= full_lo) && (j * kBN + kBN - 1 <= full_hi);
-        if (!full) {
-          const int lo_c = row_lo - j * kBN;
-          const int hi_c = row_hi - j * kBN;
+        // S row of this block -> registers (masked entries -> -inf)
+        auto load_s = [&](float (&sv)[kBN]) {
+          uint32_t sr[4][32];
+          tmem_ld_x32(tS + 0, sr[0]);
+          tmem_ld_x32(tS + 32, sr[1]);
+          tmem_ld_x32(tS + 64, sr[2]);
+          tmem_ld_x32(tS + 96, sr[3]);
+          tmem_wait_ld();
+          reg_dep(sr[0]);
+          reg_dep(sr[1]);
+          reg_dep(sr[2]);
+          reg_dep(sr[3]);
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (c < lo_c || c > hi_c) s[c] = -INFINITY;
-        }
-        // row max of this block
-        float mx[8];
+          for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
+          if (!full) {
+            const int lo_c = row_lo - j * kBN;
+            const int hi_c = row_hi - j * kBN;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx[u] = s[u];
-#pragma unroll
-        for (int c = 8; c < kBN; c += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
-        float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
-
-        // conditional rescale: only when some row's max grew by > 2^8
-        const bool need = m_new > m_use + kRescaleThreshold;
-        float alpha = 1.0f;
-        const bool warp_rescale = __any_sync(0xffffffffu, need);
-        if (warp_rescale) {
-          const float m_upd = fmaxf(m_use, m_new);
-          alpha = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
-          m_use = m_upd;
-          l *= alpha;
-        }
-        const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
-
-        // P = 2^(s*scale*log2e - m), packed two per 32-bit TMEM column
-        // P overwrites S columns [0, 64): all of S is already in registers.
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < kBN / 2; c += 2) {
-            const float p0 = ex2(fmaf(s[half * 64 + c], sl2, -m_sub));
-            const float p1 = ex2(fmaf(s[half * 64 + c + 1], sl2, -m_sub));
-            // l sums the unrounded fp32 weights: lse = m + ln(l) then keeps
-            // fp32 accuracy whatever the input type
-            ls[(c >> 1) & 3] += p0 + p1;
-            pk[c >> 1] = pack2<DT>(p0, p1);
+            for (int c = 0; c < kBN; ++c)
+              if (c < lo_c || c > hi_c) sv[c] = -INFINITY;
           }
-          tmem_st_x32(tS + half * 32, pk);
-        }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        };
+        const float2 sl2v = make_float2(sl2, sl2);
 
-        if (warp_rescale && n > 0) {
-          // O_t was completed up to block j-1 (PV_t(j-1) finished before
-          // S_t(j) was issued); scale it by alpha row by row.
-          if constexpr (D >= 32) {
+        // exact pass: the row max first (four chains of 3-input maxima), then
+        // the conditional rescale, then P; used for masked blocks, the first
+        // block of a row, and whenever the speculative pass is dropped
+        auto exact_pass = [&](float (&sv)[kBN]) {
+          // exact pass: the row max first (four chains of 3-input maxima)
+          float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-            for (int c = 0; c < D; c += 32) {
-              uint32_t o[32];
-              tmem_ld_x32(tO + c, o);
+          for (int c = 4; c < kBN - 4; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
+          const float m_blk = fmax3(fmax3(mx[0], mx[1], sv[kBN - 4]),
+                                    fmax3(mx[2], mx[3], sv[kBN - 3]),
+                                    fmaxf(sv[kBN - 2], sv[kBN - 1]));
+          const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
+
+          // conditional rescale: only when some row's max grew by > 2^8
+          const bool need = m_new > m_use + kRescaleThreshold;
+          float alpha = 1.0f;
+          const bool warp_rescale = __any_sync(0xffffffffu, need);
+          if (warp_rescale) {
+            const float m_upd = fmaxf(m_use, m_new);
+            alpha = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
+            m_use = m_upd;
+            l *= alpha;
+          }
+          const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
+
+          // P = 2^(s*scale*log2e - m), packed two per 32-bit TMEM column.
+          // P overwrites S columns [0, 64): all of S is already in registers.
+          const float2 negm = make_float2(-m_sub, -m_sub);
+          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          auto exp_block = [&](auto poly_ok) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t pk[32];
+#pragma unroll
+              for (int c = 0; c < kBN / 2; c += 2) {
+                const float2 x =
+                    __ffma2_rn(make_float2(sv[half * 64 + c], sv[half * 64 + c + 1]), sl2v, negm);
+                const int pair = (half * 64 + c) >> 1;
+                float2 pp;
+                if (decltype(poly_ok)::value && (pair % G::kPolyPeriod) == G::kPolyPeriod - 1)
+                  pp = exp2_poly2(x);
+                else
+                  pp = make_float2(ex2(x.x), ex2(x.y));
+                // l sums the unrounded fp32 weights: lse = m + ln(l) then
+                // keeps fp32 accuracy whatever the input type
+                ls[(c >> 1) & 1] = __fadd2_rn(ls[(c >> 1) & 1], pp);
+                pk[c >> 1] = pack2<DT>(pp.x, pp.y);
+              }
+              tmem_st_x32(tS + half * 32, pk);
+            }
+          };
+          // masked entries are -inf: only MUFU's ex2 turns them into exact 0
+          if (full)
+            exp_block(std::true_type{});
+          else
+            exp_block(std::false_type{});
+          l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+
+          if (warp_rescale && n > 0) {
+            // O_t was completed up to block j-1 (PV_t(j-1) finished before
+            // S_t(j) was issued); scale it by alpha row by row.
+            if constexpr (D >= 32) {
+#pragma unroll
+              for (int c = 0; c < D; c += 32) {
+                uint32_t o[32];
+                tmem_ld_x32(tO + c, o);
+                tmem_wait_ld();
+                reg_dep(o);
+#pragma unroll
+                for (int u = 0; u < 32; ++u)
+                  o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+                tmem_st_x32(tO + c, o);
+              }
+            } else {
+              uint32_t o[16];
+              tmem_ld_x16(tO, o);
               tmem_wait_ld();
               reg_dep(o);
 #pragma unroll
-              for (int u = 0; u < 32; ++u)
+              for (int u = 0; u < 16; ++u)
                 o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-              tmem_st_x32(tO + c, o);
+              tmem_st_x16(tO, o);
             }
-          } else {
-            uint32_t o[16];
-            tmem_ld_x16(tO, o);
-            tmem_wait_ld();
-            reg_dep(o);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-            tmem_st_x16(tO, o);
           }
+        };
+
+        // Speculative pass (unmasked blocks, once every row has a reference
+        // max): P = 2^(s*scale*log2e - m_use) against the current reference
+        // while the block max is reduced alongside, so that the exponentials
+        // do not wait for the max.  If some row's max grew by more than 2^8
+        // the pass is dropped and S, still intact in TMEM (P is stored only
+        // after the check), is reloaded for the exact pass.
+        if (full && __all_sync(0xffffffffu, m_use != -INFINITY)) {
+          float s[kBN];
+          load_s(s);
+          const float2 negm = make_float2(-m_use, -m_use);
+          float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          uint32_t pk[2][32];
+#pragma unroll
+          for (int c = 0; c < kBN; c += 2) {
+            const int pair = c >> 1;
+            mx[pair & 3] = fmax3(mx[pair & 3], s[c], s[c + 1]);
+            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2v, negm);
+            float2 pp;
+            if ((pair % G::kPolyPeriod) == G::kPolyPeriod - 1)
+              pp = exp2_poly2(x);
+            else
+              pp = make_float2(ex2(x.x), ex2(x.y));
+            ls2[pair & 1] = __fadd2_rn(ls2[pair & 1], pp);
+            pk[c >> 6][pair & 31] = pack2<DT>(pp.x, pp.y);
+          }
+          const float m_new = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+          if (__any_sync(0xffffffffu, m_new > m_use + kRescaleThreshold)) {
+            float s2[kBN];
+            load_s(s2);
+            exact_pass(s2);
+          } else {
+            tmem_st_x32(tS + 0, pk[0]);
+            tmem_st_x32(tS + 32, pk[1]);
+            l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
+          }
+        } else {
+          float s[kBN];
+          load_s(s);
+          exact_pass(s);
         }
         tmem_wait_st();
         tc_fence_before_sync();

@@ -93,6 +93,15 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// One lane of a converged warp: the same lane (the lowest active) every time.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
+
 // ------------------------------------------------------------------ registers
 // Warpgroup-wide register budget change (every warp of the warpgroup runs it).
 template <uint32_t N>
@@ -120,6 +129,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2),
       "l"(cache_hint)
       : "memory");
+}
+
+// Prefetch a tile of a 3-D tensor into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 // Tiled 3-D tensor copy shared -> global (bulk-group completion).
@@ -236,6 +253,20 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// The same descriptor split in two words: `desc_lo` holds the start address
+// and the leading byte offset, `desc_hi` the stride byte offset, version and
+// swizzle.  Moving the start by a multiple of 16 bytes adds to the low word
+// (the address field cannot overflow: shared memory is below 256 KB).
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo_bytes, uint32_t layout) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((layout & 7u) << 29);
+}
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 // ab_type: 0 = fp16, 1 = bf16.  a_mn / b_mn: 1 = MN-major operand.
 __host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, int ab_type, int a_mn,
@@ -316,10 +347,42 @@ __device__ __forceinline__ void reg_dep(uint32_t (&r)[N]) {
 }
 
 // ------------------------------------------------------------------ math
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for two finite inputs on the FMA pipe instead of the MUFU unit.
+// Cody-Waite style range reduction: x = n + f with n = round(x), |f| <= 1/2;
+// 2^f from a degree-3 polynomial whose coefficients were fitted for this code
+// by iterated weighted least squares to the minimax relative error on
+// [-1/2, 1/2] (max relative error 7.5e-5 in fp32 Horner evaluation); 2^n is
+// added into the exponent field.  Inputs are clamped to >= -125 so that the
+// result stays a normal float (then 2^-125 stands for anything smaller).
+// The rounding of x + 1.5*2^23 to an integer uses the fp32 add's
+// round-to-nearest; the integer then sits in the low mantissa bits of t.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  constexpr float kC0 = 0.9999281168f, kC1 = 0.6932609677f, kC2 = 0.2426108569f,
+                  kC3 = 0.0551714599f;
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 template <int DT>

@@ -39,7 +39,8 @@ typedef enum {
 
 typedef enum {
     FA_OK = 0,
-    FA_ERR_NULL = -1,     /* q, k, v or out is NULL */
+    FA_ERR_NULL = -1,     /* q or out is NULL while L_q > 0, or k or v is
+                             NULL while L_k > 0 */
     FA_ERR_SHAPE = -2,    /* B, H, H_kv < 1; L_q, L_k < 0; H % H_kv != 0;
                              or a size whose byte extent overflows */
     FA_ERR_HEADDIM = -3,  /* D not in {16, 32, 64, 128} */
@@ -72,7 +73,8 @@ typedef enum {
  *         and row j of K), so causal == 1 equals window_right = 0.
  *         A negative window means unbounded (the pages' INT_MAX default).
  *   GQA / MQA: query head h reads key/value head h / (H / H_kv).
- *   L_q == 0 is a no-op; L_k == 0 writes out = 0 and lse = -inf.
+ *   L_q == 0 is a no-op; L_k == 0 writes out = 0 and lse = -inf.  A
+ *   pointer to a tensor with no elements may be NULL.
  *
  * Buffers are owned by the caller and must not overlap out/lse with inputs.
  * The call only enqueues work: argument errors are returned before anything

@@ -77,6 +77,9 @@ def test_argument_errors(lib, kw, code):
 def test_empty_query_is_a_no_op(lib):
     # L_q == 0 returns before touching the device (pointers are never read)
     assert _call(L_q=0) == 0
+    # tensors with no elements may have NULL pointers
+    assert _call(L_q=0, q=0, out=0) == 0
+    assert _call(L_q=0, q=0, out=0, L_k=0, k=0, v=0) == 0
 
 
 def test_flash_fwd_rejects_bad_tensors(lib):
