@@ -113,9 +113,9 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
   if ((L_q > 0 && (!q || !out)) || (L_k > 0 && (!k || !v))) return FA_ERR_NULL;
   if (H % H_kv != 0) return FA_ERR_SHAPE;
   if (L_q > kMaxSeq || L_k > kMaxSeq) return FA_ERR_SHAPE;
-  if (static_cast<int64_t>(B) * H * ((static_cast<int64_t>(L_q) + 255) / 256) >
+  if (static_cast<int64_t>(B) * H * ((static_cast<int64_t>(L_q) + 127) / 128) >
       (1ll << 31) - 1)
-    return FA_ERR_SHAPE;                   // one CTA per (head, 256 query rows)
+    return FA_ERR_SHAPE;                   // at most one CTA per (head, 128 query rows)
   if (D != 16 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
@@ -151,7 +151,18 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
   prm.L_q = L_q;
   prm.L_k = L_k;
   prm.group = H / H_kv;
-  prm.n_qpairs = (L_q + 2 * kBM - 1) / (2 * kBM);
+  // Two query tiles per CTA keep the tensor pipe busy (ping-pong); when that
+  // leaves SMs idle (few heads, short sequences), one tile per CTA doubles
+  // the number of CTAs.
+  {
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t tiles_total = static_cast<int64_t>(B) * H * ((L_q + kBM - 1) / kBM);
+    prm.tiles = (tiles_total <= static_cast<int64_t>(sms)) ? 1 : 2;
+  }
+  prm.n_qpairs = (L_q + prm.tiles * kBM - 1) / (prm.tiles * kBM);
   prm.wl = wl;
   prm.wr = wr;
   prm.reverse = (wr >= 0) ? 1 : 0;         // later query tiles see more keys

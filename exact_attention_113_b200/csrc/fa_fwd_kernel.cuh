@@ -22,15 +22,23 @@
 //   2*128*kBigRegs + 128*kSmallRegs <= 384*kLaunchRegs (64512 <= 64512).
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
-// O1 [256+D, 256+2D).  P_t (fp16/bf16, two per 32-bit column) is written over
-// the first 64 columns of S_t and read by the PV MMA straight from TMEM.
+// O1 [256+D, 256+2D).  P_t (fp16/bf16, two per 32-bit column) is read by the
+// PV MMA straight from TMEM.
 //
-// MMA issue order per K/V block j (the ping-pong of the two query tiles):
+// D = 128 (TMEM full): P_t is written over the first 64 columns of S_t, and
+// the two query tiles ping-pong.  MMA issue order per K/V block j:
 //   S0(j), PV1(j-1), S1(j), PV0(j)
 // so that while softmax warpgroup 0 works on S0(j), the tensor pipe runs
 // PV1(j-1) and S1(j), and the other way round.  S_t(j+1) is issued after
 // PV_t(j), which reads P_t from the same TMEM columns; tcgen05 MMAs issued by
 // one thread execute in issue order.
+//
+// D <= 64 (room to spare): P_t has its own columns [384 + 64t, 448 + 64t).
+// The softmax frees S_t as soon as it holds the row in registers and its
+// maximum (barrier s_free), so S_t(j+1) is computed while block j's
+// exponentials run, and both tiles' softmax warps run at the same time (two
+// warps per SM sub-partition on its exp unit).  Issue order per block j:
+//   S0(j), S1(j), PV0(j-1), PV1(j-1).
 //
 // Shared memory: Q tile 0, Q tile 1, a ring of kSlotsK K tiles and a ring of
 // kSlotsV V tiles.  K_j is needed half a block before V_j, so K gets the
@@ -68,7 +76,8 @@ struct FwdParams {
   float *lse;         // [B*H, L_q] or nullptr
   int H, H_kv, L_q, L_k;
   int group;          // H / H_kv
-  int n_qpairs;       // ceil(L_q / 256)
+  int n_qpairs;       // query-tile groups per head: ceil(L_q / (128 * tiles))
+  int tiles;          // query tiles per CTA: 2 (ping-pong) or 1 (small problems)
   int wl, wr;         // visible iff i - wl <= j <= i + wr; -1 = unbounded
   int reverse;        // process query pairs last-first (causal: heavy first)
   float scale_log2;   // scale * log2(e), clamped to >= 1e-30
@@ -87,6 +96,8 @@ struct Geo {
   static constexpr int kSlots = kSlotsK + kSlotsV;
   static constexpr uint32_t kLayout = kSwBytes == 128 ? 2u : (kSwBytes == 64 ? 4u : 6u);
   static constexpr int kUnitsPerBoxRow = kSwBytes / 16;
+  // P in its own TMEM columns (decoupled from S) when there is room
+  static constexpr bool kSplitP = D <= 64;
   // In unmasked blocks one column pair in kPolyPeriod takes 2^x from the FMA
   // pipe (exp2_poly2) instead of MUFU: the MUFU rate (16/clk/SM) alone needs
   // as many cycles per block as the D=128 tensor work.
@@ -111,6 +122,7 @@ struct Bars {
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t s_full[2];
+  uint64_t s_free[2];    // split-P schedule: softmax holds S_t in registers
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t mma_done;
@@ -165,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   BlockRange rng[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    q0[t] = qpair * 2 * kBM + t * kBM;
-    rows[t] = max(0, min(kBM, p.L_q - q0[t]));
+    q0[t] = (qpair * p.tiles + t) * kBM;
+    rows[t] = t < p.tiles ? max(0, min(kBM, p.L_q - q0[t])) : 0;
     if (rows[t] > 0) {
       rng[t] = tile_block_range(q0[t], q0[t] + rows[t] - 1, p.L_k, p.wl, p.wr);
     } else {
@@ -184,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&bars->q_full[t]), 1);
       mbar_init(smem_u32(&bars->s_full[t]), 1);
+      mbar_init(smem_u32(&bars->s_free[t]), kBM);
       mbar_init(smem_u32(&bars->p_full[t]), kBM);
       mbar_init(smem_u32(&bars->pv_done[t]), 1);
     }
@@ -300,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       };
       auto issue_pv = [&](int t, int slot) {
         const uint32_t vlo = desc_lo(sRing + slot * G::kTileBytes, G::kBoxBytes);
-        const uint32_t a_tmem = tmem + (t ? 128u : 0u);
+        const uint32_t a_tmem = tmem + (G::kSplitP ? 384u + (t ? 64u : 0u) : (t ? 128u : 0u));
         const uint32_t d_tmem = tmem + 256u + (t ? D : 0u);
         const bool first = (t ? npv1 : npv0) == 0;
         if (elect_one()) {
@@ -324,6 +337,48 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       auto kpar = [&](int q) { return static_cast<uint32_t>((q / G::kSlotsK) & 1); };
       auto vpar = [&](int q) { return static_cast<uint32_t>((q / G::kSlotsV) & 1); };
 
+      if constexpr (G::kSplitP) {
+        // S0(j), S1(j), PV0(j-1), PV1(j-1): S_t(j) waits only until the
+        // softmax of tile t holds S_t(j-1) in registers (s_free)
+        int ns0 = 0, ns1 = 0;
+        auto issue_s_free = [&](int t, int slot) -> bool {
+          const int ns = t ? ns1 : ns0;
+          if (ns > 0 &&
+              !mbar_wait_warp(smem_u32(&bars->s_free[t]), (ns - 1) & 1, abort_flag))
+            return false;
+          tc_fence_after_sync();
+          issue_s(t, slot);
+          if (t) ++ns1; else ++ns0;
+          return true;
+        };
+        auto issue_pv_ready = [&](int t, int qv) -> bool {
+          const bool r = mbar_wait_warp(smem_u32(&bars->full[vslot(qv)]), vpar(qv), abort_flag) &&
+                         mbar_wait_warp(smem_u32(&bars->p_full[t]), (t ? npv1 : npv0) & 1,
+                                        abort_flag);
+          if (!r) return false;
+          tc_fence_after_sync();
+          issue_pv(t, vslot(qv));
+          return true;
+        };
+        for (int j = lo; j <= hi && ok; ++j) {
+          const int q = j - lo;
+          if (j < hi) {
+            ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (in(0, j)) ok = issue_s_free(0, kslot(q));
+            if (ok && in(1, j)) ok = issue_s_free(1, kslot(q));
+            if (!ok) break;
+            commit(smem_u32(&bars->empty[kslot(q)]));
+          }
+          if (j > lo) {
+            if (in(0, j - 1)) ok = issue_pv_ready(0, q - 1);
+            if (ok && in(1, j - 1)) ok = issue_pv_ready(1, q - 1);
+            if (!ok) break;
+            commit(smem_u32(&bars->empty[vslot(q - 1)]));
+          }
+        }
+      } else {
       for (int j = lo; j < hi && ok; ++j) {
         const int q = j - lo;
         ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
@@ -363,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
         commit(smem_u32(&bars->empty[vslot(q)]));
       }
+      }   // ping-pong schedule
     }
     if (elect_one()) tc_commit(smem_u32(&bars->mma_done));
     __syncwarp();
@@ -380,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128u;
     const uint32_t tO = tmem + lane_base + 256u + t * D;
+    const uint32_t tPs = tmem + lane_base + 384u + t * 64u;   // split-P: P_t columns
     const int i = tq0 + r;               // query index of this row
     const int row_lo = p.wl < 0 ? 0 : i - p.wl;
     const int row_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, i + p.wr);
@@ -512,6 +569,72 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           }
         };
 
+        if constexpr (G::kSplitP) {
+          // row max first, then free S_t for the next block's S MMA, then P
+          float s[kBN];
+          load_s(s);
+          float mx[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+          for (int c = 4; c < kBN - 4; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], s[c + 2 * u], s[c + 2 * u + 1]);
+          const float m_blk = fmax3(fmax3(mx[0], mx[1], s[kBN - 4]),
+                                    fmax3(mx[2], mx[3], s[kBN - 3]),
+                                    fmaxf(s[kBN - 2], s[kBN - 1]));
+          tc_fence_before_sync();
+          mbar_arrive(smem_u32(&bars->s_free[t]));
+          const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
+          const bool need = m_new > m_use + kRescaleThreshold;
+          float alpha = 1.0f;
+          const bool warp_rescale = __any_sync(0xffffffffu, need);
+          if (warp_rescale) {
+            const float m_upd = fmaxf(m_use, m_new);
+            alpha = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
+            m_use = m_upd;
+            l *= alpha;
+          }
+          const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
+          const float2 negm = make_float2(-m_sub, -m_sub);
+          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          uint32_t pk[2][32];
+#pragma unroll
+          for (int c = 0; c < kBN; c += 2) {
+            const int pair = c >> 1;
+            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2v, negm);
+            float2 pp;
+            if (full && (pair % G::kPolyPeriod) == G::kPolyPeriod - 1)
+              pp = exp2_poly2(x);
+            else
+              pp = make_float2(ex2(x.x), ex2(x.y));
+            ls[pair & 1] = __fadd2_rn(ls[pair & 1], pp);
+            pk[c >> 6][pair & 31] = pack2<DT>(pp.x, pp.y);
+          }
+          l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+          // P_t and O_t are read / written by PV_t(j-1): wait for it
+          if (n > 0) {
+            const bool got = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n - 1) & 1, abort_flag);
+            ok = ok && got;
+            tc_fence_after_sync();
+          }
+          if (ok) {
+            tmem_st_x32(tPs + 0, pk[0]);
+            tmem_st_x32(tPs + 32, pk[1]);
+            if (warp_rescale && n > 0) {
+              constexpr int kChunk = D >= 32 ? 32 : D;
+#pragma unroll
+              for (int c = 0; c < D; c += kChunk) {
+                uint32_t o[kChunk];
+                tmem_ld_cols<kChunk>(tO + c, o);
+                tmem_wait_ld();
+                reg_dep(o);
+#pragma unroll
+                for (int u = 0; u < kChunk; ++u)
+                  o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+                tmem_st_cols<kChunk>(tO + c, o);
+              }
+            }
+          }
+        } else {
         // Speculative pass (unmasked blocks, once every row has a reference
         // max): P = 2^(s*scale*log2e - m_use) against the current reference
         // while the block max is reduced alongside, so that the exponentials
@@ -553,6 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           load_s(s);
           exact_pass(s);
         }
+        }   // ping-pong schedule
         tmem_wait_st();
         tc_fence_before_sync();
         mbar_arrive(smem_u32(&bars->p_full[t]));
