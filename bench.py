@@ -1,7 +1,8 @@
 """Benchmark of the exact attention forward (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--skip-cpu-baseline] [--skip-e2e]
+                    [--workload NAME] [--splits S|auto] [--skip-cpu-baseline]
+                    [--skip-e2e]
 
 A step is one forward (one fa_fwd launch) over the whole workload; the
 default workload is the non-causal B=4, H=48, L=8192, D=128 fp16 forward.
@@ -15,6 +16,11 @@ N > 1 (torchrun, one process per GPU, NCCL for the barrier and the max):
 every rank runs the same-sized problem on its own inputs (weak scaling; the
 path has no exchange step), and the value is all ranks' FLOPs over the
 slowest rank's time.
+
+--splits S (or auto) times fa_fwd_splitkv instead: one split-KV launch plus
+one merge launch per step, for the decoding workloads (a few query rows, a
+long key/value cache), whose roofline is HBM bandwidth rather than the
+tensor pipe.
 
 --impl reference runs the fp64 CPU oracle (the only other implementation
 this path has) on the host cores, over a bounded sample of query rows of the
@@ -272,11 +278,17 @@ def run_ours(args, w: W.Workload):
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.L_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    n_splits = resolve_splits(args.splits, w)
+    ws = None
+    if n_splits:
+        ws = torch.empty(fa.fa_splitkv_workspace_bytes(w.B, w.H, w.L_q, w.D, n_splits),
+                         dtype=torch.uint8, device=dev)
+    launches_per_step = 2 if n_splits else 1
 
     def step():
         fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
                      window_left=w.window_left, window_right=w.window_right,
-                     out=out, lse=lse, stream=stream)
+                     out=out, lse=lse, stream=stream, n_splits=n_splits, workspace=ws)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -311,13 +323,23 @@ def run_ours(args, w: W.Workload):
     # ---- roofline of the (only) kernel
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = algorithmic_flops(w) / avg_launch_s / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": profiled_traffic(),
-                "peak_source": f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)",
-                "algorithmic_flop_per_launch": algorithmic_flops(w),
-                "min_hbm_bytes_per_launch": min_hbm_bytes(w)}
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    if roofline_bound(w, peak, hbm) == "tensor":
+        achieved = algorithmic_flops(w) / avg_launch_s / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "traffic": profiled_traffic() if w.name == W.ROOFLINE.name else None,
+                    "peak_source": f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)"}
+    else:
+        achieved = min_hbm_bytes(w) / avg_launch_s / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                    "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                    "peak_source": f"{peak_kind} HBM copy bandwidth"}
+    roofline.update({"algorithmic_flop_per_launch": algorithmic_flops(w),
+                     "min_hbm_bytes_per_launch": min_hbm_bytes(w)})
+    if n_splits:
+        roofline["timed"] = (f"whole step: split-KV launch ({n_splits} key slices) "
+                             "plus merge launch")
 
     # ---- end to end through host buffers (pinned), rank-local
     e2e = None
@@ -368,16 +390,35 @@ def run_ours(args, w: W.Workload):
         "data": "synthetic (seeded N(0,%g) inputs, per-rank seeds)" % w.std,
         "config": workload_config(w, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "clocks": clk.summary(), "gpu_launches": args.steps,
+        "clocks": clk.summary(), "gpu_launches": args.steps * launches_per_step,
         "pct_of_tensor_peak": round(100.0 * value / world / peak, 2),
         "launch_ms": {"min": round(min(launch_ms), 4), "median": round(statistics.median(launch_ms), 4),
                       "max": round(max(launch_ms), 4)},
     }
+    if n_splits:
+        line["config"]["entry"] = "fa_fwd_splitkv"
+        line["config"]["n_splits"] = n_splits
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def resolve_splits(arg: str, w: W.Workload, sm_count: int = 148) -> int:
+    """--splits: 0 (fa_fwd), an explicit slice count, or auto."""
+    if arg == "auto":
+        from exact_attention_113_b200.binding import choose_splits
+        return choose_splits(w.B, w.H, w.L_q, w.L_k, sm_count)
+    return int(arg)
+
+
+def roofline_bound(w: W.Workload, tflops: float, gbs: float) -> str:
+    """Whichever of the tensor pipe and HBM takes longer for the workload's
+    algorithmic FLOPs and minimum bytes."""
+    t_tensor = algorithmic_flops(w) / (tflops * 1e12)
+    t_hbm = min_hbm_bytes(w) / (gbs * 1e9)
+    return "tensor" if t_tensor >= t_hbm else "hbm"
 
 
 def min_hbm_bytes(w: W.Workload) -> int:
@@ -451,6 +492,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.ALL))
+    ap.add_argument("--splits", default="0",
+                    help="key slices for fa_fwd_splitkv (0: plain fa_fwd; auto)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,

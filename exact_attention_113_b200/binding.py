@@ -21,9 +21,10 @@ FA_OK = 0
 STATUS = {
     0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_SHAPE", -3: "FA_ERR_HEADDIM",
     -4: "FA_ERR_DTYPE", -5: "FA_ERR_ALIGN", -6: "FA_ERR_ARG", -7: "FA_ERR_CUDA",
-    -8: "FA_ERR_TIMEOUT",
+    -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE",
 }
-EXPORTS = ("fa_fwd", "fa_get_device_status", "fa_status_string", "fa_version")
+EXPORTS = ("fa_fwd", "fa_fwd_splitkv", "fa_get_device_status", "fa_splitkv_workspace_bytes",
+           "fa_status_string", "fa_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -53,6 +54,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
                                i, i, i, i, vp]
         lib.fa_fwd.restype = i
+        lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
+                                       i, i, i, i, i, vp, ctypes.c_size_t, vp]
+        lib.fa_fwd_splitkv.restype = i
+        lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_get_device_status.argtypes = [vp]
         lib.fa_get_device_status.restype = i
         lib.fa_status_string.argtypes = [i]
@@ -72,6 +78,29 @@ def fa_fwd(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
                          int(window_right), int(dtype), stream)
 
 
+def fa_fwd_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
+                   window_left, window_right, dtype, n_splits, workspace,
+                   workspace_bytes, stream) -> int:
+    """The split-KV C entry point, unchanged."""
+    return load().fa_fwd_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D,
+                                 float(scale), int(causal), int(window_left),
+                                 int(window_right), int(dtype), int(n_splits),
+                                 workspace, int(workspace_bytes), stream)
+
+
+def fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits) -> int:
+    return int(load().fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits))
+
+
+def choose_splits(B, H, L_q, L_k, sm_count=148) -> int:
+    """Key slices for fa_fwd_splitkv: enough CTAs to fill the GPU about twice,
+    at least two 128-key blocks per slice, at most 64 slices."""
+    tiles = B * H * max(1, -(-L_q // 128))
+    blocks = max(1, -(-L_k // 128))
+    want = max(1, -(-2 * sm_count // tiles))
+    return int(max(1, min(64, want, blocks // 2 if blocks >= 2 else 1)))
+
+
 def fa_get_device_status(stream=None) -> int:
     return load().fa_get_device_status(stream)
 
@@ -86,13 +115,19 @@ def fa_version() -> int:
 
 # ------------------------------------------------------------ torch call
 def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
-              return_lse=True, out=None, lse=None, stream=None):
+              return_lse=True, out=None, lse=None, stream=None, n_splits=0,
+              workspace=None):
     """Exact attention forward on CUDA tensors.
 
     q: [B, H, L_q, D]; k, v: [B, H_kv, L_k, D]; fp16 or bf16, contiguous, on
     one CUDA device.  ``scale`` defaults to 1/sqrt(D).  Returns ``(out, lse)``
     (``lse`` is None unless ``return_lse``).  Launches asynchronously on
     ``stream`` (default: torch's current stream).
+
+    ``n_splits`` > 0 computes the same result through fa_fwd_splitkv with
+    that many key slices ("auto" picks them with ``choose_splits``); the
+    workspace is allocated here with torch unless ``workspace`` (a uint8
+    CUDA tensor, 256-byte aligned) is given.
     """
     import torch
 
@@ -120,11 +155,26 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
         lse = None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    if n_splits == "auto":
+        n_splits = choose_splits(B, H, L_q, L_k,
+                                 torch.cuda.get_device_properties(q.device).multi_processor_count)
     with torch.cuda.device(q.device):
-        st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                    lse.data_ptr() if lse is not None else None,
-                    B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
-                    window_right, dtype, stream.cuda_stream)
+        if not n_splits:
+            st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                        lse.data_ptr() if lse is not None else None,
+                        B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                        window_right, dtype, stream.cuda_stream)
+            where = "fa_fwd"
+        else:
+            need = fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits)
+            if workspace is None:
+                workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+            st = fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr() if lse is not None else None,
+                                B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                                window_right, dtype, n_splits, workspace.data_ptr(),
+                                workspace.numel(), stream.cuda_stream)
+            where = "fa_fwd_splitkv"
     if st != FA_OK:
-        raise FaError(st, "fa_fwd")
+        raise FaError(st, where)
     return out, lse

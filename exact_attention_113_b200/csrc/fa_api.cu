@@ -22,6 +22,7 @@ namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
 constexpr int kMaxSeq = 1 << 30;
+constexpr int kMaxSplits = 64;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -93,20 +94,98 @@ int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
       configured[dev] = true;
     }
   }
-  dim3 grid(static_cast<unsigned>(prm.n_qpairs) * static_cast<unsigned>(B * H), 1, 1);
+  dim3 grid(static_cast<unsigned>(prm.n_qpairs) * static_cast<unsigned>(B * H) *
+                static_cast<unsigned>(prm.n_splits),
+            1, 1);
   kern<<<grid, kThreads, G::kSmemBytes, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
+
+// Split-KV workspace: partial O [n_splits][rows][D] fp32, then (m, l)
+// [n_splits][rows] as float2, starting at a 256-byte boundary.
+size_t ws_o_bytes(int64_t rows, int D, int n_splits) {
+  return static_cast<size_t>(n_splits) * rows * D * sizeof(float);
+}
+size_t ws_ml_offset(int64_t rows, int D, int n_splits) {
+  return (ws_o_bytes(rows, D, n_splits) + 255) & ~static_cast<size_t>(255);
+}
+size_t ws_total_bytes(int64_t rows, int D, int n_splits) {
+  return ws_ml_offset(rows, D, n_splits) + static_cast<size_t>(n_splits) * rows * sizeof(float2);
+}
+
+// Merge the key slices of every row: m = max_s m_s, w_s = 2^(m_s - m),
+// O = sum_s w_s O_s / sum_s w_s l_s, lse = (m + log2 l) ln 2.  One warp per
+// row; the slices' partial sums are exact softmax pieces of the same row
+// (online-softmax merge of "FlashAttention算法原理与性能优化实战" §1.2.2).
+template <int D, int DT>
+__global__ void __launch_bounds__(256) fa_combine_kernel(const float *ws_o, const float2 *ws_ml,
+                                                         void *out, float *lse, int n_splits,
+                                                         long long rows_total) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows_total) return;
+  float m = -INFINITY;
+  for (int sp = 0; sp < n_splits; ++sp) m = fmaxf(m, ws_ml[sp * rows_total + row].x);
+  constexpr int kPer = (D + 31) / 32;   // elements per lane
+  float acc[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) acc[u] = 0.0f;
+  float l = 0.0f;
+  if (m != -INFINITY) {
+    for (int sp = 0; sp < n_splits; ++sp) {
+      const float2 ml = ws_ml[sp * rows_total + row];
+      if (ml.x == -INFINITY) continue;
+      const float w = exp2f(ml.x - m);
+      l += w * ml.y;
+      const float *o = ws_o + (static_cast<size_t>(sp) * rows_total + row) * D;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int d = lane + 32 * u;
+        if (d < D) acc[u] += w * o[d];
+      }
+    }
+  }
+  const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int d = lane + 32 * u;
+    if (d >= D) continue;
+    const float val = acc[u] * inv_l;
+    if constexpr (DT == 0)
+      reinterpret_cast<__half *>(out)[row * D + d] = __float2half_rn(val);
+    else
+      reinterpret_cast<__nv_bfloat16 *>(out)[row * D + d] = __float2bfloat16_rn(val);
+  }
+  if (lse != nullptr && lane == 0)
+    lse[row] = l > 0.0f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+}
+
+template <int D, int DT>
+int launch_combine(const float *ws_o, const float2 *ws_ml, void *out, float *lse, int n_splits,
+                   long long rows_total, cudaStream_t stream) {
+  const unsigned blocks = static_cast<unsigned>((rows_total + 7) / 8);
+  fa_combine_kernel<D, DT><<<blocks, 256, 0, stream>>>(ws_o, ws_ml, out, lse, n_splits,
+                                                       rows_total);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Shared body of fa_fwd and fa_fwd_splitkv (n_splits == 0: plain forward).
+int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+             int H_kv, int L_q, int L_k, int D, float scale, int causal, int window_left,
+             int window_right, int dtype, int n_splits, void *workspace,
+             size_t workspace_bytes, cudaStream_t stream);
 
 }  // namespace
 }  // namespace fa
 
 using namespace fa;
 
-extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
-                      int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
-                      int causal, int window_left, int window_right, int dtype,
-                      cudaStream_t stream) {
+namespace fa {
+namespace {
+int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+             int H_kv, int L_q, int L_k, int D, float scale, int causal, int window_left,
+             int window_right, int dtype, int n_splits, void *workspace,
+             size_t workspace_bytes, cudaStream_t stream) {
   // ---------------------------------------------------------------- checks
   if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
   // a pointer may be NULL only when its tensor has no elements
@@ -122,6 +201,15 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
     return FA_ERR_ALIGN;
   if (lse && !aligned(lse, 4)) return FA_ERR_ALIGN;
   if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+  const int64_t rows_total = static_cast<int64_t>(B) * H * L_q;
+  if (n_splits != 0) {
+    if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
+    if (L_q > 0 && L_k > 0) {
+      if (!workspace) return FA_ERR_NULL;
+      if (!aligned(workspace, 256)) return FA_ERR_ALIGN;
+      if (workspace_bytes < ws_total_bytes(rows_total, D, n_splits)) return FA_ERR_WORKSPACE;
+    }
+  }
 
   // ---------------------------------------------------------------- edges
   if (L_q == 0) return FA_OK;
@@ -170,6 +258,13 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
     float sl2 = scale * 1.4426950408889634f;
     prm.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;
   }
+  prm.n_splits = n_splits > 0 ? n_splits : 1;
+  prm.rows_total = rows_total;
+  if (n_splits > 0) {
+    prm.ws_o = static_cast<float *>(workspace);
+    prm.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) +
+                                           ws_ml_offset(rows_total, D, n_splits));
+  }
   const int box_cols = D * 2 >= 128 ? 64 : D;
   if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
@@ -177,17 +272,55 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
       !encode_map(&prm.tm_o, out, dtype, B * H, L_q, D, box_cols))
     return FA_ERR_CUDA;
 
+  int st = FA_ERR_HEADDIM;
   switch (D * 2 + dtype) {
-    case 32: return launch<16, 0>(prm, B, H, stream);
-    case 33: return launch<16, 1>(prm, B, H, stream);
-    case 64: return launch<32, 0>(prm, B, H, stream);
-    case 65: return launch<32, 1>(prm, B, H, stream);
-    case 128: return launch<64, 0>(prm, B, H, stream);
-    case 129: return launch<64, 1>(prm, B, H, stream);
-    case 256: return launch<128, 0>(prm, B, H, stream);
-    case 257: return launch<128, 1>(prm, B, H, stream);
+    case 32: st = launch<16, 0>(prm, B, H, stream); break;
+    case 33: st = launch<16, 1>(prm, B, H, stream); break;
+    case 64: st = launch<32, 0>(prm, B, H, stream); break;
+    case 65: st = launch<32, 1>(prm, B, H, stream); break;
+    case 128: st = launch<64, 0>(prm, B, H, stream); break;
+    case 129: st = launch<64, 1>(prm, B, H, stream); break;
+    case 256: st = launch<128, 0>(prm, B, H, stream); break;
+    case 257: st = launch<128, 1>(prm, B, H, stream); break;
+  }
+  if (st != FA_OK || n_splits == 0) return st;
+  switch (D * 2 + dtype) {
+    case 32: return launch_combine<16, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 33: return launch_combine<16, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 64: return launch_combine<32, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 65: return launch_combine<32, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 128: return launch_combine<64, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 129: return launch_combine<64, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 256: return launch_combine<128, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 257: return launch_combine<128, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
   }
   return FA_ERR_HEADDIM;
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                      int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                      int causal, int window_left, int window_right, int dtype,
+                      cudaStream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                  window_right, dtype, 0, nullptr, 0, stream);
+}
+
+extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {
+  if (B < 1 || H < 1 || L_q < 0 || n_splits < 1 || n_splits > kMaxSplits) return 0;
+  if (D != 16 && D != 32 && D != 64 && D != 128) return 0;
+  return ws_total_bytes(static_cast<int64_t>(B) * H * L_q, D, n_splits);
+}
+
+extern "C" int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out,
+                              float *lse, int B, int H, int H_kv, int L_q, int L_k, int D,
+                              float scale, int causal, int window_left, int window_right,
+                              int dtype, int n_splits, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
+  return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                  window_right, dtype, n_splits, workspace, workspace_bytes, stream);
 }
 
 extern "C" int fa_get_device_status(cudaStream_t stream) {
@@ -214,6 +347,7 @@ extern "C" const char *fa_status_string(int status) {
     case FA_ERR_ARG: return "FA_ERR_ARG: scale must be finite and >= 0";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait gave up";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace smaller than fa_splitkv_workspace_bytes()";
   }
   return "unknown fa status";
 }

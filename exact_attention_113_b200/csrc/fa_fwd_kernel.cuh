@@ -81,6 +81,13 @@ struct FwdParams {
   int wl, wr;         // visible iff i - wl <= j <= i + wr; -1 = unbounded
   int reverse;        // process query pairs last-first (causal: heavy first)
   float scale_log2;   // scale * log2(e), clamped to >= 1e-30
+  // split-KV mode (ws_o != nullptr): each CTA covers one of n_splits
+  // contiguous slices of the key blocks and writes its unnormalised partial
+  // O (fp32) and (m, l) per row; a combine kernel merges the slices.
+  int n_splits;       // 1 outside split-KV mode
+  long long rows_total;   // B * H * L_q
+  float *ws_o;        // [n_splits][rows_total][D] or nullptr
+  float2 *ws_ml;      // [n_splits][rows_total]: (m in log2 units, l)
 };
 
 template <int D>
@@ -164,10 +171,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work item: (batch*head, pair of query tiles); consecutive CTAs take
-  // consecutive query pairs of one head, so a head's K/V stays hot in L2.
-  const int bh = static_cast<int>(blockIdx.x) / p.n_qpairs;
-  const int qp_idx = static_cast<int>(blockIdx.x) - bh * p.n_qpairs;
+  // ---- work item: (batch*head, pair of query tiles, key slice);
+  // consecutive CTAs take consecutive query pairs of one head, so a head's
+  // K/V stays hot in L2.
+  const int per_bh = p.n_qpairs * p.n_splits;
+  const int bh = static_cast<int>(blockIdx.x) / per_bh;
+  const int rem = static_cast<int>(blockIdx.x) - bh * per_bh;
+  const int qp_idx = rem / p.n_splits;
+  const int split = rem - qp_idx * p.n_splits;
   const int qpair = p.reverse ? (p.n_qpairs - 1 - qp_idx) : qp_idx;
   const int b = bh / p.H;
   const int h = bh - b * p.H;
@@ -184,6 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     } else {
       rng[t].lo = 0;
       rng[t].hi = 0;
+    }
+  }
+  if (p.n_splits > 1) {
+    // this CTA's slice of the union of the tiles' key-block ranges
+    const bool a0 = rng[0].hi > rng[0].lo, a1 = rng[1].hi > rng[1].lo;
+    const int ulo = a0 ? (a1 ? min(rng[0].lo, rng[1].lo) : rng[0].lo) : rng[1].lo;
+    const int uhi = a0 ? (a1 ? max(rng[0].hi, rng[1].hi) : rng[0].hi) : rng[1].hi;
+    const int cs = (uhi - ulo + p.n_splits - 1) / p.n_splits;
+    const int clo = ulo + split * cs, chi = min(uhi, clo + cs);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      rng[t].lo = max(rng[t].lo, clo);
+      rng[t].hi = min(rng[t].hi, chi);
+      if (rng[t].hi <= rng[t].lo) rng[t].lo = rng[t].hi = 0;
     }
   }
   const bool act0 = rng[0].hi > rng[0].lo, act1 = rng[1].hi > rng[1].lo;
@@ -687,6 +712,39 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         ok = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n_blocks - 1) & 1, abort_flag);
         if (ok) tc_fence_after_sync();
       }
+      if (p.ws_o != nullptr) {
+        // split-KV partial: unnormalised O (fp32) and (m, l) of this slice.
+        // tcgen05.ld is warp-collective: every lane loads (ok and n_blocks
+        // are warp-uniform), only the lanes of real rows store.
+        if (ok) {
+          const bool mine = r < trows;
+          const size_t row = static_cast<size_t>(split) * p.rows_total +
+                             static_cast<size_t>(bh) * p.L_q + i;
+          float4 *dst = reinterpret_cast<float4 *>(p.ws_o + row * D);
+          constexpr int kChunk = D >= 32 ? 32 : D;
+#pragma unroll
+          for (int c = 0; c < D; c += kChunk) {
+            uint32_t o[kChunk];
+            if (n_blocks > 0) {
+              tmem_ld_cols<kChunk>(tO + c, o);
+              tmem_wait_ld();
+              reg_dep(o);
+            } else {
+#pragma unroll
+              for (int u = 0; u < kChunk; ++u) o[u] = 0u;
+            }
+            if (mine) {
+#pragma unroll
+              for (int u = 0; u < kChunk / 4; ++u)
+                dst[c / 4 + u] = make_float4(__uint_as_float(o[4 * u]),
+                                             __uint_as_float(o[4 * u + 1]),
+                                             __uint_as_float(o[4 * u + 2]),
+                                             __uint_as_float(o[4 * u + 3]));
+            }
+          }
+          if (mine) p.ws_ml[row] = make_float2(l > 0.0f ? m_use : -INFINITY, l);
+        }
+      } else {
       const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
       uint8_t *stage = smem + G::kOffQ + t * G::kTileBytes;   // Q_t is free now
       const int sw = ((r * G::kSwBytes) >> 7) & (G::kUnitsPerBoxRow - 1);
@@ -753,6 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         const float lse = l > 0.0f ? (m_use + __log2f(l)) * 0.6931471805599453f : -INFINITY;
         p.lse[static_cast<size_t>(bh) * p.L_q + i] = lse;
       }
+      }   // normal epilogue
     }
   }
 

@@ -116,4 +116,17 @@ ROOFLINE = _c("roofline_b4h48l8192d128", B=4, H=48, H_kv=48, L_q=8192, L_k=8192,
 PROFILE = _c("profile_b4h48l2048d128", B=4, H=48, H_kv=48, L_q=2048, L_k=2048, D=128,
              dtype=F16, causal=False, seed=1015)
 
-ALL = {w.name: w for w in TINY + [GPT2] + MEMTABLE + SWEEP + [GQA_WINDOW, ROOFLINE, PROFILE]}
+# decoding: a few query rows against a long key/value cache (split-KV shapes).
+# The speculative case puts its L_q queries at the end of the cache with the
+# window (query i sees keys j <= i + L_k - L_q).
+DECODE = [
+    _c("decode_b8h32kv8_l1_k32768_d128", B=8, H=32, H_kv=8, L_q=1, L_k=32768, D=128,
+       dtype=BF16, seed=1016),
+    _c("decode_b4h32kv32_l1_k16384_d64", B=4, H=32, H_kv=32, L_q=1, L_k=16384, D=64,
+       dtype=F16, seed=1017),
+    _c("decode_b2h16kv4_l16_k65536_d128", B=2, H=16, H_kv=4, L_q=16, L_k=65536, D=128,
+       dtype=BF16, window_right=65536 - 16, seed=1018),
+]
+
+ALL = {w.name: w for w in TINY + [GPT2] + MEMTABLE + SWEEP + DECODE +
+       [GQA_WINDOW, ROOFLINE, PROFILE]}

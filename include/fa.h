@@ -26,6 +26,7 @@
 #ifndef FA_H
 #define FA_H
 
+#include <stddef.h>
 #include <cuda_runtime.h>
 
 #ifdef __cplusplus
@@ -50,8 +51,10 @@ typedef enum {
     FA_ERR_ARG = -6,      /* scale is negative, NaN or infinite */
     FA_ERR_CUDA = -7,     /* a CUDA runtime/driver call failed (launch,
                              tensor-map encoding, device query) */
-    FA_ERR_TIMEOUT = -8   /* a device-side wait gave up (watchdog); the
+    FA_ERR_TIMEOUT = -8,  /* a device-side wait gave up (watchdog); the
                              outputs of that launch are not valid */
+    FA_ERR_WORKSPACE = -9 /* workspace smaller than the size the matching
+                             *_workspace_bytes() call returns */
 } fa_status;
 
 /*
@@ -85,6 +88,35 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
            int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
            int causal, int window_left, int window_right, int dtype,
            cudaStream_t stream);
+
+/*
+ * fa_splitkv_workspace_bytes -- bytes of device workspace fa_fwd_splitkv
+ * needs for these sizes (0 if the sizes are invalid): B*H*L_q*n_splits rows
+ * of a D-wide fp32 partial output plus an (m, l) pair each.
+ */
+size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits);
+
+/*
+ * fa_fwd_splitkv -- the same forward as fa_fwd, computed in n_splits
+ * (1..64) slices of each query tile's key range: one launch writes every
+ * slice's unnormalised output and (running max, normaliser) to `workspace`,
+ * a second launch merges the slices of each row with the online-softmax
+ * rescaling ("FlashAttention算法原理与性能优化实战" §1.2.2).  Meant for
+ * shapes with few query tiles and long key ranges (decoding), where fa_fwd
+ * would leave most SMs idle.  Arguments as fa_fwd, plus
+ *   n_splits         number of key slices, 1..64 (FA_ERR_ARG otherwise)
+ *   workspace        device, 256-byte aligned, caller-owned, at least
+ *                    fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits)
+ *                    bytes (FA_ERR_WORKSPACE if smaller, FA_ERR_NULL if
+ *                    NULL while L_q, L_k > 0); its contents on entry do not
+ *                    matter and are overwritten.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
+                   int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                   int causal, int window_left, int window_right, int dtype,
+                   int n_splits, void *workspace, size_t workspace_bytes,
+                   cudaStream_t stream);
 
 /*
  * fa_get_device_status -- synchronise `stream`, then read and clear the

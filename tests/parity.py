@@ -65,25 +65,33 @@ def compare(out_gpu: np.ndarray, lse_gpu: np.ndarray | None, out_ref: np.ndarray
     return stats
 
 
-def run_gpu(q, k, v, w: Workload, with_lse: bool = True):
-    """Run the CUDA path; outputs pre-filled with NaN so unwritten rows show."""
+def run_gpu(q, k, v, w: Workload, with_lse: bool = True, n_splits=0):
+    """Run the CUDA path; outputs pre-filled with NaN so unwritten rows show.
+    ``n_splits`` > 0 goes through fa_fwd_splitkv with a NaN-filled
+    workspace, so a partial the kernel forgot to write shows too."""
     import exact_attention_113_b200 as fa
     qd, kd, vd = (t.cuda() for t in (q, k, v))
     out = torch.full_like(qd, float("nan"))
     lse = torch.full((w.B, w.H, w.L_q), float("nan"), dtype=torch.float32,
                      device="cuda") if with_lse else None
+    ws = None
+    if n_splits:
+        nbytes = fa.fa_splitkv_workspace_bytes(w.B, w.H, w.L_q, w.D, n_splits)
+        ws = torch.full((max(nbytes, 4) // 4,), float("nan"), dtype=torch.float32,
+                        device="cuda").view(torch.uint8)
     fa.flash_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal,
                  window_left=w.window_left, window_right=w.window_right,
-                 return_lse=with_lse, out=out, lse=lse)
+                 return_lse=with_lse, out=out, lse=lse, n_splits=n_splits, workspace=ws)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0, "device watchdog fired"
     return out, lse
 
 
-def check_full(w: Workload, with_lse: bool = True, derived: bool = False) -> dict:
+def check_full(w: Workload, with_lse: bool = True, derived: bool = False,
+               n_splits=0) -> dict:
     """Every row against the oracle (``derived``: the edge-case gate)."""
     q, k, v = make_qkv(w)
-    out, lse = run_gpu(q, k, v, w, with_lse)
+    out, lse = run_gpu(q, k, v, w, with_lse, n_splits)
     ref, ref_lse, _, wabs = oracle.attention_rows(
         to_bits(q), to_bits(k), to_bits(v), w.dtype, w.softmax_scale, w.causal,
         w.window_left, w.window_right, with_wabs=True)
@@ -106,10 +114,10 @@ def cached_qkv(w: Workload):
     return _cache[key]
 
 
-def check_rows(w: Workload, rows: np.ndarray, inputs=None) -> dict:
+def check_rows(w: Workload, rows: np.ndarray, inputs=None, n_splits=0) -> dict:
     """Sampled rows (flattened ids (b*H+h)*L_q+i) against the oracle."""
     q, k, v = inputs if inputs is not None else cached_qkv(w)
-    out, lse = run_gpu(q, k, v, w, True)
+    out, lse = run_gpu(q, k, v, w, True, n_splits)
     ref, ref_lse, _ = oracle.attention_rows(to_bits(q), to_bits(k), to_bits(v), w.dtype,
                                             w.softmax_scale, w.causal, w.window_left,
                                             w.window_right, rows=rows)

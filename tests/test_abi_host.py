@@ -93,3 +93,41 @@ def test_flash_fwd_rejects_bad_tensors(lib):
         fa.flash_fwd(q.float(), q.float(), q.float())
     with pytest.raises(ValueError):
         fa.flash_fwd(q, q[:, :, :, :32], q)         # D mismatch
+
+
+# ------------------------------------------------------------ split-KV entry
+def _call_split(n_splits=2, ws=256, ws_bytes=None, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    if ws_bytes is None:
+        ws_bytes = fa.fa_splitkv_workspace_bytes(a["B"], a["H"], a["L_q"], a["D"],
+                                                 max(1, min(64, n_splits)))
+    return fa.fa_fwd_splitkv(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"],
+                             a["H_kv"], a["L_q"], a["L_k"], a["D"], a["scale"], a["causal"],
+                             a["wl"], a["wr"], a["dtype"], n_splits, ws, ws_bytes, None)
+
+
+def test_splitkv_workspace_bytes(lib):
+    # B*H*L_q rows of D fp32 per slice, then (m, l) float2 per row and slice
+    rows, D, S = 2 * 4 * 8, 64, 3
+    o = S * rows * D * 4
+    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, D, S) == ((o + 255) // 256) * 256 + S * rows * 8
+    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 48, S) == 0
+    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 64, 0) == 0
+    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 64, 65) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_splits=0), -6), (dict(n_splits=65), -6), (dict(n_splits=-1), -6),
+    (dict(ws=0), -1), (dict(ws=128), -5), (dict(ws_bytes=100), -9),
+    (dict(q=0), -1), (dict(D=48), -3), (dict(scale=-1.0), -6),
+])
+def test_splitkv_argument_errors(lib, kw, code):
+    assert _call_split(**kw) == code
+
+
+def test_choose_splits():
+    assert fa.choose_splits(1, 32, 1, 32768) == 10      # 32 tiles -> fill 296 CTAs
+    assert fa.choose_splits(4, 48, 8192, 8192) == 1     # already many tiles
+    assert fa.choose_splits(1, 1, 1, 128) == 1          # one key block
+    assert fa.choose_splits(1, 1, 1, 1 << 20) == 64     # capped

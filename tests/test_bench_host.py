@@ -86,3 +86,21 @@ def test_max_over_two_gloo_ranks():
     for rank, m, v in got:
         assert m == 2.0                        # the max over ranks
         assert v == pytest.approx(3e12 * 2 * 5 / 2.0 / 1e12)
+
+
+def test_roofline_bound_by_workload():
+    # the long-sequence forward is tensor bound, one-query decoding HBM bound
+    assert bench.roofline_bound(W.ROOFLINE, 1640.0, 6461.8) == "tensor"
+    for w in W.DECODE:
+        assert bench.roofline_bound(w, 1640.0, 6461.8) == "hbm", w.name
+    # decoding moves the K/V cache once: 2 tensors * B*H_kv*L_k*D * 2 bytes
+    w = W.DECODE[0]
+    kv = 2 * w.B * w.H_kv * w.L_k * w.D * 2
+    assert kv < bench.min_hbm_bytes(w) < kv * 1.01
+
+
+def test_resolve_splits():
+    w = W.DECODE[0]
+    assert bench.resolve_splits("0", w) == 0
+    assert bench.resolve_splits("5", w) == 5
+    assert 1 <= bench.resolve_splits("auto", w) <= 64
