@@ -21,10 +21,12 @@ FA_OK = 0
 STATUS = {
     0: "FA_OK", -1: "FA_ERR_NULL", -2: "FA_ERR_SHAPE", -3: "FA_ERR_HEADDIM",
     -4: "FA_ERR_DTYPE", -5: "FA_ERR_ALIGN", -6: "FA_ERR_ARG", -7: "FA_ERR_CUDA",
-    -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE",
+    -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE", -10: "FA_ERR_SCRATCH",
 }
-EXPORTS = ("fa_fwd", "fa_fwd_splitkv", "fa_get_device_status", "fa_splitkv_workspace_bytes",
-           "fa_status_string", "fa_version")
+EXPORTS = ("fa_fwd", "fa_fwd_splitkv", "fa_fwd_splitkv_static", "fa_get_device_status",
+           "fa_splitkv_workspace_bytes", "fa_status_string", "fa_version")
+# size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
+STATIC_SCRATCH_BYTES = 16 << 20
 
 _lock = threading.Lock()
 _lib = None
@@ -57,6 +59,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
                                        i, i, i, i, i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_splitkv.restype = i
+        lib.fa_fwd_splitkv_static.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                              ctypes.c_float, i, i, i, i, i, vp]
+        lib.fa_fwd_splitkv_static.restype = i
         lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_get_device_status.argtypes = [vp]
@@ -86,6 +91,15 @@ def fa_fwd_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
                                  float(scale), int(causal), int(window_left),
                                  int(window_right), int(dtype), int(n_splits),
                                  workspace, int(workspace_bytes), stream)
+
+
+def fa_fwd_splitkv_static(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
+                          window_left, window_right, dtype, n_splits, stream) -> int:
+    """The no-allocation split-KV C entry point, unchanged (its partials
+    live in the library's static scratch; see include/fa.h)."""
+    return load().fa_fwd_splitkv_static(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D,
+                                        float(scale), int(causal), int(window_left),
+                                        int(window_right), int(dtype), int(n_splits), stream)
 
 
 def fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits) -> int:
@@ -127,7 +141,9 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
     ``n_splits`` > 0 computes the same result through fa_fwd_splitkv with
     that many key slices ("auto" picks them with ``choose_splits``); the
     workspace is allocated here with torch unless ``workspace`` (a uint8
-    CUDA tensor, 256-byte aligned) is given.
+    CUDA tensor, 256-byte aligned) is given.  ``workspace="static"`` calls
+    fa_fwd_splitkv_static instead, which uses the library's fixed scratch
+    and allocates nothing (calls must not overlap on the GPU).
     """
     import torch
 
@@ -165,6 +181,12 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
                         B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
                         window_right, dtype, stream.cuda_stream)
             where = "fa_fwd"
+        elif isinstance(workspace, str) and workspace == "static":
+            st = fa_fwd_splitkv_static(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                       lse.data_ptr() if lse is not None else None,
+                                       B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                                       window_right, dtype, n_splits, stream.cuda_stream)
+            where = "fa_fwd_splitkv_static"
         else:
             need = fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits)
             if workspace is None:

@@ -323,6 +323,58 @@ extern "C" int fa_fwd_splitkv(const void *q, const void *k, const void *v, void 
                   window_right, dtype, n_splits, workspace, workspace_bytes, stream);
 }
 
+// ---------------------------------------------------------------------------
+// No-allocation variant of the split-KV forward.  Its partials live in this
+// file-scope array (module memory: it exists once per device as soon as the
+// library's module is loaded there, no call allocates it).  The pages have
+// no counterpart; it serves callers that may not call cudaMalloc while they
+// run attention (see fa.h).
+static __device__ __align__(256) unsigned char g_fa_static_scratch[FA_STATIC_SCRATCH_BYTES];
+
+namespace fa {
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up on the
+// first call there and cached.
+int static_scratch(void **addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_static_scratch) != cudaSuccess || p == nullptr)
+      return FA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return FA_OK;
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out,
+                                     float *lse, int B, int H, int H_kv, int L_q, int L_k,
+                                     int D, float scale, int causal, int window_left,
+                                     int window_right, int dtype, int n_splits,
+                                     cudaStream_t stream) {
+  if (n_splits < 1 || n_splits > fa::kMaxSplits) return FA_ERR_ARG;
+  // the size limit first, so that an oversized problem never reaches the GPU
+  // (sizes fwd_impl would reject fall through to its own error codes)
+  if (B >= 1 && H >= 1 && L_q >= 0 && L_q <= fa::kMaxSeq &&
+      (D == 16 || D == 32 || D == 64 || D == 128) &&
+      fa::ws_total_bytes(static_cast<int64_t>(B) * H * L_q, D, n_splits) >
+          FA_STATIC_SCRATCH_BYTES)
+    return FA_ERR_SCRATCH;
+  void *scratch = nullptr;
+  const int st = fa::static_scratch(&scratch);
+  if (st != FA_OK) return st;
+  return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                  window_right, dtype, n_splits, scratch, FA_STATIC_SCRATCH_BYTES, stream);
+}
+
 extern "C" int fa_get_device_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int st = 0;
@@ -348,6 +400,7 @@ extern "C" const char *fa_status_string(int status) {
     case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call failed";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait gave up";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace smaller than fa_splitkv_workspace_bytes()";
+    case FA_ERR_SCRATCH: return "FA_ERR_SCRATCH: problem needs more than FA_STATIC_SCRATCH_BYTES of scratch";
   }
   return "unknown fa status";
 }

@@ -21,7 +21,9 @@
  * All functions return 0 (FA_OK) or a negative fa_status; none aborts.
  * Every pointer argument marked "device" must point to memory the current
  * CUDA device can read/write; the library allocates no memory and keeps no
- * state between calls other than one device-side status word.
+ * state between calls other than one device-side status word and the
+ * static scratch of fa_fwd_splitkv_static (module memory, not allocated by
+ * any call).
  */
 #ifndef FA_H
 #define FA_H
@@ -53,8 +55,10 @@ typedef enum {
                              tensor-map encoding, device query) */
     FA_ERR_TIMEOUT = -8,  /* a device-side wait gave up (watchdog); the
                              outputs of that launch are not valid */
-    FA_ERR_WORKSPACE = -9 /* workspace smaller than the size the matching
-                             *_workspace_bytes() call returns */
+    FA_ERR_WORKSPACE = -9, /* workspace smaller than the size the matching
+                              *_workspace_bytes() call returns */
+    FA_ERR_SCRATCH = -10   /* fa_fwd_splitkv_static: the problem needs more
+                              than FA_STATIC_SCRATCH_BYTES of scratch */
 } fa_status;
 
 /*
@@ -117,6 +121,38 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float
                    int causal, int window_left, int window_right, int dtype,
                    int n_splits, void *workspace, size_t workspace_bytes,
                    cudaStream_t stream);
+
+/*
+ * fa_fwd_splitkv_static -- fa_fwd_splitkv with no workspace argument: the
+ * partials live in a fixed scratch array inside the library (static device
+ * memory, FA_STATIC_SCRATCH_BYTES per device).  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory at the time they run attention: a process whose
+ * device memory is all owned by another allocator (so that a cudaMalloc
+ * beside it could fail or fragment it), a serving loop that must not take
+ * cudaMalloc's implicit device synchronisation and unbounded latency after
+ * start-up, or a plug-in that has no handle on its host's allocator.  Every
+ * call, and the library itself, allocates nothing.
+ *
+ * Arguments as fa_fwd_splitkv without `workspace` / `workspace_bytes`.
+ * Returns FA_ERR_SCRATCH, before touching the GPU, when
+ * fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits) exceeds
+ * FA_STATIC_SCRATCH_BYTES (16 MiB: e.g. 32768 query rows x n_splits at
+ * D = 128; lower n_splits to fit); other errors as fa_fwd_splitkv.
+ *
+ * Set-up: the first call on each device (with that device current) looks
+ * up the scratch's device address once and caches it; make that first call
+ * before any stream capture.  Nothing in the scratch has to start at zero:
+ * every partial the merge reads is written earlier in the same call.
+ * There is ONE scratch per device: calls whose work overlaps on the GPU
+ * (different streams, or different host threads) race on it and corrupt
+ * each other's results; serialise them (one stream, or events).
+ */
+#define FA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out,
+                          float *lse, int B, int H, int H_kv, int L_q, int L_k, int D,
+                          float scale, int causal, int window_left, int window_right,
+                          int dtype, int n_splits, cudaStream_t stream);
 
 /*
  * fa_get_device_status -- synchronise `stream`, then read and clear the

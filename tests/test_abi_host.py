@@ -131,3 +131,29 @@ def test_choose_splits():
     assert fa.choose_splits(4, 48, 8192, 8192) == 1     # already many tiles
     assert fa.choose_splits(1, 1, 1, 128) == 1          # one key block
     assert fa.choose_splits(1, 1, 1, 1 << 20) == 64     # capped
+
+
+# ------------------------------------------------------------ static-scratch entry
+def _call_static(n_splits=2, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_splitkv_static(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"],
+                                    a["H_kv"], a["L_q"], a["L_k"], a["D"], a["scale"],
+                                    a["causal"], a["wl"], a["wr"], a["dtype"], n_splits, None)
+
+
+def test_static_scratch_size_matches_header():
+    text = open(HEADER).read()
+    assert "#define FA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)" in text
+    assert binding.STATIC_SCRATCH_BYTES == 16 << 20
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_splits=0), -6), (dict(n_splits=65), -6),
+    # 32768 rows x 2 slices x (128 fp32 + one float2) = 33.5 MB > 16 MiB:
+    # refused before any CUDA call
+    (dict(n_splits=2, B=1, H=64, H_kv=64, L_q=512, D=128), -10),
+    (dict(n_splits=64, B=1, H=8, H_kv=8, L_q=128, D=128), -10),
+])
+def test_static_entry_refuses_before_the_gpu(lib, kw, code):
+    assert _call_static(**kw) == code
