@@ -409,7 +409,7 @@ def resolve_splits(arg: str, w: W.Workload, sm_count: int = 148) -> int:
     """--splits: 0 (fa_fwd), an explicit slice count, or auto."""
     if arg == "auto":
         from exact_attention_113_b200.binding import choose_splits
-        return choose_splits(w.B, w.H, w.L_q, w.L_k, sm_count)
+        return choose_splits(w.B, w.H, w.L_q, w.L_k, sm_count, H_kv=w.H_kv)
     return int(arg)
 
 

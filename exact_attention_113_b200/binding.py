@@ -106,13 +106,32 @@ def fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits) -> int:
     return int(load().fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits))
 
 
-def choose_splits(B, H, L_q, L_k, sm_count=148) -> int:
-    """Key slices for fa_fwd_splitkv: enough CTAs to fill the GPU about twice,
-    at least two 128-key blocks per slice, at most 64 slices."""
-    tiles = B * H * max(1, -(-L_q // 128))
+def query_tiles(B, H, H_kv, L_q) -> int:
+    """128-row query tiles of a launch.  With GQA (H / H_kv a power of two)
+    and L_q < 128 the library packs a group's heads into one tile:
+    128 / group query positions of each head."""
+    g = H // H_kv
+    if 2 <= g <= 128 and (g & (g - 1)) == 0 and L_q < 128:
+        return B * H_kv * max(1, -(-L_q // (128 // g)))
+    return B * H * max(1, -(-L_q // 128))
+
+
+def choose_splits(B, H, L_q, L_k, sm_count=148, H_kv=None) -> int:
+    """Key slices for fa_fwd_splitkv (1..64, at least two 128-key blocks per
+    slice) minimising a cost model fitted to B200 decode timings: a CTA costs
+    about 4.5 key blocks of fixed work (set-up, pipeline fill, epilogue) plus
+    its blocks, and CTAs run in waves of ``sm_count`` (one per SM)."""
+    tiles = query_tiles(B, H, H if H_kv is None else H_kv, L_q)
     blocks = max(1, -(-L_k // 128))
-    want = max(1, -(-2 * sm_count // tiles))
-    return int(max(1, min(64, want, blocks // 2 if blocks >= 2 else 1)))
+    best, best_cost = 1, None
+    for sp in range(1, 65):
+        per = -(-blocks // sp)
+        if sp > 1 and per < 2:
+            break
+        cost = -(-tiles * sp // sm_count) * (4.5 + per)
+        if best_cost is None or cost < best_cost:
+            best, best_cost = sp, cost
+    return best
 
 
 def fa_get_device_status(stream=None) -> int:
@@ -173,7 +192,8 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
         stream = torch.cuda.current_stream(q.device)
     if n_splits == "auto":
         n_splits = choose_splits(B, H, L_q, L_k,
-                                 torch.cuda.get_device_properties(q.device).multi_processor_count)
+                                 torch.cuda.get_device_properties(q.device).multi_processor_count,
+                                 H_kv=H_kv)
     with torch.cuda.device(q.device):
         if not n_splits:
             st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),

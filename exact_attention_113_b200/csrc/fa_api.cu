@@ -45,9 +45,10 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // A rank-3 tensor map over a contiguous [n_heads, L, D] array with a box of
-// [1, 128, box_cols] and the swizzle that matches `box_cols` 16-bit elements.
+// [box_heads, box_rows, box_cols] and the swizzle that matches `box_cols`
+// 16-bit elements.  box_heads * box_rows = 128 (one tile of rows).
 bool encode_map(CUtensorMap *map, const void *base, int dtype, int n_heads, int L, int D,
-                int box_cols) {
+                int box_cols, int box_rows = kBM, int box_heads = 1) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const CUtensorMapDataType dt =
@@ -56,7 +57,8 @@ bool encode_map(CUtensorMap *map, const void *base, int dtype, int n_heads, int 
                         static_cast<cuuint64_t>(n_heads)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                            static_cast<cuuint64_t>(L) * D * 2};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows),
+                       static_cast<cuuint32_t>(box_heads)};
   cuuint32_t estr[3] = {1, 1, 1};
   const int sw_bytes = box_cols * 2;
   const CUtensorMapSwizzle sw = sw_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -94,8 +96,8 @@ int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
       configured[dev] = true;
     }
   }
-  dim3 grid(static_cast<unsigned>(prm.n_qpairs) * static_cast<unsigned>(B * H) *
-                static_cast<unsigned>(prm.n_splits),
+  const unsigned items = static_cast<unsigned>(B) * (prm.packed ? prm.H_kv : H);
+  dim3 grid(static_cast<unsigned>(prm.n_qpairs) * items * static_cast<unsigned>(prm.n_splits),
             1, 1);
   kern<<<grid, kThreads, G::kSmemBytes, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -239,6 +241,19 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
   prm.L_q = L_q;
   prm.L_k = L_k;
   prm.group = H / H_kv;
+  // GQA packing for short query ranges: the group's heads share a tile, so
+  // a K/V head is streamed once per group instead of once per query head.
+  {
+    const int g = prm.group;
+    const bool pow2 = g >= 2 && g <= kBM && (g & (g - 1)) == 0;
+    prm.packed = (pow2 && L_q < kBM) ? 1 : 0;
+    prm.tile_q = prm.packed ? kBM / g : kBM;
+    int sh = 0;
+    while ((1 << sh) < prm.tile_q) ++sh;
+    prm.tile_q_shift = sh;
+  }
+  const int64_t q_tiles = (L_q + prm.tile_q - 1) / prm.tile_q;      // per work item
+  const int64_t items = static_cast<int64_t>(B) * (prm.packed ? H_kv : H);
   // Two query tiles per CTA keep the tensor pipe busy (ping-pong); when that
   // leaves SMs idle (few heads, short sequences), one tile per CTA doubles
   // the number of CTAs.
@@ -247,10 +262,11 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t tiles_total = static_cast<int64_t>(B) * H * ((L_q + kBM - 1) / kBM);
-    prm.tiles = (tiles_total <= static_cast<int64_t>(sms)) ? 1 : 2;
+    prm.tiles = (items * q_tiles <= static_cast<int64_t>(sms)) ? 1 : 2;
   }
-  prm.n_qpairs = (L_q + prm.tiles * kBM - 1) / (prm.tiles * kBM);
+  prm.n_qpairs = static_cast<int>((q_tiles + prm.tiles - 1) / prm.tiles);
+  if (items * prm.n_qpairs * (n_splits > 0 ? n_splits : 1) > 0x7fffffffll)
+    return FA_ERR_SHAPE;                   // grid.x limit
   prm.wl = wl;
   prm.wr = wr;
   prm.reverse = (wr >= 0) ? 1 : 0;         // later query tiles see more keys
@@ -266,10 +282,11 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
                                            ws_ml_offset(rows_total, D, n_splits));
   }
   const int box_cols = D * 2 >= 128 ? 64 : D;
-  if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
+  const int q_box_heads = prm.packed ? prm.group : 1;
+  if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols, prm.tile_q, q_box_heads) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
-      !encode_map(&prm.tm_o, out, dtype, B * H, L_q, D, box_cols))
+      !encode_map(&prm.tm_o, out, dtype, B * H, L_q, D, box_cols, prm.tile_q, q_box_heads))
     return FA_ERR_CUDA;
 
   int st = FA_ERR_HEADDIM;

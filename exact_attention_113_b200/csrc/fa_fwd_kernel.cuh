@@ -76,7 +76,15 @@ struct FwdParams {
   float *lse;         // [B*H, L_q] or nullptr
   int H, H_kv, L_q, L_k;
   int group;          // H / H_kv
-  int n_qpairs;       // query-tile groups per head: ceil(L_q / (128 * tiles))
+  int n_qpairs;       // query-tile groups per work item: ceil(ceil(L_q / tile_q) / tiles)
+  // GQA packing (packed == 1, short query ranges): a 128-row tile holds
+  // tile_q = 128 / group query rows of each of the group's heads, row
+  // r = g * tile_q + i_local, so that one pass over a K/V head serves the
+  // whole group.  The Q / O tensor maps then have a box of [group, tile_q,
+  // cols] and a work item is one (batch, K/V head).
+  int packed;
+  int tile_q;         // query positions per tile: 128, or 128 / group when packed
+  int tile_q_shift;   // log2(tile_q) when packed
   int tiles;          // query tiles per CTA: 2 (ping-pong) or 1 (small problems)
   int wl, wr;         // visible iff i - wl <= j <= i + wr; -1 = unbounded
   int reverse;        // process query pairs last-first (causal: heavy first)
@@ -174,22 +182,32 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   // ---- work item: (batch*head, pair of query tiles, key slice);
   // consecutive CTAs take consecutive query pairs of one head, so a head's
   // K/V stays hot in L2.
-  const int per_bh = p.n_qpairs * p.n_splits;
-  const int bh = static_cast<int>(blockIdx.x) / per_bh;
-  const int rem = static_cast<int>(blockIdx.x) - bh * per_bh;
+  const int per_item = p.n_qpairs * p.n_splits;
+  const int item = static_cast<int>(blockIdx.x) / per_item;
+  const int rem = static_cast<int>(blockIdx.x) - item * per_item;
   const int qp_idx = rem / p.n_splits;
   const int split = rem - qp_idx * p.n_splits;
   const int qpair = p.reverse ? (p.n_qpairs - 1 - qp_idx) : qp_idx;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-  const int bh_kv = b * p.H_kv + h / p.group;   // GQA: contiguous head groups
+  // bh: (first) query head of the tile in [B*H]; bh_kv: its K/V head
+  int bh, bh_kv;
+  if (p.packed) {
+    const int b = item / p.H_kv;
+    const int hk = item - b * p.H_kv;
+    bh = b * p.H + hk * p.group;
+    bh_kv = item;
+  } else {
+    const int b = item / p.H;
+    const int h = item - b * p.H;
+    bh = item;
+    bh_kv = b * p.H_kv + h / p.group;   // GQA: contiguous head groups
+  }
 
-  int q0[2], rows[2];
+  int q0[2], rows[2];   // first query position and query positions per head
   BlockRange rng[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    q0[t] = (qpair * p.tiles + t) * kBM;
-    rows[t] = t < p.tiles ? max(0, min(kBM, p.L_q - q0[t])) : 0;
+    q0[t] = (qpair * p.tiles + t) * p.tile_q;
+    rows[t] = t < p.tiles ? max(0, min(p.tile_q, p.L_q - q0[t])) : 0;
     if (rows[t] > 0) {
       rng[t] = tile_block_range(q0[t], q0[t] + rows[t] - 1, p.L_k, p.wl, p.wr);
     } else {
@@ -462,7 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     const uint32_t tS = tmem + lane_base + t * 128u;
     const uint32_t tO = tmem + lane_base + 256u + t * D;
     const uint32_t tPs = tmem + lane_base + 384u + t * 64u;   // split-P: P_t columns
-    const int i = tq0 + r;               // query index of this row
+    // packed tiles: row r is query position r % tile_q of head bh + r / tile_q
+    const int r_loc = p.packed ? (r & (p.tile_q - 1)) : r;
+    const int row_head = p.packed ? bh + (r >> p.tile_q_shift) : bh;
+    const int i = tq0 + r_loc;           // query index of this row
     const int row_lo = p.wl < 0 ? 0 : i - p.wl;
     const int row_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, i + p.wr);
     const int first = tq0, last = tq0 + trows - 1;
@@ -717,9 +738,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         // tcgen05.ld is warp-collective: every lane loads (ok and n_blocks
         // are warp-uniform), only the lanes of real rows store.
         if (ok) {
-          const bool mine = r < trows;
+          const bool mine = r_loc < trows;
           const size_t row = static_cast<size_t>(split) * p.rows_total +
-                             static_cast<size_t>(bh) * p.L_q + i;
+                             static_cast<size_t>(row_head) * p.L_q + i;
           float4 *dst = reinterpret_cast<float4 *>(p.ws_o + row * D);
           constexpr int kChunk = D >= 32 ? 32 : D;
 #pragma unroll
@@ -807,9 +828,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         bulk_commit_group();
         bulk_wait_group_all();
       }
-      if (ok && p.lse != nullptr && r < trows) {
+      if (ok && p.lse != nullptr && r_loc < trows) {
         const float lse = l > 0.0f ? (m_use + __log2f(l)) * 0.6931471805599453f : -INFINITY;
-        p.lse[static_cast<size_t>(bh) * p.L_q + i] = lse;
+        p.lse[static_cast<size_t>(row_head) * p.L_q + i] = lse;
       }
       }   // normal epilogue
     }

@@ -127,10 +127,17 @@ def test_splitkv_argument_errors(lib, kw, code):
 
 
 def test_choose_splits():
-    assert fa.choose_splits(1, 32, 1, 32768) == 10      # 32 tiles -> fill 296 CTAs
-    assert fa.choose_splits(4, 48, 8192, 8192) == 1     # already many tiles
+    assert fa.choose_splits(1, 32, 1, 32768) == 9       # 32 tiles -> 288 CTAs, two waves
+    assert fa.choose_splits(4, 48, 8192, 8192) == 1     # already many waves
     assert fa.choose_splits(1, 1, 1, 128) == 1          # one key block
     assert fa.choose_splits(1, 1, 1, 1 << 20) == 64     # capped
+    # GQA packing: 32 query heads over 8 K/V heads, one query row -> 8 tiles
+    assert fa.binding.query_tiles(1, 32, 8, 1) == 8
+    assert fa.binding.query_tiles(1, 32, 8, 40) == 16      # 32 rows per head per tile
+    assert fa.binding.query_tiles(1, 12, 2, 1) == 12       # group 6: not packed
+    assert fa.binding.query_tiles(1, 32, 8, 128) == 32     # long enough: not packed
+    assert fa.choose_splits(1, 32, 1, 32768, H_kv=8) == 18  # 144 CTAs, one wave
+    assert fa.choose_splits(8, 32, 1, 32768, H_kv=8) == 2   # 128 CTAs, one wave
 
 
 # ------------------------------------------------------------ static-scratch entry

@@ -143,3 +143,33 @@ def test_roofline_config_sampled():
 def test_device_status_clean_at_end():
     import exact_attention_113_b200 as fa
     assert fa.fa_get_device_status() == 0
+
+
+# ------------------------------------------------------------ GQA packing
+# With H / H_kv a power of two and L_q < 128, one 128-row tile holds
+# 128 / group query positions of each head of a group (the Q / O boxes are
+# [group, 128 / group, cols]); (12, 2) is a group of 6 and stays unpacked.
+@pytest.mark.parametrize("H,H_kv", [(4, 2), (8, 2), (16, 2), (32, 4), (128, 1), (12, 2)])
+@pytest.mark.parametrize("L_q", [1, 5, 31, 32, 33, 127])
+def test_gqa_packed_short_queries(H, H_kv, L_q):
+    check_full(_w(B=2, H=H, H_kv=H_kv, L_q=L_q, L_k=700, D=128, seed=5000 + H + L_q))
+
+
+@pytest.mark.parametrize("wl,wr,causal", [(-1, -1, True), (16, -1, True), (-1, 650, False),
+                                          (200, 40, False)])
+@pytest.mark.parametrize("D", [32, 64])
+def test_gqa_packed_masks(wl, wr, causal, D):
+    check_full(_w(B=1, H=16, H_kv=4, L_q=100, L_k=700, D=D, causal=causal, window_left=wl,
+                  window_right=wr, seed=5100 + D), derived=True)
+
+
+def test_gqa_packed_matches_repeated_heads():
+    # the packed tile and the per-head tile compute the same rows; they may
+    # differ in the last bits (rows of one warp share rescale decisions)
+    w = _w(B=2, H=8, H_kv=2, L_q=20, L_k=3000, D=128, dtype=BF16, seed=5200)
+    q, k, v = make_qkv(w)
+    o1, l1 = run_gpu(q, k, v, w)
+    wm = dataclasses.replace(w, H_kv=8)
+    o2, l2 = run_gpu(q, k.repeat_interleave(4, dim=1), v.repeat_interleave(4, dim=1), wm)
+    assert (o1.float() - o2.float()).abs().max().item() <= 2 * 3e-3 + 4e-3   # two gates
+    assert (l1 - l2).abs().max().item() <= 1e-4

@@ -133,4 +133,4 @@ def test_auto_splits_runs():
 def test_decode_workloads_sampled(w):
     import exact_attention_113_b200 as fa
     rows = np.arange(w.B * w.H * w.L_q, dtype=np.int64)     # every row: a few hundred
-    check_rows(w, rows, n_splits=fa.choose_splits(w.B, w.H, w.L_q, w.L_k))
+    check_rows(w, rows, n_splits=fa.choose_splits(w.B, w.H, w.L_q, w.L_k, H_kv=w.H_kv))
