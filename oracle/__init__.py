@@ -11,9 +11,11 @@ The C source ``attention_ref.c`` states, function by function, which passage
 of the pages it follows.  This module is a ctypes shim around it plus the
 build step that compiles it with gcc.
 
-Functions whose parity is pinned (see tests/test_oracle_pins.py):
+Functions whose parity is pinned (see tests/test_oracle_pins.py and
+tests/test_oracle_bwd_pins.py):
   attention, attention_rows, attention_rows_online, safe_softmax,
-  online_softmax, f16/bf16 decode and round-to-nearest-even.
+  online_softmax, f16/bf16 decode and round-to-nearest-even,
+  attention_f64, attention_bwd_f64 / attention_bwd (gradients).
 """
 from __future__ import annotations
 
@@ -102,6 +104,13 @@ class Oracle:
             u16p, u16p, u16p, ctypes.c_int, i64, i64, i64, i64, i64, i64,
             ctypes.c_double, ctypes.c_int, i64, i64, i64p, i64, i64, dp, dp]
         lib.oracle_attention_rows_online.restype = ctypes.c_int
+        lib.oracle_attention_f64.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, i64,
+                                             ctypes.c_double, ctypes.c_int, i64, i64, dp, dp]
+        lib.oracle_attention_f64.restype = ctypes.c_int
+        lib.oracle_attention_bwd_f64.argtypes = [
+            dp, dp, dp, dp, i64, i64, i64, i64, i64, i64, ctypes.c_double, ctypes.c_int,
+            i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.oracle_attention_bwd_f64.restype = ctypes.c_int
         self.lib = lib
         self._tables = {}
 
@@ -211,6 +220,59 @@ class Oracle:
         if rc < 0:
             raise ValueError("oracle rejected the arguments")
         return out, lse
+
+
+    # ------------------------------------------------------------- fp64 inputs
+    @staticmethod
+    def _f64(x):
+        return np.ascontiguousarray(x, dtype=np.float64)
+
+    def attention_f64(self, q, k, v, scale, causal=False, window_left=-1, window_right=-1):
+        """Forward on float64 arrays q [B,H,L_q,D], k, v [B,H_kv,L_k,D] (no
+        rounding anywhere); returns (out [B,H,L_q,D], lse [B,H,L_q])."""
+        q, k, v = self._f64(q), self._f64(k), self._f64(v)
+        B, H, L_q, D = q.shape
+        _, H_kv, L_k, _ = k.shape
+        out = np.zeros_like(q)
+        lse = np.zeros((B, H, L_q), dtype=np.float64)
+        rc = self.lib.oracle_attention_f64(
+            _ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
+            B, H, H_kv, L_q, L_k, D, float(scale), int(bool(causal)), int(window_left),
+            int(window_right), _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+        if rc < 0:
+            raise ValueError("oracle rejected the arguments")
+        return out, lse
+
+    def attention_bwd_f64(self, q, k, v, dout, scale, causal=False, window_left=-1,
+                          window_right=-1, delta_err=None, with_abs=False, n_threads=0):
+        """Gradients of sum(dout * O) on float64 arrays: returns (dq, dk, dv),
+        or (dq, dk, dv, dq_abs, dk_abs, dv_abs) with ``with_abs`` (the error
+        scales documented in attention_ref.c; ``delta_err`` [B,H,L_q])."""
+        q, k, v, dout = self._f64(q), self._f64(k), self._f64(v), self._f64(dout)
+        B, H, L_q, D = q.shape
+        _, H_kv, L_k, _ = k.shape
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        absb = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)] if with_abs else None
+        de = None if delta_err is None else self._f64(delta_err).reshape(B, H, L_q)
+        c = ctypes.c_double
+        rc = self.lib.oracle_attention_bwd_f64(
+            _ptr(q, c), _ptr(k, c), _ptr(v, c), _ptr(dout, c), B, H, H_kv, L_q, L_k, D,
+            float(scale), int(bool(causal)), int(window_left), int(window_right),
+            _ptr(dq, c), _ptr(dk, c), _ptr(dv, c), _ptr(de, c) if de is not None else None,
+            _ptr(absb[0], c) if with_abs else None, _ptr(absb[1], c) if with_abs else None,
+            _ptr(absb[2], c) if with_abs else None, int(n_threads))
+        if rc < 0:
+            raise ValueError("oracle rejected the arguments")
+        if with_abs:
+            return dq, dk, dv, absb[0], absb[1], absb[2]
+        return dq, dk, dv
+
+    def attention_bwd(self, q, k, v, dout, dtype, scale, causal=False, window_left=-1,
+                      window_right=-1, delta_err=None, with_abs=False):
+        """attention_bwd_f64 on fp16/bf16 bit patterns (decoded exactly)."""
+        dec = [self.decode(x, dtype) for x in (q, k, v, dout)]
+        return self.attention_bwd_f64(*dec, scale, causal, window_left, window_right,
+                                      delta_err, with_abs)
 
 
 _default = None

@@ -359,3 +359,175 @@ int oracle_attention_rows_online(const uint16_t *q, const uint16_t *k,
     free(sb);
     return 1;
 }
+
+/* ---------------------------------------------------------------------
+ * Attention on fp64 inputs, forward and backward.
+ *
+ * Backward: the pages keep only the softmax statistics from the forward and
+ * recompute the attention matrix from Q, K, V when the gradients are taken
+ * ("FlashAttention算法原理与性能优化实战" section 1.2.3, recomputation;
+ * "Flash Attention是怎么做到又快又省显存的？" 总结, recomputation as a
+ * tiling-based gradient checkpoint; the Triton FA2 walkthrough keeps the
+ * logsumexp for the backward pass).  They print no gradient formulas, so
+ * this is the plain definition: the gradient of sum(dO .* O) for
+ * O = softmax(scale Q K^T + mask) V, by the chain rule,
+ *     dV = P^T dO,  dP = dO V^T,  dS_ij = P_ij (dP_ij - delta_i),
+ *     delta_i = sum_j P_ij dP_ij,  dQ = scale dS K,  dK = scale dS^T Q,
+ * with P recomputed by the plain safe softmax of each row.  With GQA, the
+ * gradient of a shared K/V head sums over the query heads that read it.
+ * ------------------------------------------------------------------- */
+
+/*
+ * Forward on fp64 inputs (no rounding anywhere); layout as
+ * oracle_attention_rows, all rows.  out [B,H,L_q,D], lse [B,H,L_q]
+ * (nullable).  Returns 0, or -1 on bad sizes.
+ */
+int oracle_attention_f64(const double *q, const double *k, const double *v,
+                         int64_t B, int64_t H, int64_t H_kv, int64_t L_q,
+                         int64_t L_k, int64_t D, double scale, int causal,
+                         int64_t wl, int64_t wr, double *out, double *lse)
+{
+    if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1 ||
+        H % H_kv != 0)
+        return -1;
+    const int64_t group = H / H_kv;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(L_k > 0 ? L_k : 1));
+    double *p = (double *)malloc(sizeof(double) * (size_t)(L_k > 0 ? L_k : 1));
+    if (!s || !p) { free(s); free(p); return -2; }
+    for (int64_t b = 0; b < B; b++)
+        for (int64_t h = 0; h < H; h++) {
+            const double *kp = k + (b * H_kv + h / group) * L_k * D;
+            const double *vp = v + (b * H_kv + h / group) * L_k * D;
+            for (int64_t i = 0; i < L_q; i++) {
+                const int64_t row = (b * H + h) * L_q + i;
+                const double *qi = q + row * D;
+                for (int64_t j = 0; j < L_k; j++) {
+                    if (!visible(i, j, L_k, causal, wl, wr)) { s[j] = -INFINITY; continue; }
+                    double acc = 0.0;
+                    for (int64_t d = 0; d < D; d++) acc += qi[d] * kp[j * D + d];
+                    s[j] = scale * acc;
+                }
+                double m, den;
+                oracle_safe_softmax(s, L_k, p, &den, &m);
+                double *o = out + row * D;
+                for (int64_t d = 0; d < D; d++) o[d] = 0.0;
+                for (int64_t j = 0; j < L_k; j++)
+                    for (int64_t d = 0; d < D; d++) o[d] += p[j] * vp[j * D + d];
+                if (lse) lse[row] = (m == -INFINITY) ? -INFINITY : m + log(den);
+            }
+        }
+    free(s);
+    free(p);
+    return 0;
+}
+
+/*
+ * Backward on fp64 inputs: dq [B,H,L_q,D], dk and dv [B,H_kv,L_k,D] (all
+ * written), for the upstream gradient dout [B,H,L_q,D].
+ *
+ * Optional error scales for the parity tests (each nullable; not part of
+ * the gradient): given delta_err[row] >= 0, a bound on the error of the
+ * delta_i the tested implementation uses,
+ *   dv_abs = |P|^T |dO|,
+ *   dk_abs = scale (|dS| + P e)^T |Q|,   dq_abs = scale (|dS| + P e) |K|,
+ * with e_i = delta_err[i] (0 when delta_err is NULL): rounding P or dS to a
+ * t-bit format moves a gradient by at most 2^-t times these (first order),
+ * and an error e_i in delta_i moves dS_ij by P_ij e_i.
+ * Threads run over (b, K/V head) so that each owns its dk / dv rows.
+ * Returns the number of threads used, or a negative value on bad input.
+ */
+int oracle_attention_bwd_f64(const double *q, const double *k, const double *v,
+                             const double *dout, int64_t B, int64_t H,
+                             int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
+                             double scale, int causal, int64_t wl, int64_t wr,
+                             double *dq, double *dk, double *dv,
+                             const double *delta_err, double *dq_abs,
+                             double *dk_abs, double *dv_abs, int n_threads)
+{
+    if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1 ||
+        H % H_kv != 0)
+        return -1;
+    const int64_t group = H / H_kv;
+    int used = 1;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#endif
+#pragma omp parallel
+    {
+#ifdef _OPENMP
+#pragma omp single
+        used = omp_get_num_threads();
+#endif
+        const size_t nk = (size_t)(L_k > 0 ? L_k : 1);
+        double *s = (double *)malloc(sizeof(double) * nk);
+        double *p = (double *)malloc(sizeof(double) * nk);
+        double *dp = (double *)malloc(sizeof(double) * nk);
+        double *ds = (double *)malloc(sizeof(double) * nk);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bg = 0; bg < B * H_kv; bg++) {
+            const int64_t b = bg / H_kv, g = bg % H_kv;
+            const double *kp = k + bg * L_k * D;
+            const double *vp = v + bg * L_k * D;
+            double *dkp = dk + bg * L_k * D;
+            double *dvp = dv + bg * L_k * D;
+            double *dka = dk_abs ? dk_abs + bg * L_k * D : NULL;
+            double *dva = dv_abs ? dv_abs + bg * L_k * D : NULL;
+            for (int64_t x = 0; x < L_k * D; x++) {
+                dkp[x] = 0.0;
+                dvp[x] = 0.0;
+                if (dka) dka[x] = 0.0;
+                if (dva) dva[x] = 0.0;
+            }
+            for (int64_t h = g * group; h < (g + 1) * group; h++)
+                for (int64_t i = 0; i < L_q; i++) {
+                    const int64_t row = (b * H + h) * L_q + i;
+                    const double *qi = q + row * D;
+                    const double *doi = dout + row * D;
+                    /* recompute P_i (plain safe softmax of the scaled row) */
+                    for (int64_t j = 0; j < L_k; j++) {
+                        if (!visible(i, j, L_k, causal, wl, wr)) { s[j] = -INFINITY; continue; }
+                        double acc = 0.0;
+                        for (int64_t d = 0; d < D; d++) acc += qi[d] * kp[j * D + d];
+                        s[j] = scale * acc;
+                    }
+                    double m, den;
+                    oracle_safe_softmax(s, L_k, p, &den, &m);
+                    /* dP_ij = dO_i . V_j, delta_i = sum_j P_ij dP_ij */
+                    double delta = 0.0;
+                    for (int64_t j = 0; j < L_k; j++) {
+                        double acc = 0.0;
+                        if (p[j] != 0.0)
+                            for (int64_t d = 0; d < D; d++) acc += doi[d] * vp[j * D + d];
+                        dp[j] = acc;
+                        delta += p[j] * acc;
+                    }
+                    for (int64_t j = 0; j < L_k; j++)
+                        ds[j] = p[j] * (dp[j] - delta);
+                    const double e = delta_err ? delta_err[row] : 0.0;
+                    double *dqi = dq + row * D;
+                    double *dqa = dq_abs ? dq_abs + row * D : NULL;
+                    for (int64_t d = 0; d < D; d++) {
+                        dqi[d] = 0.0;
+                        if (dqa) dqa[d] = 0.0;
+                    }
+                    for (int64_t j = 0; j < L_k; j++) {
+                        if (p[j] == 0.0) continue;
+                        const double wabs_j = fabs(ds[j]) + p[j] * e;
+                        for (int64_t d = 0; d < D; d++) {
+                            dqi[d] += scale * ds[j] * kp[j * D + d];
+                            dkp[j * D + d] += scale * ds[j] * qi[d];
+                            dvp[j * D + d] += p[j] * doi[d];
+                            if (dqa) dqa[d] += scale * wabs_j * fabs(kp[j * D + d]);
+                            if (dka) dka[j * D + d] += scale * wabs_j * fabs(qi[d]);
+                            if (dva) dva[j * D + d] += p[j] * fabs(doi[d]);
+                        }
+                    }
+                }
+        }
+        free(s);
+        free(p);
+        free(dp);
+        free(ds);
+    }
+    return used;
+}

@@ -2,7 +2,8 @@
 
 Each case copies attention_ref.c, plants one plausible mistake (a transposed
 operand, a wrong head map, a dropped scale, an off-by-one mask, a wrong log
-base, a wrong exponent bias, the wrong rounding rule), builds the copy with
+base, a wrong exponent bias, the wrong rounding rule; in the backward a
+dropped delta term, a wrong operand, a missing head of the group), builds the copy with
 gcc and runs the pins against it: at least one pin must fail.  The planted
 copies live in a temporary directory; the committed oracle is untouched."""
 import os
@@ -10,6 +11,7 @@ import os
 import pytest
 
 import oracle
+import tests.test_oracle_bwd_pins as bwd_pins
 import tests.test_oracle_pins as pins
 from exact_attention_113_b200.inputs import F16, BF16
 
@@ -22,7 +24,7 @@ MUTATIONS = {
                   "o[d] += p[j] * tab[kp[j * D + d]];"),
     "gqa_modulo": ("int64_t g = h / group;                       /* GQA head map */",
                    "int64_t g = h % H_kv;"),
-    "scale_dropped": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "scale_dropped": ("\n                s[j] = scale * acc;", "\n                s[j] = acc;"),
     "window_off_by_one": ("if (wl >= 0 && j < i - wl) return 0;",
                           "if (wl >= 0 && j <= i - wl) return 0;"),
     "causal_off_by_one": ("if (causal && j > i) return 0;",
@@ -39,6 +41,23 @@ MUTATIONS = {
                     "w[d] += p[j] * tab[vp[j * D + d]];"),
     "online_stale_max": ("d = d * exp(m - m_new) + exp(x[i] - m_new);",
                          "d = d + exp(x[i] - m_new);"),
+    # backward
+    "bwd_delta_dropped": ("ds[j] = p[j] * (dp[j] - delta);", "ds[j] = p[j] * dp[j];"),
+    "bwd_dk_reads_k": ("dkp[j * D + d] += scale * ds[j] * qi[d];",
+                       "dkp[j * D + d] += scale * ds[j] * kp[j * D + d];"),
+    "bwd_dq_scale_dropped": ("dqi[d] += scale * ds[j] * kp[j * D + d];",
+                             "dqi[d] += ds[j] * kp[j * D + d];"),
+    "bwd_dv_uses_ds": ("dvp[j * D + d] += p[j] * doi[d];", "dvp[j * D + d] += ds[j] * doi[d];"),
+    "bwd_dp_reads_k": ("if (p[j] != 0.0)\n                            for (int64_t d = 0; d < D; d++) acc += doi[d] * vp[j * D + d];",
+                       "if (p[j] != 0.0)\n                            for (int64_t d = 0; d < D; d++) acc += doi[d] * kp[j * D + d];"),
+    "bwd_group_last_head_only": ("for (int64_t h = g * group; h < (g + 1) * group; h++)",
+                                 "for (int64_t h = (g + 1) * group - 1; h < (g + 1) * group; h++)"),
+    "bwd_abs_signed": ("if (dva) dva[j * D + d] += p[j] * fabs(doi[d]);",
+                       "if (dva) dva[j * D + d] += p[j] * doi[d];"),
+    "bwd_abs_delta_term_dropped": ("const double wabs_j = fabs(ds[j]) + p[j] * e;",
+                                   "const double wabs_j = fabs(ds[j]);"),
+    "f64_forward_wrong_head": ("const double *kp = k + (b * H_kv + h / group) * L_k * D;\n            const double *vp",
+                               "const double *kp = k + (b * H_kv + h % H_kv) * L_k * D;\n            const double *vp"),
 }
 
 
@@ -60,6 +79,17 @@ def _battery(orc):
     yield lambda: pins.test_shifting_every_key(orc)
     yield lambda: pins.test_fully_masked_rows(orc)
     yield lambda: pins.test_weighted_abs_value_closed_forms(orc)
+    for c in bwd_pins.CASES:
+        yield lambda c=c: bwd_pins.test_finite_differences_of_the_forward(orc, c)
+        yield lambda c=c: bwd_pins.test_matches_torch_fp64_autograd(orc, c)
+    yield lambda: bwd_pins.test_single_key(orc)
+    yield lambda: bwd_pins.test_scale_zero(orc)
+    yield lambda: bwd_pins.test_constant_values(orc)
+    yield lambda: bwd_pins.test_gqa_gradient_sums_the_group(orc)
+    yield lambda: bwd_pins.test_linear_in_dout(orc)
+    for dt in (F16, BF16):
+        yield lambda dt=dt: bwd_pins.test_bit_pattern_entry_decodes_exactly(orc, dt)
+    yield lambda: bwd_pins.test_error_scales(orc)
 
 
 def _first_failure(orc):
