@@ -23,8 +23,9 @@ STATUS = {
     -4: "FA_ERR_DTYPE", -5: "FA_ERR_ALIGN", -6: "FA_ERR_ARG", -7: "FA_ERR_CUDA",
     -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE", -10: "FA_ERR_SCRATCH",
 }
-EXPORTS = ("fa_fwd", "fa_fwd_splitkv", "fa_fwd_splitkv_static", "fa_get_device_status",
-           "fa_splitkv_workspace_bytes", "fa_status_string", "fa_version")
+EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_splitkv",
+           "fa_fwd_splitkv_static", "fa_get_device_status", "fa_splitkv_workspace_bytes",
+           "fa_status_string", "fa_version")
 # size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -62,6 +63,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd_splitkv_static.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i,
                                               ctypes.c_float, i, i, i, i, i, vp]
         lib.fa_fwd_splitkv_static.restype = i
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                               ctypes.c_float, i, i, i, i, vp, ctypes.c_size_t, vp]
+        lib.fa_bwd.restype = i
+        lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_get_device_status.argtypes = [vp]
@@ -100,6 +106,18 @@ def fa_fwd_splitkv_static(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, cau
     return load().fa_fwd_splitkv_static(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D,
                                         float(scale), int(causal), int(window_left),
                                         int(window_right), int(dtype), int(n_splits), stream)
+
+
+def fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, H_kv, L_q, L_k, D, scale, causal,
+           window_left, window_right, dtype, workspace, workspace_bytes, stream) -> int:
+    """The backward C entry point, unchanged."""
+    return load().fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, H_kv, L_q, L_k, D,
+                         float(scale), int(causal), int(window_left), int(window_right),
+                         int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_bwd_workspace_bytes(B, H, L_q, D) -> int:
+    return int(load().fa_bwd_workspace_bytes(B, H, L_q, D))
 
 
 def fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits) -> int:
@@ -220,3 +238,46 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
     if st != FA_OK:
         raise FaError(st, where)
     return out, lse
+
+
+def flash_bwd(q, k, v, out, dout, lse, scale=None, causal=False, window_left=-1,
+              window_right=-1, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Exact attention backward on CUDA tensors: returns (dq, dk, dv).
+
+    q, out, dout: [B, H, L_q, D]; k, v: [B, H_kv, L_k, D]; lse: [B, H, L_q]
+    fp32 from the forward (same scale and mask).  The workspace is allocated
+    here with torch unless given (a uint8 CUDA tensor, 256-byte aligned)."""
+    import torch
+
+    B, H, L_q, D = q.shape
+    _, H_kv, L_k, _ = k.shape
+    for name, t, shape in (("out", out, q.shape), ("dout", dout, q.shape), ("v", v, k.shape)):
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}")
+    if tuple(lse.shape) != (B, H, L_q) or lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32 [B, H, L_q]")
+    if q.dtype not in (torch.float16, torch.bfloat16) or any(
+            t.dtype != q.dtype for t in (k, v, out, dout)):
+        raise TypeError("q, k, v, out, dout must share dtype float16 or bfloat16")
+    ts = (q, k, v, out, dout, lse)
+    if not all(t.is_cuda for t in ts) or not all(t.is_contiguous() for t in ts):
+        raise ValueError("inputs must be contiguous CUDA tensors")
+    dtype = FA_F16 if q.dtype == torch.float16 else FA_BF16
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(fa_bwd_workspace_bytes(B, H, L_q, D), 1), dtype=torch.uint8,
+                                device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv,
+                    L_q, L_k, D, scale, causal, window_left, window_right, dtype,
+                    workspace.data_ptr(), workspace.numel(), stream.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv

@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libfa.so")
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "fa_fwd_kernel.cuh")] + [
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "fa_fwd_kernel.cuh",
+                                                     "fa_bwd_kernel.cuh")] + [
     os.path.join(INCLUDE, "fa.h")]
 
 NVCC_FLAGS = [
@@ -46,12 +47,14 @@ def is_stale() -> bool:
 # The attention kernel launches 384 threads and re-splits its registers with
 # setmaxnreg (2 warpgroups x 224 + 1 x 56 = 384 x 168).  That split is only
 # valid when every instance is compiled at exactly this many registers.
-LAUNCH_REGS = 168
-KERNEL_TAG = "fa_fwd_kernel"
+# kernels whose warpgroups re-split registers with setmaxnreg: the launch
+# allocation (registers per thread) each must be compiled at
+LAUNCH_REGS = {"fa_fwd_kernel": 168, "fa_bwd_kernel": 128}
 
 
 def check_register_counts(ptxas_log: str) -> dict:
-    """Parse `ptxas -v` output; require LAUNCH_REGS for every kernel instance."""
+    """Parse `ptxas -v` output; require LAUNCH_REGS for every instance of
+    each setmaxnreg kernel (forward and backward)."""
     counts, current = {}, None
     for line in ptxas_log.splitlines():
         m = re.search(r"Function properties for (\S+)", line)
@@ -63,14 +66,16 @@ def check_register_counts(ptxas_log: str) -> dict:
             current = m.group(1)
             continue
         m = re.search(r"Used (\d+) registers", line)
-        if m and current and KERNEL_TAG in current:
+        if m and current and any(tag in current for tag in LAUNCH_REGS):
             counts[current] = int(m.group(1))
-    if not counts:
-        raise RuntimeError("no register counts found for the attention kernel")
-    bad = {k: v for k, v in counts.items() if v != LAUNCH_REGS}
+    for tag in LAUNCH_REGS:
+        if not any(tag in k for k in counts):
+            raise RuntimeError(f"no register counts found for {tag}")
+    bad = {k: v for k, v in counts.items()
+           for tag, want in LAUNCH_REGS.items() if tag in k and v != want}
     if bad:
-        raise RuntimeError(f"attention kernel register count != {LAUNCH_REGS}: {bad}; "
-                           "the setmaxnreg split would not match the launch")
+        raise RuntimeError(f"register counts differ from the launch allocation "
+                           f"{LAUNCH_REGS}: {bad}; the setmaxnreg split would not match")
     return counts
 
 

@@ -6,6 +6,7 @@
 // fp32 softmax statistics of shape [B, H, S]; scale, pre_tokens and
 // next_tokens as attributes.  The statistics here are one log-sum-exp per row
 // (Triton FA2 walkthrough: the logsumexp kept for the backward pass).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -16,6 +17,7 @@
 
 #include "fa.h"
 #include "fa_fwd_kernel.cuh"
+#include "fa_bwd_kernel.cuh"
 
 namespace fa {
 namespace {
@@ -338,6 +340,156 @@ extern "C" int fa_fwd_splitkv(const void *q, const void *k, const void *v, void 
   if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
                   window_right, dtype, n_splits, workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Backward.  Workspace: dQ accumulator [B*H][L_q][D] fp32, then lse2 and
+// delta [B*H][L_q_pad] fp32 (L_q_pad = L_q rounded up to 128), each part at
+// a 256-byte boundary.
+namespace fa {
+namespace {
+struct BwdWs {
+  size_t dq_off, lse2_off, delta_off, total;
+};
+BwdWs bwd_ws(int64_t BH, int64_t L_q, int D) {
+  const int64_t L_q_pad = (L_q + kBM - 1) / kBM * kBM;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  BwdWs w;
+  w.dq_off = 0;
+  w.lse2_off = up(static_cast<size_t>(BH) * L_q * D * sizeof(float));
+  w.delta_off = w.lse2_off + up(static_cast<size_t>(BH) * L_q_pad * sizeof(float));
+  w.total = w.delta_off + up(static_cast<size_t>(BH) * L_q_pad * sizeof(float));
+  return w;
+}
+
+template <int D, int DT>
+int launch_bwd(const BwdParams &prm, const void *out, const void *dout, const float *lse,
+               void *dq, int B, int H, cudaStream_t stream) {
+  using BG = BwdGeo<D>;
+  auto kern = fa_bwd_kernel<D, DT>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  static bool configured[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    if (!configured[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BG::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+      configured[dev] = true;
+    }
+  }
+  const long long rows_pad = static_cast<long long>(B) * H * prm.L_q_pad;
+  fa_bwd_prep_kernel<D, DT><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, stream>>>(
+      out, dout, lse, const_cast<float *>(prm.lse2), const_cast<float *>(prm.delta),
+      prm.dq_acc, prm.L_q, prm.L_q_pad, rows_pad);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(B) * prm.H_kv * prm.n_kblocks;
+  kern<<<grid, kBwdThreads, BG::kSmemBytes, stream>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const size_t n = static_cast<size_t>(B) * H * prm.L_q * D;
+  const unsigned cblocks = static_cast<unsigned>(std::min<size_t>((n / 2 + 255) / 256, 148 * 16));
+  fa_bwd_dq_kernel<DT><<<cblocks, 256, 0, stream>>>(prm.dq_acc, dq, n);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" size_t fa_bwd_workspace_bytes(int B, int H, int L_q, int D) {
+  if (B < 1 || H < 1 || L_q < 0 || L_q > fa::kMaxSeq) return 0;
+  if (D != 16 && D != 32 && D != 64 && D != 128) return 0;
+  return fa::bwd_ws(static_cast<int64_t>(B) * H, L_q, D).total;
+}
+
+extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *out,
+                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                      int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
+                      int window_left, int window_right, int dtype, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream) {
+  using namespace fa;
+  if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
+  if (H % H_kv != 0) return FA_ERR_SHAPE;
+  if (L_q > kMaxSeq || L_k > kMaxSeq) return FA_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * H_kv * ((static_cast<int64_t>(L_k) + 127) / 128) >
+      (1ll << 31) - 1)
+    return FA_ERR_SHAPE;
+  if (D != 16 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  const bool nq = L_q > 0, nk = L_k > 0;
+  if ((nq && (!q || !out || !dout || !dq)) || (nk && (!k || !v || !dk || !dv)) ||
+      (nq && nk && (!lse || !workspace)))
+    return FA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return FA_ERR_ALIGN;
+  if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+  const int64_t BH = static_cast<int64_t>(B) * H;
+  const BwdWs ws = bwd_ws(BH, L_q, D);
+  if (nq && nk && workspace_bytes < ws.total) return FA_ERR_WORKSPACE;
+
+  // ---------------------------------------------------------------- edges
+  if (!nq && !nk) return FA_OK;
+  if (!nq) {   // no query: no gradient reaches K or V
+    const size_t bytes = static_cast<size_t>(B) * H_kv * L_k * D * 2;
+    if (cudaMemsetAsync(dk, 0, bytes, stream) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, bytes, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  if (!nk) {   // no key: O = 0 does not depend on Q
+    if (cudaMemsetAsync(dq, 0, static_cast<size_t>(BH) * L_q * D * 2, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+
+  // ---------------------------------------------------------------- params
+  BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  int wl = window_left < 0 ? -1 : window_left;
+  int wr = window_right < 0 ? -1 : window_right;
+  if (causal) wr = 0;
+  if (wl >= L_q) wl = -1;
+  if (wr >= L_k) wr = -1;
+  prm.H = H;
+  prm.H_kv = H_kv;
+  prm.L_q = L_q;
+  prm.L_k = L_k;
+  prm.L_q_pad = static_cast<int>((static_cast<int64_t>(L_q) + kBM - 1) / kBM * kBM);
+  prm.group = H / H_kv;
+  prm.n_kblocks = (L_k + kBN - 1) / kBN;
+  prm.wl = wl;
+  prm.wr = wr;
+  {
+    float sl2 = scale * 1.4426950408889634f;
+    prm.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;
+  }
+  prm.scale = scale;
+  char *wsb = static_cast<char *>(workspace);
+  prm.dq_acc = reinterpret_cast<float *>(wsb + ws.dq_off);
+  prm.lse2 = reinterpret_cast<const float *>(wsb + ws.lse2_off);
+  prm.delta = reinterpret_cast<const float *>(wsb + ws.delta_off);
+  prm.dk = dk;
+  prm.dv = dv;
+  const int box_cols = D * 2 >= 128 ? 64 : D;
+  if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
+      !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
+      !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
+      !encode_map(&prm.tm_do, dout, dtype, B * H, L_q, D, box_cols))
+    return FA_ERR_CUDA;
+  switch (D * 2 + dtype) {
+    case 32: return launch_bwd<16, 0>(prm, out, dout, lse, dq, B, H, stream);
+    case 33: return launch_bwd<16, 1>(prm, out, dout, lse, dq, B, H, stream);
+    case 64: return launch_bwd<32, 0>(prm, out, dout, lse, dq, B, H, stream);
+    case 65: return launch_bwd<32, 1>(prm, out, dout, lse, dq, B, H, stream);
+    case 128: return launch_bwd<64, 0>(prm, out, dout, lse, dq, B, H, stream);
+    case 129: return launch_bwd<64, 1>(prm, out, dout, lse, dq, B, H, stream);
+    case 256: return launch_bwd<128, 0>(prm, out, dout, lse, dq, B, H, stream);
+    case 257: return launch_bwd<128, 1>(prm, out, dout, lse, dq, B, H, stream);
+  }
+  return FA_ERR_HEADDIM;
 }
 
 // ---------------------------------------------------------------------------

@@ -1,0 +1,556 @@
+// fa_bwd_kernel.cuh -- exact attention backward for sm_100a (B200).
+//
+// The pages keep only the softmax statistics from the forward and recompute
+// the attention matrix from Q, K, V when the gradients are taken
+// ("FlashAttention算法原理与性能优化实战" §1.2.3; "Flash Attention是怎么做到又快又省
+// 显存的？" 总结; the Triton FA2 walkthrough keeps the logsumexp for this).  The
+// gradients themselves follow from the chain rule through O = P V,
+// P = softmax(S), S = scale Q K^T:
+//     dV = P^T dO,   dP = dO V^T,   dS = P o (dP - delta),
+//     delta_i = dO_i . O_i  (= sum_j P_ij dP_ij),
+//     dQ = scale dS K,   dK = scale dS^T Q.
+//
+// One CTA owns one block of 128 keys of one (batch, K/V head) and walks the
+// query blocks that can see it, for every query head of the GQA group, so
+// that dK and dV accumulate in TMEM with no atomics.  Per step (one 128-row
+// query block) five tcgen05 MMAs:
+//     S^T  = K Q^T      (SS; keys on TMEM lanes, queries along columns)
+//     dP^T = V dO^T     (SS)
+//     dV  += P^T dO     (TS: P^T from TMEM, dO MN-major from shared memory)
+//     dK  += dS^T Q     (TS: dS^T from TMEM)
+//     dQ   = dS K       (SS: dS staged in shared memory MN-major, K MN-major)
+// dQ of the step is added into an fp32 accumulator in global memory by a
+// warpgroup of its own (vector atomic adds); the other key blocks add theirs.
+//
+// Roles (512 threads): warpgroups 0 and 1 compute P and dS for query
+// columns [0, 64) and [64, 128) of every key row (thread = TMEM lane = key);
+// warp 8 issues the MMAs, warp 9 is the TMA producer; warpgroup 3 drains dQ
+// (thread = TMEM lane = query row).
+//
+// TMEM (512 columns): S^T [0,128) with P^T (two 16-bit values per column)
+// written over the first half of each warpgroup's columns; dP^T [128,256)
+// with dS^T likewise; dQ [128, 128+D) after dK has read dS^T (tcgen05 MMAs
+// of one thread run in order); dV [256, 256+D); dK [256+D, 256+2D).
+//
+// Every wait is bounded (sm100.cuh); after a timeout each role leaves its
+// loop, the producer lets its copies land, and TMEM is freed.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  CUtensorMap tm_q;    // [B*H,    L_q, D]
+  CUtensorMap tm_k;    // [B*H_kv, L_k, D]
+  CUtensorMap tm_v;    // [B*H_kv, L_k, D]
+  CUtensorMap tm_do;   // [B*H,    L_q, D]
+  const float *lse2;   // [B*H][L_q_pad]: lse * log2(e); +inf where no key is visible / past L_q
+  const float *delta;  // [B*H][L_q_pad]: dO_i . O_i; 0 past L_q
+  float *dq_acc;       // [B*H][L_q][D] fp32, zero before the launch
+  void *dk;            // [B*H_kv][L_k][D]
+  void *dv;            // [B*H_kv][L_k][D]
+  int H, H_kv, L_q, L_k, L_q_pad, group;
+  int n_kblocks;       // ceil(L_k / 128)
+  int wl, wr;          // visible iff i - wl <= j <= i + wr; -1 = unbounded
+  float scale_log2;    // scale * log2(e), clamped to >= 1e-30
+  float scale;
+};
+
+constexpr int kBwdThreads = 512;
+constexpr uint32_t kBwdLaunchRegs = 128;   // 65536 / 512
+// setmaxnreg split: P/dS warpgroups, dQ drain warpgroup, MMA/TMA warpgroup;
+// 2 * 144 + 168 + 56 = 4 * 128 (the launch allocation)
+constexpr uint32_t kBwdRegsPds = 144;
+constexpr uint32_t kBwdRegsDrain = 168;
+constexpr uint32_t kBwdRegsIssue = 56;
+static_assert(2 * kBwdRegsPds + kBwdRegsDrain + kBwdRegsIssue == 4 * kBwdLaunchRegs,
+              "register split must fit in the launch allocation");
+
+template <int D>
+struct BwdGeo {
+  using G = Geo<D>;
+  static constexpr int kTileBytes = G::kTileBytes;        // 128 rows x D, TMA-swizzled
+  static constexpr int kDsBoxBytes = 128 * 128;           // [128 keys][64 queries] 16-bit, SW128
+  static constexpr int kDsBytes = 2 * kDsBoxBytes;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;            // two stages
+  static constexpr int kOffDo = 4 * kTileBytes;           // two stages
+  static constexpr int kOffDs = 6 * kTileBytes;
+  static constexpr int kOffVec = kOffDs + kDsBytes;       // lse2[128], delta[128]
+  static constexpr int kOffBar = kOffVec + 256 * 4;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kUsed = kOffBar + kBarBytes;
+  // at least ~116 KB: one CTA (one 512-column TMEM allocation) per SM
+  static constexpr int kSmemBytes = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(256 + 2 * D <= 512, "TMEM budget");
+};
+
+struct BwdBars {
+  uint64_t kv_full;
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t s_full;
+  uint64_t dp_full;
+  uint64_t p_full;
+  uint64_t ds_full;
+  uint64_t dq_full;
+  uint64_t dq_free;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Query blocks [lo, hi) that can see any key of key block kb.
+__device__ __forceinline__ void bwd_query_range(int kb, int L_q, int L_k, int wl, int wr,
+                                                int &lo, int &hi) {
+  const int k0 = kb * kBN;
+  const int k1 = min(L_k - 1, k0 + kBN - 1);
+  const int i_lo = wr < 0 ? 0 : max(0, k0 - wr);
+  const int i_hi = wl < 0 ? L_q - 1 : min(L_q - 1, k1 + wl);
+  if (L_q <= 0 || i_hi < i_lo) {
+    lo = hi = 0;
+  } else {
+    lo = i_lo / kBM;
+    hi = i_hi / kBM + 1;
+  }
+}
+
+template <int D, int DT>
+__global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using G = Geo<D>;
+  using BG = BwdGeo<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  BwdBars *bars = reinterpret_cast<BwdBars *>(smem + BG::kOffBar);
+  volatile int *abort_flag = &bars->abort_flag;
+  float *s_vec = reinterpret_cast<float *>(smem + BG::kOffVec);   // lse2[128] | delta[128]
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+
+  // ---- work item: (batch, K/V head, key block)
+  const int kb = static_cast<int>(blockIdx.x) % p.n_kblocks;
+  const int bh_kv = static_cast<int>(blockIdx.x) / p.n_kblocks;
+  const int b = bh_kv / p.H_kv;
+  const int hk = bh_kv - b * p.H_kv;
+  const int k0 = kb * kBN;
+  int qb_lo, qb_hi;
+  bwd_query_range(kb, p.L_q, p.L_k, p.wl, p.wr, qb_lo, qb_hi);
+  const int nqb = qb_hi - qb_lo;
+  const int n_steps = nqb * p.group;          // (query head, query block) pairs
+  // step n: query head bh_of(n), first query row q0_of(n)
+  auto bh_of = [&](int n) { return b * p.H + hk * p.group + n / max(nqb, 1); };
+  auto q0_of = [&](int n) { return (qb_lo + n % max(nqb, 1)) * kBM; };
+
+  // ---- setup
+  if (tid == 0) {
+    mbar_init(smem_u32(&bars->kv_full), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->q_full[s]), 1);
+      mbar_init(smem_u32(&bars->q_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->dp_full), 1);
+    mbar_init(smem_u32(&bars->p_full), 256);
+    mbar_init(smem_u32(&bars->ds_full), 256);
+    mbar_init(smem_u32(&bars->dq_full), 1);
+    mbar_init(smem_u32(&bars->dq_free), 128);
+    mbar_init(smem_u32(&bars->mma_done), 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 9 && (tid & 31) == 0) {
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_k);
+    prefetch_tensormap(&p.tm_v);
+    prefetch_tensormap(&p.tm_do);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t sK = smem_u32(smem + BG::kOffK);
+  const uint32_t sV = smem_u32(smem + BG::kOffV);
+  const uint32_t sQ = smem_u32(smem + BG::kOffQ);
+  const uint32_t sDo = smem_u32(smem + BG::kOffDo);
+  const uint32_t sDs = smem_u32(smem + BG::kOffDs);
+
+  if (warp >= 8 && warp < 12) {
+  // ===================================================== warpgroup 2
+  regs_dec<kBwdRegsIssue>();
+  if (warp == 9) {
+    // =================================================== TMA producer
+    const uint64_t pol_keep = policy_evict_last();
+    int issued = 0;
+    bool ok = true;
+    if (n_steps > 0) {
+      const uint32_t bar = smem_u32(&bars->kv_full);
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar, 2 * G::kTileBytes);
+#pragma unroll
+        for (int bx = 0; bx < G::kNumBox; ++bx) {
+          tma_load_3d(sK + bx * G::kBoxBytes, &p.tm_k, bar, bx * G::kBoxCols, k0, bh_kv, pol_keep);
+          tma_load_3d(sV + bx * G::kBoxBytes, &p.tm_v, bar, bx * G::kBoxCols, k0, bh_kv, pol_keep);
+        }
+      }
+      __syncwarp();
+      for (int n = 0; n < n_steps; ++n) {
+        const int st = n & 1;
+        if (n >= 2) {
+          ok = mbar_wait_warp(smem_u32(&bars->q_empty[st]), ((n >> 1) - 1) & 1, abort_flag);
+          if (!ok) break;
+        }
+        const uint32_t qb = smem_u32(&bars->q_full[st]);
+        const int q0 = q0_of(n), bh = bh_of(n);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(qb, 2 * G::kTileBytes);
+#pragma unroll
+          for (int bx = 0; bx < G::kNumBox; ++bx) {
+            tma_load_3d(sQ + st * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, qb,
+                        bx * G::kBoxCols, q0, bh, pol_keep);
+            tma_load_3d(sDo + st * G::kTileBytes + bx * G::kBoxBytes, &p.tm_do, qb,
+                        bx * G::kBoxCols, q0, bh, pol_keep);
+          }
+        }
+        __syncwarp();
+        issued = n + 1;
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA exits
+        mbar_wait_slow(smem_u32(&bars->kv_full), 0, abort_flag, false);
+        for (int n = max(0, issued - 2); n < issued; ++n)
+          mbar_wait_slow(smem_u32(&bars->q_full[n & 1]), (n >> 1) & 1, abort_flag, false);
+      }
+    }
+  } else if (warp == 8) {
+    // =================================================== MMA issuer
+    constexpr uint32_t kIdescS = make_idesc_f16(kBN, kBM, DT, 0, 0);      // M keys, N queries
+    constexpr uint32_t kIdescKV = make_idesc_f16(kBN, D, DT, 0, 1);       // dV, dK (A in TMEM)
+    constexpr uint32_t kIdescQ = make_idesc_f16(kBM, D, DT, 1, 1);        // dQ (A MN-major)
+    constexpr uint32_t kHi = desc_hi(8 * G::kSwBytes, G::kLayout);
+    constexpr uint32_t kHiDs = desc_hi(1024, 2u);                         // SW128
+    const uint32_t tS = tmem, tDP = tmem + 128u, tDV = tmem + 256u, tDK = tmem + 256u + D;
+    const uint32_t tDQ = tmem + 128u;
+    if (n_steps > 0) {
+      bool ok = mbar_wait_warp(smem_u32(&bars->kv_full), 0, abort_flag);
+      // X^T = A B^T over D with A, B K-major 128 x D tiles (A: K or V; B: Q or dO)
+      auto issue_kmajor = [&](uint32_t d_tmem, uint32_t a_tile, uint32_t b_tile, uint32_t bar) {
+        const uint32_t alo = desc_lo(a_tile, 16), blo = desc_lo(b_tile, 16);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int byte = kk * 32;
+            const uint32_t off = ((byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes)) >> 4;
+            mma_ss(d_tmem, desc_join(alo + off, kHi), desc_join(blo + off, kHi), kIdescS,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar);
+        }
+        __syncwarp();
+      };
+      // D_acc += X^T(TMEM, 16-bit, two warpgroups' halves) * B (MN-major tile)
+      auto issue_ts = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_tile, bool first) {
+        const uint32_t blo = desc_lo(b_tile, G::kBoxBytes);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kBM / 16; ++kk) {
+            const uint32_t a = a_base + (kk >> 2) * 64u + (kk & 3) * 8u;
+            mma_ts(d_tmem, a, desc_join(blo + ((kk * 16 * G::kSwBytes) >> 4), kHi), kIdescKV,
+                   (!first || kk > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+      };
+      auto commit = [&](uint32_t bar) {
+        if (elect_one()) tc_commit(bar);
+        __syncwarp();
+      };
+      if (ok) ok = mbar_wait_warp(smem_u32(&bars->q_full[0]), 0, abort_flag);
+      if (ok) {
+        tc_fence_after_sync();
+        issue_kmajor(tS, sK, sQ, smem_u32(&bars->s_full));
+        issue_kmajor(tDP, sV, sDo, smem_u32(&bars->dp_full));
+      }
+      for (int n = 0; n < n_steps && ok; ++n) {
+        const int st = n & 1;
+        ok = mbar_wait_warp(smem_u32(&bars->p_full), n & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_ts(tDV, tS, sDo + st * G::kTileBytes, n == 0);
+        if (n + 1 < n_steps) {
+          const int st1 = (n + 1) & 1;
+          ok = mbar_wait_warp(smem_u32(&bars->q_full[st1]), ((n + 1) >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_kmajor(tS, sK, sQ + st1 * G::kTileBytes, smem_u32(&bars->s_full));
+        }
+        ok = mbar_wait_warp(smem_u32(&bars->ds_full), n & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_ts(tDK, tDP, sQ + st * G::kTileBytes, n == 0);
+        {
+          // dQ = dS K: A = dS [128 q][128 keys] MN-major (two 64-query boxes),
+          // B = K [128 keys][D] MN-major
+          const uint32_t alo = desc_lo(sDs, BG::kDsBoxBytes);
+          const uint32_t blo = desc_lo(sK, G::kBoxBytes);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              mma_ss(tDQ, desc_join(alo + ((kk * 16 * 128) >> 4), kHiDs),
+                     desc_join(blo + ((kk * 16 * G::kSwBytes) >> 4), kHi), kIdescQ,
+                     kk > 0 ? 1u : 0u);
+          }
+          __syncwarp();
+        }
+        commit(smem_u32(&bars->dq_full));
+        commit(smem_u32(&bars->q_empty[st]));
+        if (n + 1 < n_steps) {
+          ok = mbar_wait_warp(smem_u32(&bars->dq_free), n & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_kmajor(tDP, sV, sDo + ((n + 1) & 1) * G::kTileBytes, smem_u32(&bars->dp_full));
+        }
+      }
+    }
+    if (elect_one()) tc_commit(smem_u32(&bars->mma_done));
+    __syncwarp();
+  }
+  } else if (warp < 8) {
+    // =================================================== P and dS
+    regs_inc<kBwdRegsPds>();
+    const int wg = warp >> 2;                      // query columns [64 wg, 64 wg + 64)
+    const int r = tid & 127;                       // key row = TMEM lane
+    const int tc = tid;                            // 0..255: slot in the lse2 / delta buffer
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + 64u * wg;
+    const uint32_t tDP = tmem + lane_base + 128u + 64u * wg;
+    const int j = k0 + r;                          // key index of this row
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    // lse2 / delta of the next step, one value per thread
+    auto fetch = [&](int n) -> float {
+      const size_t base = static_cast<size_t>(bh_of(n)) * p.L_q_pad + q0_of(n) + (tc & 127);
+      return tc < 128 ? p.lse2[base] : p.delta[base];
+    };
+    float nxt = n_steps > 0 ? fetch(0) : 0.0f;
+    // Every warp of both warpgroups passes the two named barriers of every
+    // step, also after a timeout (then the step's work is skipped).
+    for (int n = 0; n < n_steps; ++n) {
+      named_barrier_sync(1, 256);                  // the buffer of step n-1 is no longer read
+      s_vec[tc] = nxt;
+      named_barrier_sync(1, 256);
+      if (n + 1 < n_steps) nxt = fetch(n + 1);
+      if (!ok) continue;
+      const int q0 = q0_of(n);
+      const int qc = q0 + 64 * wg;                 // first query column of this thread
+      const bool full = (k0 + kBN - 1 < p.L_k) && (p.wr < 0 || k0 + kBN - 1 <= q0 + p.wr) &&
+                        (p.wl < 0 || k0 >= q0 + kBM - 1 - p.wl);
+      const float *lse2 = s_vec + 64 * wg;
+      const float *dlt = s_vec + 128 + 64 * wg;
+
+      // ---- P^T = 2^(s * scale * log2e - lse2), masked entries 0
+      ok = mbar_wait_warp(smem_u32(&bars->s_full), n & 1, abort_flag);
+      if (!ok) continue;
+      tc_fence_after_sync();
+      float pr[64];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[32];
+        tmem_ld_x32(tS + 32 * h, sr);
+        tmem_wait_ld();
+        reg_dep(sr);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          pr[32 * h + c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse2[32 * h + c]));
+      }
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int i = qc + c;
+          const bool vis = (j < p.L_k) && (p.wr < 0 || j <= i + p.wr) && (p.wl < 0 || j >= i - p.wl);
+          if (!vis) pr[c] = 0.0f;
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) pk[u] = pack2<DT>(pr[2 * u], pr[2 * u + 1]);
+        tmem_st_x32(tS, pk);                       // over S^T columns already read
+        tmem_wait_st();
+      }
+      tc_fence_before_sync();
+      mbar_arrive(smem_u32(&bars->p_full));
+
+      // ---- dS = P o (dP - delta) * scale, to TMEM (for dK) and shared memory (for dQ)
+      ok = mbar_wait_warp(smem_u32(&bars->dp_full), n & 1, abort_flag);
+      if (!ok) continue;
+      tc_fence_after_sync();
+      if (n > 0) {
+        // the dQ MMA of the previous step has read the dS staging buffer
+        ok = mbar_wait_warp(smem_u32(&bars->dq_full), (n - 1) & 1, abort_flag);
+        if (!ok) continue;
+      }
+      uint8_t *ds_row = smem + BG::kOffDs + wg * BG::kDsBoxBytes + r * 128;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t dp[32];
+        tmem_ld_x32(tDP + 32 * h, dp);
+        tmem_wait_ld();
+        reg_dep(dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int c = 32 * h + 2 * u;
+          const float d0 = pr[c] * (__uint_as_float(dp[2 * u]) - dlt[c]) * p.scale;
+          const float d1 = pr[c + 1] * (__uint_as_float(dp[2 * u + 1]) - dlt[c + 1]) * p.scale;
+          pk[u] = pack2<DT>(d0, d1);
+        }
+        tmem_st_x16(tDP + 16 * h, pk);             // over dP^T columns already read
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = 4 * h + u;              // 16-byte unit of the 128-byte row
+          *reinterpret_cast<uint4 *>(ds_row + ((unit ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      mbar_arrive(smem_u32(&bars->ds_full));
+    }
+
+    // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 dK (row j of this block)
+    if (ok && n_steps > 0) {
+      ok = mbar_wait_warp(smem_u32(&bars->mma_done), 0, abort_flag);
+      if (ok) tc_fence_after_sync();
+    }
+    if (ok) {
+      const uint32_t tAcc = tmem + lane_base + 256u + (wg ? D : 0);
+      uint8_t *dst = static_cast<uint8_t *>(wg ? p.dk : p.dv) +
+                     (static_cast<size_t>(bh_kv) * p.L_k + j) * D * 2;
+      constexpr int kChunk = D >= 32 ? 32 : D;
+#pragma unroll
+      for (int c = 0; c < D; c += kChunk) {
+        uint32_t o[kChunk];
+        if (n_steps > 0) {
+          tmem_ld_cols<kChunk>(tAcc + c, o);
+          tmem_wait_ld();
+          reg_dep(o);
+        } else {
+#pragma unroll
+          for (int u = 0; u < kChunk; ++u) o[u] = 0u;
+        }
+        if (j < p.L_k) {
+#pragma unroll
+          for (int u = 0; u < kChunk / 8; ++u)
+            *reinterpret_cast<uint4 *>(dst + (c + 8 * u) * 2) = make_uint4(
+                pack2<DT>(__uint_as_float(o[8 * u]), __uint_as_float(o[8 * u + 1])),
+                pack2<DT>(__uint_as_float(o[8 * u + 2]), __uint_as_float(o[8 * u + 3])),
+                pack2<DT>(__uint_as_float(o[8 * u + 4]), __uint_as_float(o[8 * u + 5])),
+                pack2<DT>(__uint_as_float(o[8 * u + 6]), __uint_as_float(o[8 * u + 7])));
+        }
+      }
+    }
+  } else {
+    // =================================================== dQ drain (warps 12-15)
+    regs_inc<kBwdRegsDrain>();
+    const int r = tid & 127;                       // query row within the block = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tDQ = tmem + lane_base + 128u;
+    for (int n = 0; n < n_steps; ++n) {
+      if (!mbar_wait_warp(smem_u32(&bars->dq_full), n & 1, abort_flag)) break;
+      tc_fence_after_sync();
+      const int i = q0_of(n) + r;
+      float *dst = p.dq_acc + (static_cast<size_t>(bh_of(n)) * p.L_q + i) * D;
+      constexpr int kChunk = D >= 32 ? 32 : D;
+      uint32_t acc[D];
+#pragma unroll
+      for (int c = 0; c < D; c += kChunk)
+        tmem_ld_cols<kChunk>(tDQ + c, *reinterpret_cast<uint32_t(*)[kChunk]>(acc + c));
+      tmem_wait_ld();
+      reg_dep(acc);
+      tc_fence_before_sync();
+      mbar_arrive(smem_u32(&bars->dq_free));       // TMEM columns free for dP^T of the next step
+      if (i < p.L_q) {
+#pragma unroll
+        for (int u = 0; u < D / 4; ++u)
+          atomicAdd(reinterpret_cast<float4 *>(dst) + u,
+                    make_float4(__uint_as_float(acc[4 * u]), __uint_as_float(acc[4 * u + 1]),
+                                __uint_as_float(acc[4 * u + 2]), __uint_as_float(acc[4 * u + 3])));
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after_sync();
+    mbar_wait_slow(smem_u32(&bars->mma_done), 0, abort_flag, false);
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// delta_i = dO_i . O_i (fp32), lse2_i = lse_i * log2(e) (+inf where lse is
+// -inf or i >= L_q), and dQ_acc zeroed: one warp per padded query row.
+template <int D, int DT>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const void *out, const void *dout,
+                                                          const float *lse, float *lse2,
+                                                          float *delta, float *dq_acc, int L_q,
+                                                          int L_q_pad, long long rows_pad) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows_pad) return;
+  const long long bh = row / L_q_pad;
+  const int i = static_cast<int>(row - bh * L_q_pad);
+  float dsum = 0.0f;
+  if (i < L_q) {
+    const size_t base = (static_cast<size_t>(bh) * L_q + i) * D;
+    for (int d = lane; d < D; d += 32) {
+      float o, g;
+      if constexpr (DT == 0) {
+        o = __half2float(reinterpret_cast<const __half *>(out)[base + d]);
+        g = __half2float(reinterpret_cast<const __half *>(dout)[base + d]);
+      } else {
+        o = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(out)[base + d]);
+        g = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(dout)[base + d]);
+      }
+      dsum = fmaf(o, g, dsum);
+      dq_acc[base + d] = 0.0f;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+  if (lane == 0) {
+    delta[row] = dsum;
+    float l2 = INFINITY;
+    if (i < L_q) {
+      const float l = lse[static_cast<size_t>(bh) * L_q + i];
+      if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+    }
+    lse2[row] = l2;
+  }
+}
+
+// dQ = dQ_acc rounded to the element type (the scale is already in dS).
+template <int DT>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float *dq_acc, void *dq,
+                                                        size_t n) {
+  size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x * 2;
+  for (; i < n; i += stride) {
+    const float2 v = *reinterpret_cast<const float2 *>(dq_acc + i);
+    reinterpret_cast<uint32_t *>(dq)[i / 2] = pack2<DT>(v.x, v.y);
+  }
+}
+
+}  // namespace fa

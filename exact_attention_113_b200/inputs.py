@@ -59,6 +59,14 @@ def make_qkv(w: Workload, device="cpu"):
     return tuple(out)
 
 
+def make_dout(w: Workload, device="cpu"):
+    """The upstream gradient dO [B,H,L_q,D] for a backward of workload ``w``
+    (seeded N(0, 1), its own stream: seed + 7919)."""
+    g = torch.Generator(device="cpu").manual_seed(int(w.seed) + 7919)
+    x = torch.randn((w.B, w.H, w.L_q, w.D), generator=g, dtype=torch.float32)
+    return x.to(TORCH_DTYPE[w.dtype]).to(device)
+
+
 def to_bits(t: torch.Tensor) -> np.ndarray:
     """A CPU copy of an fp16/bf16 tensor as uint16 bit patterns."""
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -123,6 +123,45 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float
                    cudaStream_t stream);
 
 /*
+ * fa_bwd_workspace_bytes -- bytes of device workspace fa_bwd needs (0 if
+ * the sizes are invalid): an fp32 dQ accumulator [B, H, L_q, D] and two
+ * fp32 row vectors [B, H, roundup(L_q, 128)].
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int L_q, int D);
+
+/*
+ * fa_bwd -- exact attention backward on `stream` (asynchronous): the
+ * gradients of sum(dout .* out) for out = fa_fwd(q, k, v, ...), with the
+ * attention matrix recomputed from q, k and the forward's lse instead of
+ * stored ("FlashAttention算法原理与性能优化实战" §1.2.3, recomputation; the
+ * Triton FA2 walkthrough keeps the logsumexp for the backward pass).  With
+ * P = softmax(scale q k^T + mask):
+ *     dv = P^T dout,  dS = P .* (dout v^T - delta),  delta_i = dout_i . out_i,
+ *     dq = scale dS k,  dk = scale dS^T q,
+ * and for GQA the query heads that share a key/value head add into it.
+ *
+ *   q, out, dout  device, [B, H,    L_q, D], element type `dtype`
+ *   k, v          device, [B, H_kv, L_k, D], element type `dtype`
+ *   lse           device, [B, H, L_q] fp32: the forward's lse (-inf rows
+ *                 see no key and get dq = 0)
+ *   dq            device, [B, H,    L_q, D] written (RNE of fp32)
+ *   dk, dv        device, [B, H_kv, L_k, D] written
+ *   scale, causal, window_left, window_right, dtype: as fa_fwd, and the
+ *                 same values the forward used
+ *   workspace     device, 256-byte aligned, caller-owned, at least
+ *                 fa_bwd_workspace_bytes(B, H, L_q, D) bytes
+ *                 (FA_ERR_WORKSPACE if smaller); contents on entry do not
+ *                 matter.  Calls that share a workspace must not overlap.
+ * L_q == 0 writes dk = dv = 0; L_k == 0 writes dq = 0.  Pointers to tensors
+ * with no elements may be NULL.  q, k, v, out, dout, dq, dk, dv need
+ * 16-byte alignment, lse 4 bytes (FA_ERR_ALIGN).  Errors as fa_fwd.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int H, int H_kv, int L_q,
+           int L_k, int D, float scale, int causal, int window_left, int window_right,
+           int dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * fa_fwd_splitkv_static -- fa_fwd_splitkv with no workspace argument: the
  * partials live in a fixed scratch array inside the library (static device
  * memory, FA_STATIC_SCRATCH_BYTES per device).  The pages have no

@@ -291,6 +291,7 @@ def __getattr__(name):
     # module-level convenience: oracle.attention(...), oracle.decode(...), ...
     if name in {"f16_to_f64", "bf16_to_f64", "f64_to_f16", "f64_to_bf16",
                 "decode", "round_to", "safe_softmax", "online_softmax",
-                "attention_rows", "attention", "attention_rows_online"}:
+                "attention_rows", "attention", "attention_rows_online",
+                "attention_f64", "attention_bwd_f64", "attention_bwd"}:
         return getattr(get(), name)
     raise AttributeError(name)

@@ -164,3 +164,38 @@ def test_static_scratch_size_matches_header():
 ])
 def test_static_entry_refuses_before_the_gpu(lib, kw, code):
     assert _call_static(**kw) == code
+
+
+# ------------------------------------------------------------ backward entry
+BWD_GOOD = dict(q=16, k=16, v=16, out=16, dout=16, lse=16, dq=16, dk=16, dv=16, B=1, H=4,
+                H_kv=2, L_q=8, L_k=8, D=64, scale=0.125, causal=0, wl=-1, wr=-1, dtype=0,
+                ws=256, ws_bytes=1 << 30)
+
+
+def _call_bwd(**kw):
+    a = dict(BWD_GOOD)
+    a.update(kw)
+    return fa.fa_bwd(a["q"], a["k"], a["v"], a["out"], a["dout"], a["lse"], a["dq"], a["dk"],
+                     a["dv"], a["B"], a["H"], a["H_kv"], a["L_q"], a["L_k"], a["D"], a["scale"],
+                     a["causal"], a["wl"], a["wr"], a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+def test_bwd_workspace_bytes(lib):
+    # dQ accumulator (B*H*L_q*D fp32), then lse2 and delta over L_q padded to 128
+    up = lambda x: (x + 255) // 256 * 256
+    B, H, L_q, D = 2, 3, 130, 64
+    want = up(B * H * L_q * D * 4) + 2 * up(B * H * 256 * 4)
+    assert fa.fa_bwd_workspace_bytes(B, H, L_q, D) == want
+    assert fa.fa_bwd_workspace_bytes(B, H, L_q, 48) == 0
+    assert fa.fa_bwd_workspace_bytes(0, H, L_q, 64) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(dout=0), -1), (dict(lse=0), -1), (dict(dk=0), -1), (dict(ws=0), -1),
+    (dict(B=0), -2), (dict(H=4, H_kv=3), -2), (dict(L_k=-1), -2),
+    (dict(D=48), -3), (dict(dtype=2), -4),
+    (dict(dq=8), -5), (dict(lse=2), -5), (dict(ws=128), -5),
+    (dict(scale=float("nan")), -6), (dict(ws_bytes=1000), -9),
+])
+def test_bwd_argument_errors(lib, kw, code):
+    assert _call_bwd(**kw) == code

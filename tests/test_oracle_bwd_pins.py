@@ -187,3 +187,13 @@ def test_error_scales(orc):
                                rtol=1e-14)
     np.testing.assert_allclose(dka[0, 0, 0], 0.7 * (e[0, 0, :, None] * np.abs(q[0, 0])).sum(0),
                                rtol=1e-14)
+
+
+def test_module_level_entries():
+    # the GPU tests call these through the module
+    import oracle
+    c = CASES[0]
+    q, k, v, do = _inputs(c, 12)
+    assert np.array_equal(oracle.attention_bwd_f64(q, k, v, do, 0.7)[0],
+                          oracle.get().attention_bwd_f64(q, k, v, do, 0.7)[0])
+    assert callable(oracle.attention_bwd) and callable(oracle.attention_f64)
