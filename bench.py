@@ -17,6 +17,10 @@ every rank runs the same-sized problem on its own inputs (weak scaling; the
 path has no exchange step), and the value is all ranks' FLOPs over the
 slowest rank's time.
 
+--pass bwd times fa_bwd (the backward, after one untimed forward for O and
+lse): a step is its three launches (delta / lse prep, the gradient kernel,
+the dQ conversion); the metric counts 2.5x the forward's FLOPs.
+
 --splits S (or auto) times fa_fwd_splitkv instead: one split-KV launch plus
 one merge launch per step, for the decoding workloads (a few query rows, a
 long key/value cache), whose roofline is HBM bandwidth rather than the
@@ -49,7 +53,9 @@ if ROOT not in sys.path:
 from exact_attention_113_b200 import inputs as W  # noqa: E402
 
 METRIC = "attention fwd TFLOPS (and % of B200 fp16 tensor peak) vs seq len"
+METRIC_BWD = "attention bwd TFLOPS (five GEMMs: 2.5x the forward's FLOPs)"
 UNIT = "TFLOPS"
+BWD_FLOP_FACTOR = 2.5      # backward: S, dP, dV, dK, dQ = 5 GEMMs vs the forward's 2
 DEFAULT_WORKLOAD = W.ROOFLINE.name
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fa_fwd_roofline_b4h48l8192d128_ncu.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_113_b200", "csrc", f)
@@ -278,17 +284,35 @@ def run_ours(args, w: W.Workload):
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.L_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    n_splits = resolve_splits(args.splits, w)
+    bwd = args.pass_ == "bwd"
+    n_splits = 0 if bwd else resolve_splits(args.splits, w)
     ws = None
     if n_splits:
         ws = torch.empty(fa.fa_splitkv_workspace_bytes(w.B, w.H, w.L_q, w.D, n_splits),
                          dtype=torch.uint8, device=dev)
-    launches_per_step = 2 if n_splits else 1
+    launches_per_step = 3 if bwd else (2 if n_splits else 1)
+    fm = BWD_FLOP_FACTOR if bwd else 1.0
 
-    def step():
-        fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
-                     window_left=w.window_left, window_right=w.window_right,
-                     out=out, lse=lse, stream=stream, n_splits=n_splits, workspace=ws)
+    if bwd:
+        do_cpu = W.make_dout(w_rank)
+        dout = do_cpu.to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.H, w.L_q, w.D), dtype=torch.uint8,
+                          device=dev)
+        with torch.cuda.stream(stream):
+            fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
+                         window_left=w.window_left, window_right=w.window_right,
+                         out=out, lse=lse, stream=stream)
+
+        def step():
+            fa.flash_bwd(q, k, v, out, dout, lse, scale=w.softmax_scale, causal=w.causal,
+                         window_left=w.window_left, window_right=w.window_right, dq=dq, dk=dk,
+                         dv=dv, workspace=bws, stream=stream)
+    else:
+        def step():
+            fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
+                         window_left=w.window_left, window_right=w.window_right,
+                         out=out, lse=lse, stream=stream, n_splits=n_splits, workspace=ws)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -317,15 +341,15 @@ def run_ours(args, w: W.Workload):
     if fa.fa_get_device_status(stream.cuda_stream) != 0:
         raise RuntimeError("device watchdog fired during the timed steps")
     max_total = max_over_ranks(total_s, world, dev)
-    value = whole_job_value(metric_flops(w), world, args.steps, max_total)
+    value = whole_job_value(fm * metric_flops(w), world, args.steps, max_total)
     avg_launch_s = sum(launch_ms) / len(launch_ms) / 1e3
 
     # ---- roofline of the (only) kernel
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    if roofline_bound(w, peak, hbm) == "tensor":
-        achieved = algorithmic_flops(w) / avg_launch_s / 1e12
+    if bwd or roofline_bound(w, peak, hbm) == "tensor":
+        achieved = fm * algorithmic_flops(w) / avg_launch_s / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "traffic": profiled_traffic() if w.name == W.ROOFLINE.name else None,
@@ -335,8 +359,11 @@ def run_ours(args, w: W.Workload):
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
                     "peak_source": f"{peak_kind} HBM copy bandwidth"}
-    roofline.update({"algorithmic_flop_per_launch": algorithmic_flops(w),
+    roofline.update({"algorithmic_flop_per_launch": fm * algorithmic_flops(w),
                      "min_hbm_bytes_per_launch": min_hbm_bytes(w)})
+    if bwd:
+        roofline["traffic"] = None
+        roofline["timed"] = "whole step: prep, gradient kernel and dQ conversion launches"
     if n_splits:
         roofline["timed"] = (f"whole step: split-KV launch ({n_splits} key slices) "
                              "plus merge launch")
@@ -345,16 +372,24 @@ def run_ours(args, w: W.Workload):
     e2e = None
     if not args.skip_e2e:
         hq, hk, hv = (t.pin_memory() for t in (q_cpu, k_cpu, v_cpu))
-        hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        if bwd:
+            # inputs: q, k, v, out, dout, lse; results: dq, dk, dv
+            h_in = [hq, hk, hv, out.cpu().pin_memory(), do_cpu.pin_memory(),
+                    lse.cpu().pin_memory()]
+            d_in = [q, k, v, out, dout, lse]
+            d_out = [dq, dk, dv]
+        else:
+            h_in = [hq, hk, hv]
+            d_in = [q, k, v]
+            d_out = [out, lse]
+        h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in d_out]
 
         def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
+            for d, h in zip(d_in, h_in):
+                d.copy_(h, non_blocking=True)
             step()
-            hout.copy_(out, non_blocking=True)
-            hlse.copy_(lse, non_blocking=True)
+            for h, d in zip(h_out, d_out):
+                h.copy_(d, non_blocking=True)
 
         n_e2e = max(3, min(args.steps, 10))
         with torch.cuda.stream(stream):
@@ -369,20 +404,21 @@ def run_ours(args, w: W.Workload):
             e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-        d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
-        e2e = {"value": round(whole_job_value(metric_flops(w), world, n_e2e, e2e_s), 2),
+        h2d = sum(t.numel() * t.element_size() for t in h_in)
+        d2h = sum(t.numel() * t.element_size() for t in h_out)
+        e2e = {"value": round(whole_job_value(fm * metric_flops(w), world, n_e2e, e2e_s), 2),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e, "ms_per_step": round(e2e_s / n_e2e * 1e3, 3)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline and not bwd:
         tf, cores, desc = cpu_oracle_sample(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
         cpu = {"value": round(tf, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": desc, "host_nproc": os.cpu_count()}
 
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC_BWD if bwd else METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(max_total / args.steps * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -492,6 +528,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.ALL))
+    ap.add_argument("--pass", dest="pass_", choices=("fwd", "bwd"), default="fwd",
+                    help="time the forward (default) or the backward")
     ap.add_argument("--splits", default="0",
                     help="key slices for fa_fwd_splitkv (0: plain fa_fwd; auto)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")

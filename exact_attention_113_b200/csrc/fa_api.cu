@@ -72,6 +72,26 @@ bool encode_map(CUtensorMap *map, const void *base, int dtype, int n_heads, int 
   return r == CUDA_SUCCESS;
 }
 
+// A rank-3 fp32 tensor map over a contiguous [n_heads, L, D] array with a
+// box of [1, 128, box_cols] (box_cols 32: 128-byte swizzle; 16: 64-byte).
+bool encode_map_f32(CUtensorMap *map, const void *base, int n_heads, int L, int D,
+                    int box_cols) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(n_heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4,
+                           static_cast<cuuint64_t>(L) * D * 4};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw =
+      box_cols * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 __global__ void fill_kernel(float *p, size_t n, float value) {
@@ -477,7 +497,8 @@ extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *o
   if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
-      !encode_map(&prm.tm_do, dout, dtype, B * H, L_q, D, box_cols))
+      !encode_map(&prm.tm_do, dout, dtype, B * H, L_q, D, box_cols) ||
+      !encode_map_f32(&prm.tm_dq, prm.dq_acc, B * H, L_q, D, D >= 32 ? 32 : 16))
     return FA_ERR_CUDA;
   switch (D * 2 + dtype) {
     case 32: return launch_bwd<16, 0>(prm, out, dout, lse, dq, B, H, stream);

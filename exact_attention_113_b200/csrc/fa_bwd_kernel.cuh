@@ -20,7 +20,9 @@
 //     dK  += dS^T Q     (TS: dS^T from TMEM)
 //     dQ   = dS K       (SS: dS staged in shared memory MN-major, K MN-major)
 // dQ of the step is added into an fp32 accumulator in global memory by a
-// warpgroup of its own (vector atomic adds); the other key blocks add theirs.
+// warpgroup of its own: TMEM -> swizzled fp32 staging in shared memory ->
+// TMA bulk reduce-add (the addition happens in L2, a tile at a time); the
+// other key blocks add theirs.
 //
 // Roles (512 threads): warpgroups 0 and 1 compute P and dS for query
 // columns [0, 64) and [64, 128) of every key row (thread = TMEM lane = key);
@@ -45,6 +47,7 @@ struct BwdParams {
   CUtensorMap tm_k;    // [B*H_kv, L_k, D]
   CUtensorMap tm_v;    // [B*H_kv, L_k, D]
   CUtensorMap tm_do;   // [B*H,    L_q, D]
+  CUtensorMap tm_dq;   // dq_acc as [B*H, L_q, D] fp32, box [128 rows, min(32, D) cols]
   const float *lse2;   // [B*H][L_q_pad]: lse * log2(e); +inf where no key is visible / past L_q
   const float *delta;  // [B*H][L_q_pad]: dO_i . O_i; 0 past L_q
   float *dq_acc;       // [B*H][L_q][D] fp32, zero before the launch
@@ -73,12 +76,22 @@ struct BwdGeo {
   static constexpr int kTileBytes = G::kTileBytes;        // 128 rows x D, TMA-swizzled
   static constexpr int kDsBoxBytes = 128 * 128;           // [128 keys][64 queries] 16-bit, SW128
   static constexpr int kDsBytes = 2 * kDsBoxBytes;
+  // dO is single-buffered at D = 128 (its last reader, dV of the step, runs
+  // early) to make room for the dQ staging buffer
+  static constexpr int kDoStages = D == 128 ? 1 : 2;
+  // dQ staging: two fp32 boxes of [128 rows][kDqBoxCols], 64 columns a round
+  static constexpr int kDqBoxCols = D >= 32 ? 32 : D;
+  static constexpr int kDqBoxBytes = 128 * kDqBoxCols * 4;
+  static constexpr int kDqBoxes = D >= 64 ? 2 : 1;        // boxes per round
+  static constexpr int kDqRounds = D / (kDqBoxCols * kDqBoxes);
+  static constexpr int kDqSwBytes = kDqBoxCols * 4;       // 128 (SW128) or 64 (SW64)
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;            // two stages
-  static constexpr int kOffDo = 4 * kTileBytes;           // two stages
-  static constexpr int kOffDs = 6 * kTileBytes;
-  static constexpr int kOffVec = kOffDs + kDsBytes;       // lse2[128], delta[128]
+  static constexpr int kOffDo = 4 * kTileBytes;           // kDoStages stages
+  static constexpr int kOffDs = kOffDo + kDoStages * kTileBytes;
+  static constexpr int kOffDq = kOffDs + kDsBytes;
+  static constexpr int kOffVec = kOffDq + kDqBoxes * kDqBoxBytes;   // lse2[128], delta[128]
   static constexpr int kOffBar = kOffVec + 256 * 4;
   static constexpr int kBarBytes = 256;
   static constexpr int kUsed = kOffBar + kBarBytes;
@@ -90,8 +103,10 @@ struct BwdGeo {
 
 struct BwdBars {
   uint64_t kv_full;
-  uint64_t q_full[2];
+  uint64_t q_full[2];     // Q (and, with two dO stages, dO) of a stage
   uint64_t q_empty[2];
+  uint64_t do_full;       // single dO stage: dO of the step
+  uint64_t do_empty;      // single dO stage: dV (its last reader) done
   uint64_t s_full;
   uint64_t dp_full;
   uint64_t p_full;
@@ -153,6 +168,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       mbar_init(smem_u32(&bars->q_full[s]), 1);
       mbar_init(smem_u32(&bars->q_empty[s]), 1);
     }
+    mbar_init(smem_u32(&bars->do_full), 1);
+    mbar_init(smem_u32(&bars->do_empty), 1);
     mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
     mbar_init(smem_u32(&bars->p_full), 256);
@@ -172,6 +189,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
     prefetch_tensormap(&p.tm_do);
+    prefetch_tensormap(&p.tm_dq);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -189,7 +207,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   if (warp == 9) {
     // =================================================== TMA producer
     const uint64_t pol_keep = policy_evict_last();
-    int issued = 0;
+    int issued = 0;       // steps whose Q copy was issued
+    int do_issued = 0;    // single dO stage: steps whose dO copy was issued
     bool ok = true;
     if (n_steps > 0) {
       const uint32_t bar = smem_u32(&bars->kv_full);
@@ -211,16 +230,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         const uint32_t qb = smem_u32(&bars->q_full[st]);
         const int q0 = q0_of(n), bh = bh_of(n);
         if (elect_one()) {
-          mbar_arrive_expect_tx(qb, 2 * G::kTileBytes);
+          mbar_arrive_expect_tx(qb, (BG::kDoStages == 2 ? 2 : 1) * G::kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < G::kNumBox; ++bx) {
             tma_load_3d(sQ + st * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, qb,
                         bx * G::kBoxCols, q0, bh, pol_keep);
-            tma_load_3d(sDo + st * G::kTileBytes + bx * G::kBoxBytes, &p.tm_do, qb,
-                        bx * G::kBoxCols, q0, bh, pol_keep);
+            if constexpr (BG::kDoStages == 2)
+              tma_load_3d(sDo + st * G::kTileBytes + bx * G::kBoxBytes, &p.tm_do, qb,
+                          bx * G::kBoxCols, q0, bh, pol_keep);
           }
         }
         __syncwarp();
+        if constexpr (BG::kDoStages == 1) {
+          if (n >= 1) {
+            ok = mbar_wait_warp(smem_u32(&bars->do_empty), (n - 1) & 1, abort_flag);
+            if (!ok) {
+              issued = n + 1;   // Q of step n is in flight, its dO is not
+              break;
+            }
+          }
+          const uint32_t db = smem_u32(&bars->do_full);
+          if (elect_one()) {
+            mbar_arrive_expect_tx(db, G::kTileBytes);
+#pragma unroll
+            for (int bx = 0; bx < G::kNumBox; ++bx)
+              tma_load_3d(sDo + bx * G::kBoxBytes, &p.tm_do, db, bx * G::kBoxCols, q0, bh,
+                          pol_keep);
+          }
+          __syncwarp();
+          do_issued = n + 1;
+        }
         issued = n + 1;
       }
       if (!ok) {
@@ -228,6 +267,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         mbar_wait_slow(smem_u32(&bars->kv_full), 0, abort_flag, false);
         for (int n = max(0, issued - 2); n < issued; ++n)
           mbar_wait_slow(smem_u32(&bars->q_full[n & 1]), (n >> 1) & 1, abort_flag, false);
+        if constexpr (BG::kDoStages == 1) {
+          if (do_issued > 0)   // the latest dO copy (phases complete in order)
+            mbar_wait_slow(smem_u32(&bars->do_full), (do_issued - 1) & 1, abort_flag, false);
+        }
       }
     }
   } else if (warp == 8) {
@@ -273,18 +316,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         if (elect_one()) tc_commit(bar);
         __syncwarp();
       };
+      // dO of step n: its own stage, or the single stage after do_full(n)
+      auto do_tile = [&](int n) -> uint32_t {
+        return BG::kDoStages == 2 ? sDo + (n & 1) * G::kTileBytes : sDo;
+      };
+      auto wait_do = [&](int n) -> bool {
+        return BG::kDoStages == 2 || mbar_wait_warp(smem_u32(&bars->do_full), n & 1, abort_flag);
+      };
       if (ok) ok = mbar_wait_warp(smem_u32(&bars->q_full[0]), 0, abort_flag);
       if (ok) {
         tc_fence_after_sync();
         issue_kmajor(tS, sK, sQ, smem_u32(&bars->s_full));
-        issue_kmajor(tDP, sV, sDo, smem_u32(&bars->dp_full));
+        ok = wait_do(0);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_kmajor(tDP, sV, do_tile(0), smem_u32(&bars->dp_full));
+        }
       }
       for (int n = 0; n < n_steps && ok; ++n) {
         const int st = n & 1;
         ok = mbar_wait_warp(smem_u32(&bars->p_full), n & 1, abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
-        issue_ts(tDV, tS, sDo + st * G::kTileBytes, n == 0);
+        issue_ts(tDV, tS, do_tile(n), n == 0);
+        if constexpr (BG::kDoStages == 1) commit(smem_u32(&bars->do_empty));
         if (n + 1 < n_steps) {
           const int st1 = (n + 1) & 1;
           ok = mbar_wait_warp(smem_u32(&bars->q_full[st1]), ((n + 1) >> 1) & 1, abort_flag);
@@ -313,10 +368,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         commit(smem_u32(&bars->dq_full));
         commit(smem_u32(&bars->q_empty[st]));
         if (n + 1 < n_steps) {
-          ok = mbar_wait_warp(smem_u32(&bars->dq_free), n & 1, abort_flag);
+          ok = mbar_wait_warp(smem_u32(&bars->dq_free), n & 1, abort_flag) && wait_do(n + 1);
           if (!ok) break;
           tc_fence_after_sync();
-          issue_kmajor(tDP, sV, sDo + ((n + 1) & 1) * G::kTileBytes, smem_u32(&bars->dp_full));
+          issue_kmajor(tDP, sV, do_tile(n + 1), smem_u32(&bars->dp_full));
         }
       }
     }
@@ -465,28 +520,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     const int r = tid & 127;                       // query row within the block = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tDQ = tmem + lane_base + 128u;
+    uint8_t *stage = smem + BG::kOffDq;
+    const bool leader = tid == 384;                // issues the bulk reductions
+    constexpr int kUnits = BG::kDqSwBytes / 16;    // 16-byte units per staged row
+    const int sw = ((r * BG::kDqSwBytes) >> 7) & (kUnits - 1);
+    bool ok = true;
+    // Every drain warp passes the same named barriers, also after a timeout.
     for (int n = 0; n < n_steps; ++n) {
-      if (!mbar_wait_warp(smem_u32(&bars->dq_full), n & 1, abort_flag)) break;
-      tc_fence_after_sync();
-      const int i = q0_of(n) + r;
-      float *dst = p.dq_acc + (static_cast<size_t>(bh_of(n)) * p.L_q + i) * D;
-      constexpr int kChunk = D >= 32 ? 32 : D;
-      uint32_t acc[D];
+      if (ok) ok = mbar_wait_warp(smem_u32(&bars->dq_full), n & 1, abort_flag);
+      if (ok) tc_fence_after_sync();
+      const int q0 = q0_of(n), bh = bh_of(n);
 #pragma unroll
-      for (int c = 0; c < D; c += kChunk)
-        tmem_ld_cols<kChunk>(tDQ + c, *reinterpret_cast<uint32_t(*)[kChunk]>(acc + c));
-      tmem_wait_ld();
-      reg_dep(acc);
-      tc_fence_before_sync();
-      mbar_arrive(smem_u32(&bars->dq_free));       // TMEM columns free for dP^T of the next step
-      if (i < p.L_q) {
+      for (int rd = 0; rd < BG::kDqRounds; ++rd) {
+        uint32_t v[BG::kDqBoxes][BG::kDqBoxCols];
+        if (ok) {
 #pragma unroll
-        for (int u = 0; u < D / 4; ++u)
-          atomicAdd(reinterpret_cast<float4 *>(dst) + u,
-                    make_float4(__uint_as_float(acc[4 * u]), __uint_as_float(acc[4 * u + 1]),
-                                __uint_as_float(acc[4 * u + 2]), __uint_as_float(acc[4 * u + 3])));
+          for (int bx = 0; bx < BG::kDqBoxes; ++bx)
+            tmem_ld_cols<BG::kDqBoxCols>(
+                tDQ + (rd * BG::kDqBoxes + bx) * BG::kDqBoxCols, v[bx]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int bx = 0; bx < BG::kDqBoxes; ++bx) reg_dep(v[bx]);
+          if (rd == BG::kDqRounds - 1) {
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&bars->dq_free));   // TMEM columns free for dP^T
+          }
+        }
+        if (leader) bulk_wait_group_read_all();    // the staging buffer has been read
+        named_barrier_sync(2, 128);
+        if (ok) {
+#pragma unroll
+          for (int bx = 0; bx < BG::kDqBoxes; ++bx)
+#pragma unroll
+            for (int u = 0; u < kUnits; ++u)
+              *reinterpret_cast<uint4 *>(stage + bx * BG::kDqBoxBytes + r * BG::kDqSwBytes +
+                                         ((u ^ sw) << 4)) =
+                  make_uint4(v[bx][4 * u], v[bx][4 * u + 1], v[bx][4 * u + 2], v[bx][4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        named_barrier_sync(2, 128);
+        if (leader && ok) {
+#pragma unroll
+          for (int bx = 0; bx < BG::kDqBoxes; ++bx)
+            tma_reduce_add_3d(&p.tm_dq, smem_u32(stage + bx * BG::kDqBoxBytes),
+                              (rd * BG::kDqBoxes + bx) * BG::kDqBoxCols, q0, bh);
+          bulk_commit_group();
+        }
       }
     }
+    if (leader) bulk_wait_group_all();             // the reductions have landed
   }
 
   // ---- teardown
