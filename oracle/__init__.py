@@ -15,7 +15,8 @@ Functions whose parity is pinned (see tests/test_oracle_pins.py and
 tests/test_oracle_bwd_pins.py):
   attention, attention_rows, attention_rows_online, safe_softmax,
   online_softmax, f16/bf16 decode and round-to-nearest-even,
-  attention_f64, attention_bwd_f64 / attention_bwd (gradients).
+  attention_f64, attention_bwd_f64 / attention_bwd (gradients),
+  attention_rows_ex (mask, softmax max / sum; tests/test_oracle_mask_pins.py).
 """
 from __future__ import annotations
 
@@ -104,6 +105,11 @@ class Oracle:
             u16p, u16p, u16p, ctypes.c_int, i64, i64, i64, i64, i64, i64,
             ctypes.c_double, ctypes.c_int, i64, i64, i64p, i64, i64, dp, dp]
         lib.oracle_attention_rows_online.restype = ctypes.c_int
+        lib.oracle_attention_rows_ex.argtypes = [
+            u16p, u16p, u16p, ctypes.c_int, i64, i64, i64, i64, i64, i64,
+            ctypes.c_double, ctypes.c_int, i64, i64, ctypes.c_void_p, ctypes.c_int, i64, i64,
+            i64, i64p, i64, dp, dp, dp, dp, ctypes.c_int]
+        lib.oracle_attention_rows_ex.restype = ctypes.c_int
         lib.oracle_attention_f64.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, i64,
                                              ctypes.c_double, ctypes.c_int, i64, i64, dp, dp]
         lib.oracle_attention_f64.restype = ctypes.c_int
@@ -222,6 +228,56 @@ class Oracle:
         return out, lse
 
 
+    # ------------------------------------------------------------- mask, statistics
+    @staticmethod
+    def mask_args(mask, B, H, L_q, L_k):
+        """(pointer-owner array, type, stride_b, stride_h, stride_q) for a
+        mask array of shape (B|1, H|1, L_q|1, L_k), dtype bool / float16 /
+        float32, contiguous along the last axis; a size-1 axis broadcasts."""
+        if mask is None:
+            return None, 0, 0, 0, 0
+        m = np.asarray(mask)
+        types = {np.dtype(np.bool_): 1, np.dtype(np.uint8): 1, np.dtype(np.float16): 2,
+                 np.dtype(np.float32): 3}
+        if m.ndim != 4 or m.dtype not in types:
+            raise ValueError("mask must be 4-D bool / float16 / float32")
+        if m.shape[3] != L_k or m.strides[3] != m.itemsize:
+            raise ValueError("mask must be contiguous along keys")
+        want = (B, H, L_q)
+        st = []
+        for d in range(3):
+            if m.shape[d] == 1:
+                st.append(0)
+            elif m.shape[d] == want[d]:
+                st.append(m.strides[d] // m.itemsize)
+            else:
+                raise ValueError("mask shape does not broadcast")
+        return m, types[m.dtype], st[0], st[1], st[2]
+
+    def attention_rows_ex(self, q, k, v, dtype, scale, causal=False, window_left=-1,
+                          window_right=-1, mask=None, rows=None, n_threads=0):
+        """Exact attention with an optional mask (see attention_ref.c for
+        its reading); returns (out [n, D], lse, softmax_max, softmax_sum)."""
+        q, k, v, B, H, H_kv, L_q, L_k, D = _shape_args(q, k, v)
+        m, mtype, sb, sh, sq = self.mask_args(mask, B, H, L_q, L_k)
+        if rows is None:
+            n, rows_p = B * H * L_q, None
+        else:
+            rows = np.ascontiguousarray(rows, dtype=np.int64)
+            n, rows_p = rows.size, _ptr(rows, ctypes.c_int64)
+        out = np.zeros((n, D), dtype=np.float64)
+        lse, smax, ssum = (np.zeros((n,), dtype=np.float64) for _ in range(3))
+        rc = self.lib.oracle_attention_rows_ex(
+            _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+            int(dtype), B, H, H_kv, L_q, L_k, D, float(scale), int(bool(causal)),
+            int(window_left), int(window_right),
+            m.ctypes.data_as(ctypes.c_void_p) if m is not None else None, mtype, sb, sh, sq,
+            rows_p, n, _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
+            _ptr(smax, ctypes.c_double), _ptr(ssum, ctypes.c_double), int(n_threads))
+        if rc < 0:
+            raise ValueError("oracle rejected the arguments")
+        return out, lse, smax, ssum
+
     # ------------------------------------------------------------- fp64 inputs
     @staticmethod
     def _f64(x):
@@ -292,6 +348,7 @@ def __getattr__(name):
     if name in {"f16_to_f64", "bf16_to_f64", "f64_to_f16", "f64_to_bf16",
                 "decode", "round_to", "safe_softmax", "online_softmax",
                 "attention_rows", "attention", "attention_rows_online",
-                "attention_f64", "attention_bwd_f64", "attention_bwd"}:
+                "attention_f64", "attention_bwd_f64", "attention_bwd",
+                "attention_rows_ex", "mask_args"}:
         return getattr(get(), name)
     raise AttributeError(name)

@@ -178,6 +178,42 @@ static void build_decode_table(int dtype, double *tab)
                             : oracle_bf16_to_f64((uint16_t)b);
 }
 
+/* ---------------------------------------------------------------------
+ * Forward with an optional attention mask and the two softmax statistics.
+ *
+ * The operator statement of "FlashAttention算法原理与性能优化实战" section 2.2
+ * takes an optional attn_mask (fp16, fp32 or bool) and returns, beside the
+ * output, softmax_max and softmax_sum of shape [B, H, S] for the backward.
+ * The Triton FA2 walkthrough notes that mask (and dropout) act on S before
+ * the softmax, as step MASK of FlashAttention's Algorithm 2.  The pages do
+ * not spell out the mask's meaning; the reading taken here:
+ *   - a float mask (fp16 / fp32) is added to the scaled scores:
+ *       s_ij = scale * q_i . k_j + mask_ij   (-inf hides the key);
+ *   - a bool mask hides the keys where it is true (nonzero byte), like the
+ *     MASK step that sets those scores to -inf;
+ *   - the causal / window visibility still applies on top;
+ *   - element (b, h, i, j) of the mask is element
+ *       b*stride_b + h*stride_h + i*stride_q + j  of the array,
+ *     a stride of 0 broadcasts over that index;
+ *   - softmax_max_i = max_j s_ij over the visible keys and
+ *     softmax_sum_i = sum_j e^{s_ij - softmax_max_i}, so that
+ *     lse_i = softmax_max_i + ln(softmax_sum_i); a row with no visible key
+ *     has softmax_max = -inf and softmax_sum = 0.
+ * mask_type: 0 none, 1 bool (uint8), 2 fp16, 3 fp32.
+ * ------------------------------------------------------------------- */
+static double mask_value(const void *mask, int mask_type, int64_t idx, int *hidden)
+{
+    *hidden = 0;
+    if (mask_type == 1) {
+        *hidden = ((const uint8_t *)mask)[idx] != 0;
+        return 0.0;
+    }
+    if (mask_type == 2) return oracle_f16_to_f64(((const uint16_t *)mask)[idx]);
+    if (mask_type == 3) return (double)((const float *)mask)[idx];
+    return 0.0;
+}
+
+
 /*
  * Exact attention for a list of query rows.
  *   q    : [B, H,    L_q, D] bit patterns (dtype 0 = fp16, 1 = bf16)
@@ -189,19 +225,27 @@ static void build_decode_table(int dtype, double *tab)
  *          it is the scale of the error that rounding the weights p_j to a
  *          t-bit format causes in O (at most 2^-t * wabs per element, first
  *          order), which the parity tests use in their tolerance.
+ *   mask, mask_type, stride_b/h/q : the optional mask (type 0 = none),
+ *          read as stated above mask_value();
+ *   smax, ssum : [n_rows] fp64 (may be NULL): softmax_max, softmax_sum.
+ * Shared by oracle_attention_rows (no mask, no statistics) and
+ * oracle_attention_rows_ex.
  * Returns the number of threads used, or a negative value on bad input.
  */
-int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
-                          const uint16_t *v, int dtype, int64_t B, int64_t H,
-                          int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
-                          double scale, int causal, int64_t window_left,
-                          int64_t window_right, const int64_t *rows,
-                          int64_t n_rows, double *out, double *lse,
-                          double *wabs, int n_threads)
+static int rows_core(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     int dtype, int64_t B, int64_t H, int64_t H_kv, int64_t L_q,
+                     int64_t L_k, int64_t D, double scale, int causal,
+                     int64_t window_left, int64_t window_right,
+                     const void *mask, int mask_type, int64_t stride_b,
+                     int64_t stride_h, int64_t stride_q, const int64_t *rows,
+                     int64_t n_rows, double *out, double *lse, double *wabs,
+                     double *smax, double *ssum, int n_threads)
 {
     if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1)
         return -1;
     if (H % H_kv != 0 || (dtype != 0 && dtype != 1))
+        return -1;
+    if (mask_type < 0 || mask_type > 3 || (mask_type != 0 && mask == NULL))
         return -1;
     if (rows == NULL)
         n_rows = B * H * L_q;
@@ -236,7 +280,12 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
                 qrow[d] = tab[qp[d]];
             /* the full row of S, with masked entries at -inf */
             for (int64_t j = 0; j < L_k; j++) {
-                if (!visible(i, j, L_k, causal, window_left, window_right)) {
+                int hidden = 0;
+                double bias = 0.0;
+                if (mask_type != 0)
+                    bias = mask_value(mask, mask_type,
+                                      b * stride_b + h * stride_h + i * stride_q + j, &hidden);
+                if (hidden || !visible(i, j, L_k, causal, window_left, window_right)) {
                     s[j] = -INFINITY;
                     continue;
                 }
@@ -244,6 +293,7 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
                 for (int64_t d = 0; d < D; d++)
                     acc += qrow[d] * tab[kp[j * D + d]];
                 s[j] = scale * acc;
+                s[j] += bias;
             }
             double m, den;
             oracle_safe_softmax(s, L_k, p, &den, &m);
@@ -257,6 +307,8 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
             }
             if (lse)
                 lse[t] = (m == -INFINITY) ? -INFINITY : m + log(den);
+            if (smax) smax[t] = m;
+            if (ssum) ssum[t] = (m == -INFINITY) ? 0.0 : den;
             if (wabs) {
                 double *w = wabs + t * D;
                 for (int64_t d = 0; d < D; d++)
@@ -274,6 +326,37 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
     }
     free(tab);
     return used;
+}
+
+int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
+                          const uint16_t *v, int dtype, int64_t B, int64_t H,
+                          int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
+                          double scale, int causal, int64_t window_left,
+                          int64_t window_right, const int64_t *rows,
+                          int64_t n_rows, double *out, double *lse,
+                          double *wabs, int n_threads)
+{
+    return rows_core(q, k, v, dtype, B, H, H_kv, L_q, L_k, D, scale, causal,
+                     window_left, window_right, NULL, 0, 0, 0, 0, rows, n_rows,
+                     out, lse, wabs, NULL, NULL, n_threads);
+}
+
+/* The same with a mask and the two softmax statistics (smax, ssum
+ * nullable), as stated above the mask helpers. */
+int oracle_attention_rows_ex(const uint16_t *q, const uint16_t *k,
+                             const uint16_t *v, int dtype, int64_t B, int64_t H,
+                             int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
+                             double scale, int causal, int64_t window_left,
+                             int64_t window_right, const void *mask,
+                             int mask_type, int64_t stride_b, int64_t stride_h,
+                             int64_t stride_q, const int64_t *rows,
+                             int64_t n_rows, double *out, double *lse,
+                             double *smax, double *ssum, int n_threads)
+{
+    return rows_core(q, k, v, dtype, B, H, H_kv, L_q, L_k, D, scale, causal,
+                     window_left, window_right, mask, mask_type, stride_b,
+                     stride_h, stride_q, rows, n_rows, out, lse, NULL, smax,
+                     ssum, n_threads);
 }
 
 /*
@@ -531,3 +614,4 @@ int oracle_attention_bwd_f64(const double *q, const double *k, const double *v,
     }
     return used;
 }
+

@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import tests.test_oracle_bwd_pins as bwd_pins
+import tests.test_oracle_mask_pins as mask_pins
 import tests.test_oracle_pins as pins
 from exact_attention_113_b200.inputs import F16, BF16
 
@@ -56,6 +57,14 @@ MUTATIONS = {
                        "if (dva) dva[j * D + d] += p[j] * doi[d];"),
     "bwd_abs_delta_term_dropped": ("const double wabs_j = fabs(ds[j]) + p[j] * e;",
                                    "const double wabs_j = fabs(ds[j]);"),
+    # mask and statistics
+    "mask_bool_inverted": ("*hidden = ((const uint8_t *)mask)[idx] != 0;",
+                           "*hidden = ((const uint8_t *)mask)[idx] == 0;"),
+    "mask_bias_dropped": ("s[j] += bias;", "s[j] += 0.0;"),
+    "mask_row_stride_ignored": ("b * stride_b + h * stride_h + i * stride_q + j",
+                                "b * stride_b + h * stride_h + j"),
+    "ssum_not_relative_to_max": ("if (ssum) ssum[t] = (m == -INFINITY) ? 0.0 : den;",
+                                 "if (ssum) ssum[t] = (m == -INFINITY) ? 0.0 : den * exp(m);"),
     "f64_forward_wrong_head": ("const double *kp = k + (b * H_kv + h / group) * L_k * D;\n            const double *vp",
                                "const double *kp = k + (b * H_kv + h % H_kv) * L_k * D;\n            const double *vp"),
 }
@@ -90,6 +99,14 @@ def _battery(orc):
     for dt in (F16, BF16):
         yield lambda dt=dt: bwd_pins.test_bit_pattern_entry_decodes_exactly(orc, dt)
     yield lambda: bwd_pins.test_error_scales(orc)
+    yield lambda: mask_pins.test_empty_masks_change_nothing(orc)
+    yield lambda: mask_pins.test_causal_pattern_masks(orc)
+    yield lambda: mask_pins.test_row_constant_shift(orc)
+    yield lambda: mask_pins.test_log_weight_mask_reweights_keys(orc)
+    for c in (False, True):
+        yield lambda c=c: mask_pins.test_statistics(orc, c)
+    yield lambda: mask_pins.test_fully_hidden_rows(orc)
+    yield lambda: mask_pins.test_broadcast_strides_equal_materialised(orc)
 
 
 def _first_failure(orc):
