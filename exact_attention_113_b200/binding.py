@@ -23,7 +23,8 @@ STATUS = {
     -4: "FA_ERR_DTYPE", -5: "FA_ERR_ALIGN", -6: "FA_ERR_ARG", -7: "FA_ERR_CUDA",
     -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE", -10: "FA_ERR_SCRATCH",
 }
-EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_splitkv",
+FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
+EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_splitkv_workspace_bytes",
            "fa_status_string", "fa_version")
 # size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
@@ -57,6 +58,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
                                i, i, i, i, vp]
         lib.fa_fwd.restype = i
+        ll = ctypes.c_longlong
+        lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, ll, ll, ll, i, i, i, i, i,
+                                  i, ctypes.c_float, i, i, i, i, vp]
+        lib.fa_fwd_ex.restype = i
         lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
                                        i, i, i, i, i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_splitkv.restype = i
@@ -87,6 +92,38 @@ def fa_fwd(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
     return load().fa_fwd(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D,
                          float(scale), int(causal), int(window_left),
                          int(window_right), int(dtype), stream)
+
+
+def fa_fwd_ex(q, k, v, out, lse, softmax_max, softmax_sum, mask, mask_type, mask_stride_b,
+              mask_stride_h, mask_stride_q, B, H, H_kv, L_q, L_k, D, scale, causal,
+              window_left, window_right, dtype, stream) -> int:
+    """The masked / statistics C entry point, unchanged."""
+    return load().fa_fwd_ex(q, k, v, out, lse, softmax_max, softmax_sum, mask, int(mask_type),
+                            int(mask_stride_b), int(mask_stride_h), int(mask_stride_q), B, H,
+                            H_kv, L_q, L_k, D, float(scale), int(causal), int(window_left),
+                            int(window_right), int(dtype), stream)
+
+
+def mask_layout(mask, B, H, L_q, L_k):
+    """(type, stride_b, stride_h, stride_q) of a torch mask of shape
+    (B|1, H|1, L_q|1, L_k), dtype bool / float16 / float32, contiguous along
+    the keys; a size-1 axis broadcasts (stride 0)."""
+    import torch
+    types = {torch.bool: FA_MASK_BOOL, torch.uint8: FA_MASK_BOOL, torch.float16: FA_MASK_F16,
+             torch.float32: FA_MASK_F32}
+    if mask.dim() != 4 or mask.dtype not in types:
+        raise ValueError("mask must be 4-D bool / uint8 / float16 / float32")
+    if mask.shape[3] != L_k or (L_k > 1 and mask.stride(3) != 1):
+        raise ValueError("mask must be [.., .., .., L_k], contiguous along the keys")
+    st = []
+    for d, want in enumerate((B, H, L_q)):
+        if mask.shape[d] == 1:
+            st.append(0)
+        elif mask.shape[d] == want:
+            st.append(mask.stride(d))
+        else:
+            raise ValueError("mask shape does not broadcast to [B, H, L_q, L_k]")
+    return types[mask.dtype], st[0], st[1], st[2]
 
 
 def fa_fwd_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal,
@@ -167,7 +204,7 @@ def fa_version() -> int:
 # ------------------------------------------------------------ torch call
 def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
               return_lse=True, out=None, lse=None, stream=None, n_splits=0,
-              workspace=None):
+              workspace=None, mask=None, return_softmax_stats=False):
     """Exact attention forward on CUDA tensors.
 
     q: [B, H, L_q, D]; k, v: [B, H_kv, L_k, D]; fp16 or bf16, contiguous, on
@@ -181,6 +218,12 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
     CUDA tensor, 256-byte aligned) is given.  ``workspace="static"`` calls
     fa_fwd_splitkv_static instead, which uses the library's fixed scratch
     and allocates nothing (calls must not overlap on the GPU).
+
+    ``mask`` (bool: True hides the key; float16 / float32: added to the
+    scaled scores), shape (B|1, H|1, L_q|1, L_k), and
+    ``return_softmax_stats`` (the row max and sum_j exp(s_j - max)) go
+    through fa_fwd_ex; the result is then (out, lse, softmax_max,
+    softmax_sum).
     """
     import torch
 
@@ -208,6 +251,28 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
         lse = None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    if mask is not None or return_softmax_stats:
+        if n_splits:
+            raise ValueError("mask / softmax statistics are not available with n_splits")
+        mtype, sb, sh, sq = (FA_MASK_NONE, 0, 0, 0) if mask is None else \
+            mask_layout(mask, B, H, L_q, L_k)
+        if mask is not None and (not mask.is_cuda or mask.device != q.device):
+            raise ValueError("mask must be on q's device")
+        smax = ssum = None
+        if return_softmax_stats:
+            smax = torch.empty((B, H, L_q), dtype=torch.float32, device=q.device)
+            ssum = torch.empty_like(smax)
+        with torch.cuda.device(q.device):
+            st = fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           lse.data_ptr() if lse is not None else None,
+                           smax.data_ptr() if smax is not None else None,
+                           ssum.data_ptr() if ssum is not None else None,
+                           mask.data_ptr() if mask is not None else None, mtype, sb, sh, sq,
+                           B, H, H_kv, L_q, L_k, D, scale, causal, window_left, window_right,
+                           dtype, stream.cuda_stream)
+        if st != FA_OK:
+            raise FaError(st, "fa_fwd_ex")
+        return out, lse, smax, ssum
     if n_splits == "auto":
         n_splits = choose_splits(B, H, L_q, L_k,
                                  torch.cuda.get_device_properties(q.device).multi_processor_count,

@@ -100,10 +100,10 @@ __global__ void fill_kernel(float *p, size_t n, float value) {
   for (; i < n; i += stride) p[i] = value;
 }
 
-template <int D, int DT>
+template <int D, int DT, bool kMask>
 int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
   using G = Geo<D>;
-  auto kern = fa_fwd_kernel<D, DT>;
+  auto kern = fa_fwd_kernel<D, DT, kMask>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   static bool configured[64] = {};
@@ -193,11 +193,20 @@ int launch_combine(const float *ws_o, const float2 *ws_ml, void *out, float *lse
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// Shared body of fa_fwd and fa_fwd_splitkv (n_splits == 0: plain forward).
+// Optional mask and softmax statistics of fa_fwd_ex.
+struct MaskArgs {
+  const void *mask;
+  int type;                        // FA_MASK_*
+  long long sb, sh, sq;            // element strides
+  float *smax, *ssum;
+};
+
+// Shared body of fa_fwd, fa_fwd_ex and fa_fwd_splitkv (n_splits == 0: plain
+// forward; mx == nullptr: no mask, no statistics).
 int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
              int H_kv, int L_q, int L_k, int D, float scale, int causal, int window_left,
              int window_right, int dtype, int n_splits, void *workspace,
-             size_t workspace_bytes, cudaStream_t stream);
+             size_t workspace_bytes, const MaskArgs *mx, cudaStream_t stream);
 
 }  // namespace
 }  // namespace fa
@@ -209,7 +218,7 @@ namespace {
 int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
              int H_kv, int L_q, int L_k, int D, float scale, int causal, int window_left,
              int window_right, int dtype, int n_splits, void *workspace,
-             size_t workspace_bytes, cudaStream_t stream) {
+             size_t workspace_bytes, const MaskArgs *mx, cudaStream_t stream) {
   // ---------------------------------------------------------------- checks
   if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
   // a pointer may be NULL only when its tensor has no elements
@@ -225,6 +234,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     return FA_ERR_ALIGN;
   if (lse && !aligned(lse, 4)) return FA_ERR_ALIGN;
   if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+  const bool masked = mx != nullptr && mx->type != FA_MASK_NONE;
+  if (mx != nullptr) {
+    if (mx->type < FA_MASK_NONE || mx->type > FA_MASK_F32) return FA_ERR_ARG;
+    if (mx->sb < 0 || mx->sh < 0 || mx->sq < 0) return FA_ERR_ARG;
+    if (masked && L_q > 0 && L_k > 0 && !mx->mask) return FA_ERR_NULL;
+    if ((mx->smax == nullptr) != (mx->ssum == nullptr)) return FA_ERR_NULL;
+    if (L_q > 0 && (!aligned(mx->smax, 4) || !aligned(mx->ssum, 4))) return FA_ERR_ALIGN;
+  }
   const int64_t rows_total = static_cast<int64_t>(B) * H * L_q;
   if (n_splits != 0) {
     if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
@@ -241,9 +258,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     // no key is visible: O = 0, lse = -inf
     const size_t n_out = static_cast<size_t>(B) * H * L_q * D * 2;
     if (cudaMemsetAsync(out, 0, n_out, stream) != cudaSuccess) return FA_ERR_CUDA;
+    const size_t n = static_cast<size_t>(B) * H * L_q;
     if (lse) {
-      const size_t n = static_cast<size_t>(B) * H * L_q;
       fill_kernel<<<148, 256, 0, stream>>>(lse, n, -INFINITY);
+      if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    if (mx != nullptr && mx->smax != nullptr) {
+      fill_kernel<<<148, 256, 0, stream>>>(mx->smax, n, -INFINITY);
+      fill_kernel<<<148, 256, 0, stream>>>(mx->ssum, n, 0.0f);
       if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     return FA_OK;
@@ -296,6 +318,20 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     float sl2 = scale * 1.4426950408889634f;
     prm.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;
   }
+  if (mx != nullptr) {
+    prm.smax = mx->smax;
+    prm.ssum = mx->ssum;
+    if (masked) {
+      const long long esz = mx->type == FA_MASK_BOOL ? 1 : (mx->type == FA_MASK_F16 ? 2 : 4);
+      prm.mask = mx->mask;
+      prm.mask_type = mx->type;
+      prm.mask_sb = mx->sb;
+      prm.mask_sh = mx->sh;
+      prm.mask_sq = mx->sq;
+      prm.mask_vec = aligned(mx->mask, 16) && (mx->sb * esz) % 16 == 0 &&
+                     (mx->sh * esz) % 16 == 0 && (mx->sq * esz) % 16 == 0;
+    }
+  }
   prm.n_splits = n_splits > 0 ? n_splits : 1;
   prm.rows_total = rows_total;
   if (n_splits > 0) {
@@ -312,15 +348,23 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     return FA_ERR_CUDA;
 
   int st = FA_ERR_HEADDIM;
-  switch (D * 2 + dtype) {
-    case 32: st = launch<16, 0>(prm, B, H, stream); break;
-    case 33: st = launch<16, 1>(prm, B, H, stream); break;
-    case 64: st = launch<32, 0>(prm, B, H, stream); break;
-    case 65: st = launch<32, 1>(prm, B, H, stream); break;
-    case 128: st = launch<64, 0>(prm, B, H, stream); break;
-    case 129: st = launch<64, 1>(prm, B, H, stream); break;
-    case 256: st = launch<128, 0>(prm, B, H, stream); break;
-    case 257: st = launch<128, 1>(prm, B, H, stream); break;
+  switch (D * 2 + dtype + (masked ? 1000 : 0)) {
+    case 32: st = launch<16, 0, false>(prm, B, H, stream); break;
+    case 33: st = launch<16, 1, false>(prm, B, H, stream); break;
+    case 64: st = launch<32, 0, false>(prm, B, H, stream); break;
+    case 65: st = launch<32, 1, false>(prm, B, H, stream); break;
+    case 128: st = launch<64, 0, false>(prm, B, H, stream); break;
+    case 129: st = launch<64, 1, false>(prm, B, H, stream); break;
+    case 256: st = launch<128, 0, false>(prm, B, H, stream); break;
+    case 257: st = launch<128, 1, false>(prm, B, H, stream); break;
+    case 1032: st = launch<16, 0, true>(prm, B, H, stream); break;
+    case 1033: st = launch<16, 1, true>(prm, B, H, stream); break;
+    case 1064: st = launch<32, 0, true>(prm, B, H, stream); break;
+    case 1065: st = launch<32, 1, true>(prm, B, H, stream); break;
+    case 1128: st = launch<64, 0, true>(prm, B, H, stream); break;
+    case 1129: st = launch<64, 1, true>(prm, B, H, stream); break;
+    case 1256: st = launch<128, 0, true>(prm, B, H, stream); break;
+    case 1257: st = launch<128, 1, true>(prm, B, H, stream); break;
   }
   if (st != FA_OK || n_splits == 0) return st;
   switch (D * 2 + dtype) {
@@ -343,7 +387,25 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
                       int causal, int window_left, int window_right, int dtype,
                       cudaStream_t stream) {
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
-                  window_right, dtype, 0, nullptr, 0, stream);
+                  window_right, dtype, 0, nullptr, 0, nullptr, stream);
+}
+
+extern "C" int fa_fwd_ex(const void *q, const void *k, const void *v, void *out, float *lse,
+                         float *softmax_max, float *softmax_sum, const void *mask,
+                         int mask_type, long long mask_stride_b, long long mask_stride_h,
+                         long long mask_stride_q, int B, int H, int H_kv, int L_q, int L_k,
+                         int D, float scale, int causal, int window_left, int window_right,
+                         int dtype, cudaStream_t stream) {
+  fa::MaskArgs mx;
+  mx.mask = mask;
+  mx.type = mask_type;
+  mx.sb = mask_stride_b;
+  mx.sh = mask_stride_h;
+  mx.sq = mask_stride_q;
+  mx.smax = softmax_max;
+  mx.ssum = softmax_sum;
+  return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                  window_right, dtype, 0, nullptr, 0, &mx, stream);
 }
 
 extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {
@@ -359,7 +421,7 @@ extern "C" int fa_fwd_splitkv(const void *q, const void *k, const void *v, void 
                               cudaStream_t stream) {
   if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
-                  window_right, dtype, n_splits, workspace, workspace_bytes, stream);
+                  window_right, dtype, n_splits, workspace, workspace_bytes, nullptr, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -562,7 +624,8 @@ extern "C" int fa_fwd_splitkv_static(const void *q, const void *k, const void *v
   const int st = fa::static_scratch(&scratch);
   if (st != FA_OK) return st;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
-                  window_right, dtype, n_splits, scratch, FA_STATIC_SCRATCH_BYTES, stream);
+                  window_right, dtype, n_splits, scratch, FA_STATIC_SCRATCH_BYTES, nullptr,
+                  stream);
 }
 
 extern "C" int fa_get_device_status(cudaStream_t stream) {

@@ -96,6 +96,17 @@ struct FwdParams {
   long long rows_total;   // B * H * L_q
   float *ws_o;        // [n_splits][rows_total][D] or nullptr
   float2 *ws_ml;      // [n_splits][rows_total]: (m in log2 units, l)
+  // optional attention mask (instances with kMask): element (b, h, i, j) at
+  // mask + b*mask_sb + h*mask_sh + i*mask_sq + j; type 1 bool (nonzero
+  // hides the key), 2 fp16 / 3 fp32 added to the scaled score
+  const void *mask;
+  int mask_type;
+  int mask_vec;       // base and strides 16-byte aligned: 16-byte loads
+  long long mask_sb, mask_sh, mask_sq;
+  // optional softmax statistics [B*H, L_q] (natural-log units): the row max
+  // of the scaled, masked scores and sum_j e^{s_j - max}; nullptr = skip
+  float *smax;
+  float *ssum;
 };
 
 template <int D>
@@ -165,7 +176,78 @@ __device__ __forceinline__ BlockRange tile_block_range(int first, int last, int 
   return r;
 }
 
-template <int D, int DT>
+// Adds the mask of key block j to a row of raw scores and applies the scale:
+// t_c = s_c * scale * log2(e) + mask_c * log2(e) (-inf where hidden), so
+// that the rest of the softmax runs in log2 units with a unit scale.
+// `base` is the row's first mask element; `n_cols` the valid keys of the
+// block (the rest are already -inf); `row_ok` false: scale only.
+__device__ __forceinline__ float mask_bias_f16(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+template <int kBNc>
+__device__ __forceinline__ void apply_mask(float (&sv)[kBNc], const FwdParams &p, long long base,
+                                           int n_cols, bool row_ok, float sl2) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (!row_ok) {
+#pragma unroll
+    for (int c = 0; c < kBNc; ++c) sv[c] *= sl2;
+    return;
+  }
+  const bool vec = p.mask_vec && n_cols >= kBNc;
+  if (p.mask_type == 1) {
+    const uint8_t *m = static_cast<const uint8_t *>(p.mask) + base;
+    if (vec) {
+#pragma unroll
+      for (int c0 = 0; c0 < kBNc; c0 += 16) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(m + c0));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          sv[c0 + u] = ((ws[u >> 2] >> (8 * (u & 3))) & 0xffu) ? -INFINITY : sv[c0 + u] * sl2;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kBNc; ++c)
+        sv[c] = (c < n_cols && m[c] != 0) ? -INFINITY : sv[c] * sl2;
+    }
+  } else if (p.mask_type == 2) {
+    const uint16_t *m = static_cast<const uint16_t *>(p.mask) + base;
+    if (vec) {
+#pragma unroll
+      for (int c0 = 0; c0 < kBNc; c0 += 8) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(m + c0));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          sv[c0 + u] = fmaf(sv[c0 + u], sl2,
+                            mask_bias_f16(static_cast<uint16_t>(ws[u >> 1] >> (16 * (u & 1)))) *
+                                kLog2e);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kBNc; ++c)
+        sv[c] = fmaf(sv[c], sl2, c < n_cols ? mask_bias_f16(m[c]) * kLog2e : 0.0f);
+    }
+  } else {
+    const float *m = static_cast<const float *>(p.mask) + base;
+    if (vec) {
+#pragma unroll
+      for (int c0 = 0; c0 < kBNc; c0 += 4) {
+        const float4 w = __ldg(reinterpret_cast<const float4 *>(m + c0));
+        sv[c0] = fmaf(sv[c0], sl2, w.x * kLog2e);
+        sv[c0 + 1] = fmaf(sv[c0 + 1], sl2, w.y * kLog2e);
+        sv[c0 + 2] = fmaf(sv[c0 + 2], sl2, w.z * kLog2e);
+        sv[c0 + 3] = fmaf(sv[c0 + 3], sl2, w.w * kLog2e);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kBNc; ++c)
+        sv[c] = fmaf(sv[c], sl2, c < n_cols ? m[c] * kLog2e : 0.0f);
+    }
+  }
+}
+
+template <int D, int DT, bool kMask>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using G = Geo<D>;
   constexpr int kSlots = G::kSlots;
@@ -489,9 +571,17 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     const int first = tq0, last = tq0 + trows - 1;
     const int full_lo = p.wl < 0 ? 0 : last - p.wl;               // block start bound
     const int full_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, first + p.wr);
-    const float sl2 = p.scale_log2;
+    // with a mask the scores are scaled (and biased) as they are loaded and
+    // the softmax below runs with a unit scale
+    const float sl2 = kMask ? 1.0f : p.scale_log2;
+    long long mask_row = 0;
+    if constexpr (kMask) {
+      const int mb = row_head / p.H, mh = row_head - (row_head / p.H) * p.H;
+      mask_row = mb * p.mask_sb + mh * p.mask_sh + static_cast<long long>(i) * p.mask_sq;
+    }
 
     float m_use = -INFINITY;   // running max (log2 units of scaled scores)
+    float m_true = -INFINITY;  // exact running max, for the softmax statistics
     float l = 0.0f;            // running normaliser, relative to m_use
     bool ok = true;
 
@@ -524,6 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             for (int c = 0; c < kBN; ++c)
               if (c < lo_c || c > hi_c) sv[c] = -INFINITY;
           }
+          if constexpr (kMask)
+            apply_mask(sv, p, mask_row + static_cast<long long>(j) * kBN,
+                       min(kBN, p.L_k - j * kBN), r_loc < trows, p.scale_log2);
         };
         const float2 sl2v = make_float2(sl2, sl2);
 
@@ -541,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                                     fmax3(mx[2], mx[3], sv[kBN - 3]),
                                     fmaxf(sv[kBN - 2], sv[kBN - 1]));
           const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
+          m_true = fmaxf(m_true, m_new);
 
           // conditional rescale: only when some row's max grew by > 2^8
           const bool need = m_new > m_use + kRescaleThreshold;
@@ -630,6 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           tc_fence_before_sync();
           mbar_arrive(smem_u32(&bars->s_free[t]));
           const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
+          m_true = fmaxf(m_true, m_new);
           const bool need = m_new > m_use + kRescaleThreshold;
           float alpha = 1.0f;
           const bool warp_rescale = __any_sync(0xffffffffu, need);
@@ -708,6 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             pk[c >> 6][pair & 31] = pack2<DT>(pp.x, pp.y);
           }
           const float m_new = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
+          m_true = fmaxf(m_true, m_new);
           if (__any_sync(0xffffffffu, m_new > m_use + kRescaleThreshold)) {
             float s2[kBN];
             load_s(s2);
@@ -827,6 +923,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                        bh);
         bulk_commit_group();
         bulk_wait_group_all();
+      }
+      if (ok && p.smax != nullptr && r_loc < trows) {
+        // statistics against the exact max: sum_j 2^(t_j - m_true) = l 2^(m_use - m_true)
+        const size_t row = static_cast<size_t>(row_head) * p.L_q + i;
+        p.smax[row] = l > 0.0f ? m_true * 0.6931471805599453f : -INFINITY;
+        p.ssum[row] = l > 0.0f ? l * ex2(m_use - m_true) : 0.0f;
       }
       if (ok && p.lse != nullptr && r_loc < trows) {
         const float lse = l > 0.0f ? (m_use + __log2f(l)) * 0.6931471805599453f : -INFINITY;

@@ -41,6 +41,13 @@ typedef enum {
 } fa_dtype;
 
 typedef enum {
+    FA_MASK_NONE = 0,
+    FA_MASK_BOOL = 1,   /* uint8; nonzero hides the key */
+    FA_MASK_F16 = 2,    /* IEEE binary16, added to the scaled score */
+    FA_MASK_F32 = 3     /* binary32, added to the scaled score */
+} fa_mask_type;
+
+typedef enum {
     FA_OK = 0,
     FA_ERR_NULL = -1,     /* q or out is NULL while L_q > 0, or k or v is
                              NULL while L_k > 0 */
@@ -92,6 +99,34 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
            int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
            int causal, int window_left, int window_right, int dtype,
            cudaStream_t stream);
+
+/*
+ * fa_fwd_ex -- fa_fwd with the optional inputs and outputs of the operator
+ * statement in "FlashAttention算法原理与性能优化实战" §2.2: an attention mask
+ * and the two softmax statistics kept for the backward pass.
+ *
+ *   mask, mask_type  device, or NULL with FA_MASK_NONE.  Element
+ *               (b, h, i, j) is mask[b*mask_stride_b + h*mask_stride_h +
+ *               i*mask_stride_q + j] (strides in elements, >= 0; a stride
+ *               of 0 broadcasts, e.g. [L_q, L_k] for every batch and head:
+ *               0, 0, L_k).  FA_MASK_BOOL: a nonzero byte hides key j from
+ *               query i.  FA_MASK_F16 / FA_MASK_F32: the value is added to
+ *               scale * q_i . k_j before the softmax (-inf hides).  The
+ *               causal / window rule applies on top.  The caller guarantees
+ *               every addressed element lies in the buffer.  16-byte
+ *               aligned base and strides take the vectorised load path.
+ *   softmax_max, softmax_sum  device [B, H, L_q] fp32, both or neither
+ *               (NULL): the row max m_i of the scaled, masked scores and
+ *               sum_j exp(s_ij - m_i); lse = m + ln(sum).  A row with no
+ *               visible key gets -inf and 0.
+ * Other arguments, errors and edge cases as fa_fwd; FA_ERR_ARG for a bad
+ * mask_type or a negative stride.
+ */
+int fa_fwd_ex(const void *q, const void *k, const void *v, void *out, float *lse,
+              float *softmax_max, float *softmax_sum, const void *mask, int mask_type,
+              long long mask_stride_b, long long mask_stride_h, long long mask_stride_q,
+              int B, int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
+              int window_left, int window_right, int dtype, cudaStream_t stream);
 
 /*
  * fa_splitkv_workspace_bytes -- bytes of device workspace fa_fwd_splitkv

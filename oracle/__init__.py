@@ -108,7 +108,7 @@ class Oracle:
         lib.oracle_attention_rows_ex.argtypes = [
             u16p, u16p, u16p, ctypes.c_int, i64, i64, i64, i64, i64, i64,
             ctypes.c_double, ctypes.c_int, i64, i64, ctypes.c_void_p, ctypes.c_int, i64, i64,
-            i64, i64p, i64, dp, dp, dp, dp, ctypes.c_int]
+            i64, i64p, i64, dp, dp, dp, dp, dp, ctypes.c_int]
         lib.oracle_attention_rows_ex.restype = ctypes.c_int
         lib.oracle_attention_f64.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, i64,
                                              ctypes.c_double, ctypes.c_int, i64, i64, dp, dp]
@@ -255,9 +255,11 @@ class Oracle:
         return m, types[m.dtype], st[0], st[1], st[2]
 
     def attention_rows_ex(self, q, k, v, dtype, scale, causal=False, window_left=-1,
-                          window_right=-1, mask=None, rows=None, n_threads=0):
+                          window_right=-1, mask=None, rows=None, n_threads=0,
+                          with_wabs=False):
         """Exact attention with an optional mask (see attention_ref.c for
-        its reading); returns (out [n, D], lse, softmax_max, softmax_sum)."""
+        its reading); returns (out [n, D], lse, softmax_max, softmax_sum),
+        plus wabs [n, D] with ``with_wabs``."""
         q, k, v, B, H, H_kv, L_q, L_k, D = _shape_args(q, k, v)
         m, mtype, sb, sh, sq = self.mask_args(mask, B, H, L_q, L_k)
         if rows is None:
@@ -266,6 +268,7 @@ class Oracle:
             rows = np.ascontiguousarray(rows, dtype=np.int64)
             n, rows_p = rows.size, _ptr(rows, ctypes.c_int64)
         out = np.zeros((n, D), dtype=np.float64)
+        wabs = np.zeros((n, D), dtype=np.float64) if with_wabs else None
         lse, smax, ssum = (np.zeros((n,), dtype=np.float64) for _ in range(3))
         rc = self.lib.oracle_attention_rows_ex(
             _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
@@ -273,9 +276,12 @@ class Oracle:
             int(window_left), int(window_right),
             m.ctypes.data_as(ctypes.c_void_p) if m is not None else None, mtype, sb, sh, sq,
             rows_p, n, _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
+            _ptr(wabs, ctypes.c_double) if with_wabs else None,
             _ptr(smax, ctypes.c_double), _ptr(ssum, ctypes.c_double), int(n_threads))
         if rc < 0:
             raise ValueError("oracle rejected the arguments")
+        if with_wabs:
+            return out, lse, smax, ssum, wabs
         return out, lse, smax, ssum
 
     # ------------------------------------------------------------- fp64 inputs

@@ -341,7 +341,7 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
                      out, lse, wabs, NULL, NULL, n_threads);
 }
 
-/* The same with a mask and the two softmax statistics (smax, ssum
+/* The same with a mask and the two softmax statistics (wabs, smax, ssum
  * nullable), as stated above the mask helpers. */
 int oracle_attention_rows_ex(const uint16_t *q, const uint16_t *k,
                              const uint16_t *v, int dtype, int64_t B, int64_t H,
@@ -351,11 +351,12 @@ int oracle_attention_rows_ex(const uint16_t *q, const uint16_t *k,
                              int mask_type, int64_t stride_b, int64_t stride_h,
                              int64_t stride_q, const int64_t *rows,
                              int64_t n_rows, double *out, double *lse,
-                             double *smax, double *ssum, int n_threads)
+                             double *wabs, double *smax, double *ssum,
+                             int n_threads)
 {
     return rows_core(q, k, v, dtype, B, H, H_kv, L_q, L_k, D, scale, causal,
                      window_left, window_right, mask, mask_type, stride_b,
-                     stride_h, stride_q, rows, n_rows, out, lse, NULL, smax,
+                     stride_h, stride_q, rows, n_rows, out, lse, wabs, smax,
                      ssum, n_threads);
 }
 

@@ -199,3 +199,21 @@ def test_bwd_workspace_bytes(lib):
 ])
 def test_bwd_argument_errors(lib, kw, code):
     assert _call_bwd(**kw) == code
+
+
+# ------------------------------------------------------------ masked / statistics entry
+def _call_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, smax=0, ssum=0, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_ex(a["q"], a["k"], a["v"], a["out"], a["lse"], smax, ssum, mask, mtype,
+                        sb, sh, sq, a["B"], a["H"], a["H_kv"], a["L_q"], a["L_k"], a["D"],
+                        a["scale"], a["causal"], a["wl"], a["wr"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mtype=4), -6), (dict(mtype=-1), -6), (dict(sq=-1), -6), (dict(sb=-8), -6),
+    (dict(mask=0), -1), (dict(smax=16, ssum=0), -1), (dict(smax=0, ssum=16), -1),
+    (dict(smax=18, ssum=16), -5), (dict(q=0), -1), (dict(D=48), -3),
+])
+def test_ex_argument_errors(lib, kw, code):
+    assert _call_ex(**kw) == code
