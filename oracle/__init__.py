@@ -33,7 +33,7 @@ _BUILD_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
 _lock = threading.Lock()
 
-F16, BF16 = 0, 1
+F16, BF16, E4M3 = 0, 1, 2
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
@@ -55,12 +55,17 @@ def _ptr(a: np.ndarray, ctype):
 
 
 def _bits(x) -> np.ndarray:
-    """Accept a numpy uint16/int16 array of bit patterns."""
+    """Accept a numpy uint16/int16 array of fp16/bf16 bit patterns, or a
+    uint8/int8 array of fp8 e4m3 codes (widened to uint16)."""
     a = np.ascontiguousarray(x)
     if a.dtype == np.int16:
         a = a.view(np.uint16)
+    if a.dtype == np.int8:
+        a = a.view(np.uint8)
+    if a.dtype == np.uint8:
+        a = a.astype(np.uint16)
     if a.dtype != np.uint16:
-        raise TypeError("oracle inputs are fp16/bf16 bit patterns (uint16)")
+        raise TypeError("oracle inputs are fp16/bf16 (uint16) or e4m3 (uint8) bit patterns")
     return a
 
 
@@ -88,6 +93,8 @@ class Oracle:
         lib.oracle_f16_to_f64.restype = ctypes.c_double
         lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_to_f64.restype = ctypes.c_double
+        lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f64.restype = ctypes.c_double
         lib.oracle_f64_to_f16.argtypes = [ctypes.c_double]
         lib.oracle_f64_to_f16.restype = ctypes.c_uint16
         lib.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
@@ -127,6 +134,9 @@ class Oracle:
     def bf16_to_f64(self, bits: int) -> float:
         return self.lib.oracle_bf16_to_f64(int(bits) & 0xFFFF)
 
+    def e4m3_to_f64(self, bits: int) -> float:
+        return self.lib.oracle_e4m3_to_f64(int(bits) & 0xFF)
+
     def f64_to_f16(self, x: float) -> int:
         return int(self.lib.oracle_f64_to_f16(float(x)))
 
@@ -134,10 +144,10 @@ class Oracle:
         return int(self.lib.oracle_f64_to_bf16(float(x)))
 
     def decode(self, bits, dtype: int) -> np.ndarray:
-        """Elementwise decode of fp16/bf16 bit patterns to float64."""
+        """Elementwise decode of fp16/bf16 (or e4m3) bit patterns to float64."""
         dtype = int(dtype)
         if dtype not in self._tables:
-            fn = self.f16_to_f64 if dtype == F16 else self.bf16_to_f64
+            fn = {F16: self.f16_to_f64, BF16: self.bf16_to_f64, E4M3: self.e4m3_to_f64}[dtype]
             self._tables[dtype] = np.array([fn(b) for b in range(65536)],
                                            dtype=np.float64)
         return self._tables[dtype][_bits(bits)]
@@ -351,7 +361,7 @@ def get() -> Oracle:
 
 def __getattr__(name):
     # module-level convenience: oracle.attention(...), oracle.decode(...), ...
-    if name in {"f16_to_f64", "bf16_to_f64", "f64_to_f16", "f64_to_bf16",
+    if name in {"f16_to_f64", "bf16_to_f64", "e4m3_to_f64", "f64_to_f16", "f64_to_bf16",
                 "decode", "round_to", "safe_softmax", "online_softmax",
                 "attention_rows", "attention", "attention_rows_online",
                 "attention_f64", "attention_bwd_f64", "attention_bwd",

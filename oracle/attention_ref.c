@@ -32,7 +32,8 @@
  *   A row with no visible key has O = 0 and lse = -inf (the pages are
  *   silent; this is the stated reading).
  *
- * Inputs are raw fp16 or bf16 bit patterns; this file decodes them itself.
+ * Inputs are raw bit patterns (fp16, bf16, or fp8 e4m3 codes widened to 16
+ * bits); this file decodes them itself.
  */
 #include <math.h>
 #include <stdint.h>
@@ -111,6 +112,26 @@ static uint16_t round_rne(double x, int mbits, int bias)
     return sign | (uint16_t)(eb << mbits) | (uint16_t)((uint32_t)r - (1u << mbits));
 }
 
+/* FP8 E4M3 (the "fn" variant: no infinities, S.1111.111 is NaN, largest
+ * finite 448): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+ * exponent field 0 holds the subnormals m * 2^-9.  The pages name fp8 as an
+ * input type of FlashAttention-2 ("PyTorch Transformer Flash Attention机制",
+ * section 5); the format itself is the standard OCP FP8 E4M3 encoding. */
+double oracle_e4m3_to_f64(uint8_t x)
+{
+    int sign = (x >> 7) & 1;
+    int e = (x >> 3) & 0xf;
+    int m = x & 0x7;
+    double v;
+    if (e == 0xf && m == 0x7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -9);                /* subnormal: m * 2^-9 */
+    else
+        v = ldexp((double)(8 + m), e - 10);      /* 1.m * 2^(e-7) */
+    return sign ? -v : v;
+}
+
 uint16_t oracle_f64_to_f16(double x) { return round_rne(x, 10, 15); }
 uint16_t oracle_f64_to_bf16(double x) { return round_rne(x, 7, 127); }
 
@@ -171,11 +192,13 @@ static int visible(int64_t i, int64_t j, int64_t L_k, int causal,
     return 1;
 }
 
+/* dtype 0 fp16, 1 bf16, 2 fp8 e4m3 (the code in the low byte). */
 static void build_decode_table(int dtype, double *tab)
 {
     for (uint32_t b = 0; b < 65536u; b++)
         tab[b] = dtype == 0 ? oracle_f16_to_f64((uint16_t)b)
-                            : oracle_bf16_to_f64((uint16_t)b);
+               : dtype == 1 ? oracle_bf16_to_f64((uint16_t)b)
+                            : oracle_e4m3_to_f64((uint8_t)(b & 0xff));
 }
 
 /* ---------------------------------------------------------------------
@@ -243,7 +266,7 @@ static int rows_core(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 {
     if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1)
         return -1;
-    if (H % H_kv != 0 || (dtype != 0 && dtype != 1))
+    if (H % H_kv != 0 || dtype < 0 || dtype > 2)
         return -1;
     if (mask_type < 0 || mask_type > 3 || (mask_type != 0 && mask == NULL))
         return -1;

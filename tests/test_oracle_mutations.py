@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import tests.test_oracle_bwd_pins as bwd_pins
+import tests.test_oracle_fp8_pins as fp8_pins
 import tests.test_oracle_mask_pins as mask_pins
 import tests.test_oracle_pins as pins
 from exact_attention_113_b200.inputs import F16, BF16
@@ -57,6 +58,11 @@ MUTATIONS = {
                        "if (dva) dva[j * D + d] += p[j] * doi[d];"),
     "bwd_abs_delta_term_dropped": ("const double wabs_j = fabs(ds[j]) + p[j] * e;",
                                    "const double wabs_j = fabs(ds[j]);"),
+    # fp8
+    "e4m3_bias": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 9);"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);                /* subnormal: m * 2^-9 */",
+                             "v = ldexp((double)m, -10);"),
+    "e4m3_nan_missed": ("if (e == 0xf && m == 0x7)", "if (e == 0xf && m == 0x8)"),
     # mask and statistics
     "mask_bool_inverted": ("*hidden = ((const uint8_t *)mask)[idx] != 0;",
                            "*hidden = ((const uint8_t *)mask)[idx] == 0;"),
@@ -99,6 +105,9 @@ def _battery(orc):
     for dt in (F16, BF16):
         yield lambda dt=dt: bwd_pins.test_bit_pattern_entry_decodes_exactly(orc, dt)
     yield lambda: bwd_pins.test_error_scales(orc)
+    yield lambda: fp8_pins.test_decode_every_code_matches_torch(orc)
+    yield lambda: fp8_pins.test_decode_closed_points(orc)
+    yield lambda: fp8_pins.test_attention_on_e4m3_equals_fp16_of_same_values(orc)
     yield lambda: mask_pins.test_empty_masks_change_nothing(orc)
     yield lambda: mask_pins.test_causal_pattern_masks(orc)
     yield lambda: mask_pins.test_row_constant_shift(orc)
