@@ -21,6 +21,10 @@ slowest rank's time.
 lse): a step is its three launches (delta / lse prep, the gradient kernel,
 the dQ conversion); the metric counts 2.5x the forward's FLOPs.
 
+--fp8 times fa_fwd_fp8 on the workload's inputs converted to E4M3 (bf16
+output); its roofline peak is the measured bf16 rate x 2 (the nominal
+fp8 / bf16 ratio of the tensor cores).
+
 --splits S (or auto) times fa_fwd_splitkv instead: one split-KV launch plus
 one merge launch per step, for the decoding workloads (a few query rows, a
 long key/value cache), whose roofline is HBM bandwidth rather than the
@@ -279,9 +283,10 @@ def run_ours(args, w: W.Workload):
 
     # per-rank problem: same shape, its own seed (weak scaling)
     w_rank = W.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
-    q_cpu, k_cpu, v_cpu = W.make_qkv(w_rank)
+    fp8 = getattr(args, "fp8", False)
+    q_cpu, k_cpu, v_cpu = W.make_qkv_fp8(w_rank) if fp8 else W.make_qkv(w_rank)
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev) if fp8 else torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.L_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     bwd = args.pass_ == "bwd"
@@ -308,6 +313,11 @@ def run_ours(args, w: W.Workload):
             fa.flash_bwd(q, k, v, out, dout, lse, scale=w.softmax_scale, causal=w.causal,
                          window_left=w.window_left, window_right=w.window_right, dq=dq, dk=dk,
                          dv=dv, workspace=bws, stream=stream)
+    elif fp8:
+        def step():
+            fa.flash_fwd_fp8(q, k, v, scale=w.softmax_scale, causal=w.causal,
+                             window_left=w.window_left, window_right=w.window_right,
+                             out=out, lse=lse, stream=stream)
     else:
         def step():
             fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
@@ -347,13 +357,16 @@ def run_ours(args, w: W.Workload):
     # ---- roofline of the (only) kernel
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    if fp8:
+        peak *= 2.0                 # nominal fp8 / bf16 dense ratio
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     if bwd or roofline_bound(w, peak, hbm) == "tensor":
         achieved = fm * algorithmic_flops(w) / avg_launch_s / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "traffic": profiled_traffic() if w.name == W.ROOFLINE.name else None,
-                    "peak_source": f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)"}
+                    "peak_source": (f"{peak_kind} cuBLAS bf16 burst x 2 (nominal fp8 ratio)" if fp8
+                                    else f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)")}
     else:
         achieved = min_hbm_bytes(w) / avg_launch_s / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
@@ -411,7 +424,7 @@ def run_ours(args, w: W.Workload):
                "steps": n_e2e, "ms_per_step": round(e2e_s / n_e2e * 1e3, 3)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu_baseline and not bwd:
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline and not bwd and not fp8:
         tf, cores, desc = cpu_oracle_sample(w, q_cpu, k_cpu, v_cpu, args.cpu_seconds)
         cpu = {"value": round(tf, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": desc, "host_nproc": os.cpu_count()}
@@ -422,7 +435,7 @@ def run_ours(args, w: W.Workload):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(max_total / args.steps * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16" if w.dtype == W.F16 else "bf16",
+        "dtype": "e4m3" if fp8 else ("f16" if w.dtype == W.F16 else "bf16"),
         "data": "synthetic (seeded N(0,%g) inputs, per-rank seeds)" % w.std,
         "config": workload_config(w, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
@@ -530,6 +543,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.ALL))
     ap.add_argument("--pass", dest="pass_", choices=("fwd", "bwd"), default="fwd",
                     help="time the forward (default) or the backward")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time fa_fwd_fp8 on the inputs converted to E4M3")
     ap.add_argument("--splits", default="0",
                     help="key slices for fa_fwd_splitkv (0: plain fa_fwd; auto)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")

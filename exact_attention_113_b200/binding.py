@@ -24,7 +24,8 @@ STATUS = {
     -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE", -10: "FA_ERR_SCRATCH",
 }
 FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
-EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_splitkv",
+EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
+           "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_splitkv_workspace_bytes",
            "fa_status_string", "fa_version")
 # size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
@@ -62,6 +63,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, ll, ll, ll, i, i, i, i, i,
                                   i, ctypes.c_float, i, i, i, i, vp]
         lib.fa_fwd_ex.restype = i
+        f = ctypes.c_float
+        lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, i, i, vp]
+        lib.fa_fwd_fp8.restype = i
         lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
                                        i, i, i, i, i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_splitkv.restype = i
@@ -102,6 +106,14 @@ def fa_fwd_ex(q, k, v, out, lse, softmax_max, softmax_sum, mask, mask_type, mask
                             int(mask_stride_b), int(mask_stride_h), int(mask_stride_q), B, H,
                             H_kv, L_q, L_k, D, float(scale), int(causal), int(window_left),
                             int(window_right), int(dtype), stream)
+
+
+def fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
+               descale_v, causal, window_left, window_right, stream) -> int:
+    """The fp8 (E4M3) C entry point, unchanged."""
+    return load().fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, float(scale),
+                             float(descale_q), float(descale_k), float(descale_v), int(causal),
+                             int(window_left), int(window_right), stream)
 
 
 def mask_layout(mask, B, H, L_q, L_k):
@@ -346,3 +358,38 @@ def flash_bwd(q, k, v, out, dout, lse, scale=None, causal=False, window_left=-1,
     if st != FA_OK:
         raise FaError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1.0,
+                  causal=False, window_left=-1, window_right=-1, return_lse=True, out=None,
+                  lse=None, stream=None):
+    """Exact attention forward on fp8 E4M3 CUDA tensors (torch.float8_e4m3fn
+    or uint8 codes), q [B, H, L_q, D], k, v [B, H_kv, L_k, D]; real values are
+    code * descale.  Returns (out bf16 [B, H, L_q, D], lse or None)."""
+    import torch
+
+    B, H, L_q, D = q.shape
+    _, H_kv, L_k, _ = k.shape
+    ok_types = (torch.float8_e4m3fn, torch.uint8)
+    if any(t.dtype not in ok_types for t in (q, k, v)) or tuple(v.shape) != tuple(k.shape):
+        raise TypeError("q, k, v must be float8_e4m3fn (or uint8 codes), k and v of one shape")
+    if not all(t.is_cuda and t.is_contiguous() for t in (q, k, v)):
+        raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, H, L_q, D), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, L_q), dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        st = fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                        lse.data_ptr() if lse is not None else None, B, H, H_kv, L_q, L_k, D,
+                        scale, descale_q, descale_k, descale_v, causal, window_left,
+                        window_right, stream.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_fp8")
+    return out, lse

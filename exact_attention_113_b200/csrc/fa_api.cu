@@ -53,16 +53,19 @@ bool encode_map(CUtensorMap *map, const void *base, int dtype, int n_heads, int 
                 int box_cols, int box_rows = kBM, int box_heads = 1) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const CUtensorMapDataType dt =
-      dtype == FA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // dtype 0 fp16, 1 bf16, 2 fp8 e4m3 (moved as bytes)
+  const CUtensorMapDataType dt = dtype == FA_F16    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                 : dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const cuuint64_t es = dtype == 2 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                         static_cast<cuuint64_t>(n_heads)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                           static_cast<cuuint64_t>(L) * D * 2};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * es,
+                           static_cast<cuuint64_t>(L) * D * es};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows),
                        static_cast<cuuint32_t>(box_heads)};
   cuuint32_t estr[3] = {1, 1, 1};
-  const int sw_bytes = box_cols * 2;
+  const int sw_bytes = box_cols * static_cast<int>(es);
   const CUtensorMapSwizzle sw = sw_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : sw_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -193,20 +196,24 @@ int launch_combine(const float *ws_o, const float2 *ws_ml, void *out, float *lse
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// Optional mask and softmax statistics of fa_fwd_ex.
-struct MaskArgs {
-  const void *mask;
-  int type;                        // FA_MASK_*
-  long long sb, sh, sq;            // element strides
-  float *smax, *ssum;
+// Optional inputs / outputs beyond fa_fwd's: the mask and softmax
+// statistics of fa_fwd_ex, the value descale of fa_fwd_fp8.
+struct FwdExtras {
+  const void *mask = nullptr;
+  int type = FA_MASK_NONE;         // FA_MASK_*
+  long long sb = 0, sh = 0, sq = 0;   // element strides
+  float *smax = nullptr, *ssum = nullptr;
+  float descale_v = 1.0f;
 };
+
+constexpr int kE4M3 = 2;           // internal dtype code of fp8 e4m3 inputs
 
 // Shared body of fa_fwd, fa_fwd_ex and fa_fwd_splitkv (n_splits == 0: plain
 // forward; mx == nullptr: no mask, no statistics).
 int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
              int H_kv, int L_q, int L_k, int D, float scale, int causal, int window_left,
              int window_right, int dtype, int n_splits, void *workspace,
-             size_t workspace_bytes, const MaskArgs *mx, cudaStream_t stream);
+             size_t workspace_bytes, const FwdExtras *mx, cudaStream_t stream);
 
 }  // namespace
 }  // namespace fa
@@ -218,7 +225,7 @@ namespace {
 int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
              int H_kv, int L_q, int L_k, int D, float scale, int causal, int window_left,
              int window_right, int dtype, int n_splits, void *workspace,
-             size_t workspace_bytes, const MaskArgs *mx, cudaStream_t stream) {
+             size_t workspace_bytes, const FwdExtras *mx, cudaStream_t stream) {
   // ---------------------------------------------------------------- checks
   if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
   // a pointer may be NULL only when its tensor has no elements
@@ -229,7 +236,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
       (1ll << 31) - 1)
     return FA_ERR_SHAPE;                   // at most one CTA per (head, 128 query rows)
   if (D != 16 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
-  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (dtype != FA_F16 && dtype != FA_BF16 && dtype != kE4M3) return FA_ERR_DTYPE;
+  if (dtype == kE4M3 && D < 32) return FA_ERR_HEADDIM;   // rows of >= 32 bytes
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return FA_ERR_ALIGN;
   if (lse && !aligned(lse, 4)) return FA_ERR_ALIGN;
@@ -242,6 +250,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     if ((mx->smax == nullptr) != (mx->ssum == nullptr)) return FA_ERR_NULL;
     if (L_q > 0 && (!aligned(mx->smax, 4) || !aligned(mx->ssum, 4))) return FA_ERR_ALIGN;
   }
+  // fp8 inputs only through fa_fwd_fp8: no key slices, no mask
+  if (dtype == kE4M3 && (n_splits != 0 || masked)) return FA_ERR_DTYPE;
   const int64_t rows_total = static_cast<int64_t>(B) * H * L_q;
   if (n_splits != 0) {
     if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
@@ -332,6 +342,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
                      (mx->sh * esz) % 16 == 0 && (mx->sq * esz) % 16 == 0;
     }
   }
+  prm.out_ptr = out;
+  prm.descale_v = mx != nullptr ? mx->descale_v : 1.0f;
   prm.n_splits = n_splits > 0 ? n_splits : 1;
   prm.rows_total = rows_total;
   if (n_splits > 0) {
@@ -339,12 +351,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     prm.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) +
                                            ws_ml_offset(rows_total, D, n_splits));
   }
-  const int box_cols = D * 2 >= 128 ? 64 : D;
+  const int esz = dtype == kE4M3 ? 1 : 2;
+  const int box_cols = D * esz >= 128 ? 128 / esz : D;
   const int q_box_heads = prm.packed ? prm.group : 1;
   if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols, prm.tile_q, q_box_heads) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
-      !encode_map(&prm.tm_o, out, dtype, B * H, L_q, D, box_cols, prm.tile_q, q_box_heads))
+      !encode_map(&prm.tm_o, out, dtype == kE4M3 ? FA_BF16 : dtype, B * H, L_q, D,
+                  D * 2 >= 128 ? 64 : D, prm.tile_q, q_box_heads))
     return FA_ERR_CUDA;
 
   int st = FA_ERR_HEADDIM;
@@ -365,6 +379,9 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 1129: st = launch<64, 1, true>(prm, B, H, stream); break;
     case 1256: st = launch<128, 0, true>(prm, B, H, stream); break;
     case 1257: st = launch<128, 1, true>(prm, B, H, stream); break;
+    case 66: st = launch<32, kE4M3, false>(prm, B, H, stream); break;
+    case 130: st = launch<64, kE4M3, false>(prm, B, H, stream); break;
+    case 258: st = launch<128, kE4M3, false>(prm, B, H, stream); break;
   }
   if (st != FA_OK || n_splits == 0) return st;
   switch (D * 2 + dtype) {
@@ -386,6 +403,7 @@ extern "C" int fa_fwd(const void *q, const void *k, const void *v, void *out, fl
                       int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
                       int causal, int window_left, int window_right, int dtype,
                       cudaStream_t stream) {
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
                   window_right, dtype, 0, nullptr, 0, nullptr, stream);
 }
@@ -396,7 +414,8 @@ extern "C" int fa_fwd_ex(const void *q, const void *k, const void *v, void *out,
                          long long mask_stride_q, int B, int H, int H_kv, int L_q, int L_k,
                          int D, float scale, int causal, int window_left, int window_right,
                          int dtype, cudaStream_t stream) {
-  fa::MaskArgs mx;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  fa::FwdExtras mx;
   mx.mask = mask;
   mx.type = mask_type;
   mx.sb = mask_stride_b;
@@ -406,6 +425,21 @@ extern "C" int fa_fwd_ex(const void *q, const void *k, const void *v, void *out,
   mx.ssum = softmax_sum;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
                   window_right, dtype, 0, nullptr, 0, &mx, stream);
+}
+
+extern "C" int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse,
+                          int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                          float descale_q, float descale_k, float descale_v, int causal,
+                          int window_left, int window_right, cudaStream_t stream) {
+  for (float d : {descale_q, descale_k, descale_v})
+    if (!std::isfinite(d) || d < 0.0f) return FA_ERR_ARG;
+  if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+  const float s = scale * descale_q * descale_k;   // the scores' full scale
+  if (!std::isfinite(s)) return FA_ERR_ARG;
+  fa::FwdExtras ex;
+  ex.descale_v = descale_v;
+  return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, s, causal, window_left,
+                  window_right, fa::kE4M3, 0, nullptr, 0, &ex, stream);
 }
 
 extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {

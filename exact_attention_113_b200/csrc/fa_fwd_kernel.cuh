@@ -103,22 +103,29 @@ struct FwdParams {
   int mask_type;
   int mask_vec;       // base and strides 16-byte aligned: 16-byte loads
   long long mask_sb, mask_sh, mask_sq;
+  // fp8 inputs (DT = 2): bf16 output written straight from registers to
+  // out_ptr [B*H, L_q, D], O scaled by descale_v
+  void *out_ptr;
+  float descale_v;
   // optional softmax statistics [B*H, L_q] (natural-log units): the row max
   // of the scaled, masked scores and sum_j e^{s_j - max}; nullptr = skip
   float *smax;
   float *ssum;
 };
 
-template <int D>
+// Tile geometry for head dim D and element size ES bytes (2: fp16 / bf16,
+// 1: fp8 e4m3).
+template <int D, int ES = 2>
 struct Geo {
-  static constexpr int kRowBytes = D * 2;
+  static constexpr int kRowBytes = D * ES;
   static constexpr int kSwBytes = kRowBytes >= 128 ? 128 : kRowBytes;  // swizzle span
-  static constexpr int kBoxCols = kSwBytes / 2;                       // elements per box row
+  static constexpr int kBoxCols = kSwBytes / ES;                      // elements per box row
   static constexpr int kNumBox = kRowBytes / kSwBytes;                 // column boxes per tile
   static constexpr int kBoxBytes = kBM * kSwBytes;
   static constexpr int kTileBytes = kBM * kRowBytes;
-  static constexpr int kSlotsK = D == 128 ? 3 : (D == 64 ? 4 : 8);
-  static constexpr int kSlotsV = D == 128 ? 2 : (D == 64 ? 4 : 8);
+  static_assert(kSwBytes >= 32, "rows of at least 32 bytes (a swizzle span)");
+  static constexpr int kSlotsK = kTileBytes >= 32768 ? 3 : (kTileBytes >= 16384 ? 4 : 8);
+  static constexpr int kSlotsV = kTileBytes >= 32768 ? 2 : (kTileBytes >= 16384 ? 4 : 8);
   static constexpr int kSlots = kSlotsK + kSlotsV;
   static constexpr uint32_t kLayout = kSwBytes == 128 ? 2u : (kSwBytes == 64 ? 4u : 6u);
   static constexpr int kUnitsPerBoxRow = kSwBytes / 16;
@@ -247,9 +254,33 @@ __device__ __forceinline__ void apply_mask(float (&sv)[kBNc], const FwdParams &p
   }
 }
 
+// P of one half-row (64 keys) into 32-bit TMEM words: two 16-bit values a
+// word, or four E4M3 codes a word (fp8 inputs); pair index p = key / 2.
+template <int DT>
+__device__ __forceinline__ void put_p(uint32_t (&pk)[32], int p, float a, float b) {
+  if constexpr (DT == 2) {
+    const uint32_t h = pack_e4m3x2(a, b);
+    pk[p >> 1] = (p & 1) ? (pk[p >> 1] | (h << 16)) : h;
+  } else {
+    pk[p] = pack2<DT>(a, b);
+  }
+}
+// Store a half-row of P at TMEM columns base + half * (32 or 16).
+template <int DT>
+__device__ __forceinline__ void store_p_half(uint32_t base, int half, const uint32_t (&pk)[32]) {
+  if constexpr (DT == 2)
+    tmem_st_x16(base + 16u * half, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+  else
+    tmem_st_x32(base + 32u * half, pk);
+}
+
 template <int D, int DT, bool kMask>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using G = Geo<D>;
+  // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 inputs (bf16 output)
+  constexpr bool kF8 = DT == 2;
+  constexpr int kES = kF8 ? 1 : 2;
+  constexpr int kKStep = 32 / kES;             // K of one MMA instruction (32 bytes)
+  using G = Geo<D, kES>;
   constexpr int kSlots = G::kSlots;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -410,8 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     // =================================================== MMA issuer
     // The whole warp runs the loop; one elected lane (always the same one,
     // so that its commits track its own MMAs) issues the tcgen05 ops.
-    constexpr uint32_t kIdescS = make_idesc_f16(kBM, kBN, DT, 0, 0);
-    constexpr uint32_t kIdescPV = make_idesc_f16(kBM, D, DT, 0, 1);
+    constexpr uint32_t kIdescS =
+        kF8 ? make_idesc_e4m3(kBM, kBN, 0, 0) : make_idesc_f16(kBM, kBN, DT, 0, 0);
+    constexpr uint32_t kIdescPV =
+        kF8 ? make_idesc_e4m3(kBM, D, 0, 1) : make_idesc_f16(kBM, D, DT, 0, 1);
     constexpr uint32_t kHi = desc_hi(8 * G::kSwBytes, G::kLayout);   // K- and MN-major
     if (any_work) {
       bool ok = true;
@@ -426,11 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         const uint32_t d_tmem = tmem + (t ? 128u : 0u);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D / kKStep; ++kk) {
             const int byte = kk * 32;
             const uint32_t off = ((byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes)) >> 4;
-            mma_ss(d_tmem, desc_join(qlo + off, kHi), desc_join(klo + off, kHi), kIdescS,
-                   kk > 0 ? 1u : 0u);
+            mma_ss_t<kF8>(d_tmem, desc_join(qlo + off, kHi), desc_join(klo + off, kHi), kIdescS,
+                          kk > 0 ? 1u : 0u);
           }
           tc_commit(smem_u32(&bars->s_full[t]));
         }
@@ -443,9 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         const bool first = (t ? npv1 : npv0) == 0;
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(d_tmem, a_tmem + kk * 8, desc_join(vlo + ((kk * 16 * G::kSwBytes) >> 4), kHi),
-                   kIdescPV, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBN / kKStep; ++kk)
+            mma_ts_t<kF8>(d_tmem, a_tmem + kk * 8,
+                          desc_join(vlo + ((kk * kKStep * G::kSwBytes) >> 4), kHi), kIdescPV,
+                          (!first || kk > 0) ? 1u : 0u);
           tc_commit(smem_u32(&bars->pv_done[t]));
         }
         __syncwarp();
@@ -669,9 +703,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                 // l sums the unrounded fp32 weights: lse = m + ln(l) then
                 // keeps fp32 accuracy whatever the input type
                 ls[(c >> 1) & 1] = __fadd2_rn(ls[(c >> 1) & 1], pp);
-                pk[c >> 1] = pack2<DT>(pp.x, pp.y);
+                put_p<DT>(pk, c >> 1, pp.x, pp.y);
               }
-              tmem_st_x32(tS + half * 32, pk);
+              store_p_half<DT>(tS, half, pk);
             }
           };
           // masked entries are -inf: only MUFU's ex2 turns them into exact 0
@@ -748,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             else
               pp = make_float2(ex2(x.x), ex2(x.y));
             ls[pair & 1] = __fadd2_rn(ls[pair & 1], pp);
-            pk[c >> 6][pair & 31] = pack2<DT>(pp.x, pp.y);
+            put_p<DT>(pk[c >> 6], pair & 31, pp.x, pp.y);
           }
           l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
           // P_t and O_t are read / written by PV_t(j-1): wait for it
@@ -758,8 +792,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             tc_fence_after_sync();
           }
           if (ok) {
-            tmem_st_x32(tPs + 0, pk[0]);
-            tmem_st_x32(tPs + 32, pk[1]);
+            store_p_half<DT>(tPs, 0, pk[0]);
+            store_p_half<DT>(tPs, 1, pk[1]);
             if (warp_rescale && n > 0) {
               constexpr int kChunk = D >= 32 ? 32 : D;
 #pragma unroll
@@ -800,7 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             else
               pp = make_float2(ex2(x.x), ex2(x.y));
             ls2[pair & 1] = __fadd2_rn(ls2[pair & 1], pp);
-            pk[c >> 6][pair & 31] = pack2<DT>(pp.x, pp.y);
+            put_p<DT>(pk[c >> 6], pair & 31, pp.x, pp.y);
           }
           const float m_new = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
           m_true = fmaxf(m_true, m_new);
@@ -809,8 +843,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             load_s(s2);
             exact_pass(s2);
           } else {
-            tmem_st_x32(tS + 0, pk[0]);
-            tmem_st_x32(tS + 32, pk[1]);
+            store_p_half<DT>(tS, 0, pk[0]);
+            store_p_half<DT>(tS, 1, pk[1]);
             l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
           }
         } else {
@@ -877,6 +911,37 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
       };
+      if constexpr (kF8) {
+        // fp8 inputs: bf16 rows straight to global memory (the 8-bit Q
+        // tile is too small to stage them); every lane loads TMEM, the
+        // lanes of real rows store
+        if (ok) {
+          const float sc = inv_l * p.descale_v;
+          uint8_t *orow = static_cast<uint8_t *>(p.out_ptr) +
+                          (static_cast<size_t>(row_head) * p.L_q + i) * D * 2;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            if (n_blocks > 0) {
+              tmem_ld_x32(tO + c, o);
+              tmem_wait_ld();
+              reg_dep(o);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) o[u] = 0u;
+            }
+            if (r_loc < trows) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<uint4 *>(orow + (c + 8 * u) * 2) = make_uint4(
+                    pack2<1>(__uint_as_float(o[8 * u]) * sc, __uint_as_float(o[8 * u + 1]) * sc),
+                    pack2<1>(__uint_as_float(o[8 * u + 2]) * sc, __uint_as_float(o[8 * u + 3]) * sc),
+                    pack2<1>(__uint_as_float(o[8 * u + 4]) * sc, __uint_as_float(o[8 * u + 5]) * sc),
+                    pack2<1>(__uint_as_float(o[8 * u + 6]) * sc, __uint_as_float(o[8 * u + 7]) * sc));
+            }
+          }
+        }
+      } else {
       if (ok) {
         if constexpr (D >= 32) {
 #pragma unroll
@@ -924,6 +989,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         bulk_commit_group();
         bulk_wait_group_all();
       }
+      }   // 16-bit output through TMA
       if (ok && p.smax != nullptr && r_loc < trows) {
         // statistics against the exact max: sum_j 2^(t_j - m_true) = l 2^(m_use - m_true)
         const size_t row = static_cast<size_t>(row_head) * p.L_q + i;

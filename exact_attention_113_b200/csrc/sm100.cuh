@@ -261,6 +261,44 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// The same two products with 8-bit operands (kind::f8f6f4; both E4M3 here).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::f16 or kind::f8f6f4 by a compile-time flag.
+template <bool kF8>
+__device__ __forceinline__ void mma_ss_t(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  if constexpr (kF8)
+    mma_ss_f8(d_tmem, adesc, bdesc, idesc, accumulate);
+  else
+    mma_ss(d_tmem, adesc, bdesc, idesc, accumulate);
+}
+template <bool kF8>
+__device__ __forceinline__ void mma_ts_t(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  if constexpr (kF8)
+    mma_ts_f8(d_tmem, a_tmem, bdesc, idesc, accumulate);
+  else
+    mma_ts(d_tmem, a_tmem, bdesc, idesc, accumulate);
+}
+
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor" format):
 // start address, leading / stride byte offsets (16-byte units), version 1,
 // base offset 0, swizzle layout code (2 = 128B, 4 = 64B, 6 = 32B).
@@ -287,6 +325,14 @@ __device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) 
 }
 __device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi) {
   return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Instruction descriptor for kind::f8f6f4, E4M3 x E4M3 -> fp32: the format
+// fields hold 0 (E4M3), so the word has the layout of make_idesc_f16 with
+// ab_type 0.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16 with fp32 accumulation.
@@ -473,6 +519,14 @@ template <>
 __device__ __forceinline__ uint32_t pack2<1>(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Two floats -> two E4M3 codes (round to nearest even, saturating to +-448),
+// `lo` in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 }  // namespace fa

@@ -59,6 +59,20 @@ def make_qkv(w: Workload, device="cpu"):
     return tuple(out)
 
 
+def make_qkv_fp8(w: Workload, device="cpu"):
+    """Q, K, V of workload ``w`` as fp8 E4M3 tensors: the same seeded normals
+    as make_qkv, converted to float8_e4m3fn (round to nearest)."""
+    g = torch.Generator(device="cpu").manual_seed(int(w.seed))
+    out = []
+    for shape in ((w.B, w.H, w.L_q, w.D), (w.B, w.H_kv, w.L_k, w.D),
+                  (w.B, w.H_kv, w.L_k, w.D)):
+        x = torch.randn(shape, generator=g, dtype=torch.float32)
+        if w.std != 1.0:
+            x.mul_(w.std)
+        out.append(x.to(torch.float8_e4m3fn).to(device))
+    return tuple(out)
+
+
 def make_dout(w: Workload, device="cpu"):
     """The upstream gradient dO [B,H,L_q,D] for a backward of workload ``w``
     (seeded N(0, 1), its own stream: seed + 7919)."""
@@ -68,8 +82,12 @@ def make_dout(w: Workload, device="cpu"):
 
 
 def to_bits(t: torch.Tensor) -> np.ndarray:
-    """A CPU copy of an fp16/bf16 tensor as uint16 bit patterns."""
-    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    """A CPU copy of an fp16/bf16 tensor as uint16 bit patterns (fp8
+    tensors: uint8 codes)."""
+    t = t.detach().cpu().contiguous()
+    if t.element_size() == 1:
+        return t.view(torch.uint8).numpy()
+    return t.view(torch.int16).numpy().view(np.uint16)
 
 
 def sample_rows(w: Workload, per_head_random: int = 8, seed: int = 7) -> np.ndarray:

@@ -129,6 +129,30 @@ int fa_fwd_ex(const void *q, const void *k, const void *v, void *out, float *lse
               int window_left, int window_right, int dtype, cudaStream_t stream);
 
 /*
+ * fa_fwd_fp8 -- exact attention forward on fp8 (E4M3) inputs.  The pages
+ * list fp8 among FlashAttention-2's input types ("PyTorch Transformer Flash
+ * Attention机制" §5) without details; this entry reads them as: q, k, v hold
+ * E4M3 codes (OCP "fn" encoding: bias 7, no infinities, largest 448) whose
+ * real values are code * descale_{q,k,v}; the scores are
+ * scale * descale_q * descale_k * (q_i . k_j) accumulated in fp32; P enters
+ * the P.V product rounded to E4M3 (the tensor cores' fp8 kind takes both
+ * operands in 8 bits) while the normaliser sums the unrounded fp32 weights;
+ * O = descale_v * P.V / l is written as bf16.
+ *
+ *   q         device, [B, H,    L_q, D] E4M3 codes (1 byte each)
+ *   k, v      device, [B, H_kv, L_k, D] E4M3 codes
+ *   out       device, [B, H,    L_q, D] bfloat16 (written)
+ *   lse       device, [B, H, L_q] fp32 or NULL (natural log, as fa_fwd)
+ *   descale_q, descale_k, descale_v  finite, >= 0 (1 = codes are the values)
+ *   D in {32, 64, 128} (rows of at least 32 bytes), else FA_ERR_HEADDIM.
+ * Masks, windows, GQA, edge cases and errors as fa_fwd.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+               int H, int H_kv, int L_q, int L_k, int D, float scale, float descale_q,
+               float descale_k, float descale_v, int causal, int window_left,
+               int window_right, cudaStream_t stream);
+
+/*
  * fa_splitkv_workspace_bytes -- bytes of device workspace fa_fwd_splitkv
  * needs for these sizes (0 if the sizes are invalid): B*H*L_q*n_splits rows
  * of a D-wide fp32 partial output plus an (m, l) pair each.

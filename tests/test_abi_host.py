@@ -217,3 +217,27 @@ def _call_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, smax=0, ssum=0, **kw):
 ])
 def test_ex_argument_errors(lib, kw, code):
     assert _call_ex(**kw) == code
+
+
+# ------------------------------------------------------------ fp8 entry
+def _call_fp8(dq=1.0, dk=1.0, dv=1.0, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_fp8(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"], a["H_kv"],
+                         a["L_q"], a["L_k"], a["D"], a["scale"], dq, dk, dv, a["causal"],
+                         a["wl"], a["wr"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=16), -3), (dict(D=48), -3), (dict(q=0), -1), (dict(q=8), -5),
+    (dict(dq=-1.0), -6), (dict(dv=float("inf")), -6), (dict(scale=-1.0), -6),
+    (dict(dq=1e30, dk=1e30), -6),
+])
+def test_fp8_argument_errors(lib, kw, code):
+    assert _call_fp8(**kw) == code
+
+
+def test_16bit_entries_refuse_the_fp8_code(lib):
+    # dtype 2 is internal to fa_fwd_fp8
+    assert _call(dtype=2) == -4
+    assert _call_split(dtype=2) == -4
