@@ -95,6 +95,16 @@ bool encode_map_f32(CUtensorMap *map, const void *base, int n_heads, int L, int 
   return r == CUDA_SUCCESS;
 }
 
+// Head dims of the 16-bit forward: every multiple of 16 up to 128 (rows of
+// 32..256 bytes, swizzled in 128-, 64- or 32-byte atoms).
+bool valid_fwd_d(int D) { return D >= 16 && D <= 128 && D % 16 == 0; }
+
+// The swizzle span (bytes) of a row of D elements of `es` bytes.
+int sw_span(int D, int es) {
+  const int rb = D * es;
+  return rb % 128 == 0 ? 128 : (rb % 64 == 0 ? 64 : 32);
+}
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 __global__ void fill_kernel(float *p, size_t n, float value) {
@@ -235,9 +245,9 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
   if (static_cast<int64_t>(B) * H * ((static_cast<int64_t>(L_q) + 127) / 128) >
       (1ll << 31) - 1)
     return FA_ERR_SHAPE;                   // at most one CTA per (head, 128 query rows)
-  if (D != 16 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (!valid_fwd_d(D)) return FA_ERR_HEADDIM;
   if (dtype != FA_F16 && dtype != FA_BF16 && dtype != kE4M3) return FA_ERR_DTYPE;
-  if (dtype == kE4M3 && D < 32) return FA_ERR_HEADDIM;   // rows of >= 32 bytes
+  if (dtype == kE4M3 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return FA_ERR_ALIGN;
   if (lse && !aligned(lse, 4)) return FA_ERR_ALIGN;
@@ -352,13 +362,13 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
                                            ws_ml_offset(rows_total, D, n_splits));
   }
   const int esz = dtype == kE4M3 ? 1 : 2;
-  const int box_cols = D * esz >= 128 ? 128 / esz : D;
+  const int box_cols = sw_span(D, esz) / esz;
   const int q_box_heads = prm.packed ? prm.group : 1;
   if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols, prm.tile_q, q_box_heads) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_o, out, dtype == kE4M3 ? FA_BF16 : dtype, B * H, L_q, D,
-                  D * 2 >= 128 ? 64 : D, prm.tile_q, q_box_heads))
+                  sw_span(D, 2) / 2, prm.tile_q, q_box_heads))
     return FA_ERR_CUDA;
 
   int st = FA_ERR_HEADDIM;
@@ -371,6 +381,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 129: st = launch<64, 1, false>(prm, B, H, stream); break;
     case 256: st = launch<128, 0, false>(prm, B, H, stream); break;
     case 257: st = launch<128, 1, false>(prm, B, H, stream); break;
+    case 96: st = launch<48, 0, false>(prm, B, H, stream); break;
+    case 97: st = launch<48, 1, false>(prm, B, H, stream); break;
+    case 160: st = launch<80, 0, false>(prm, B, H, stream); break;
+    case 161: st = launch<80, 1, false>(prm, B, H, stream); break;
+    case 192: st = launch<96, 0, false>(prm, B, H, stream); break;
+    case 193: st = launch<96, 1, false>(prm, B, H, stream); break;
+    case 224: st = launch<112, 0, false>(prm, B, H, stream); break;
+    case 225: st = launch<112, 1, false>(prm, B, H, stream); break;
     case 1032: st = launch<16, 0, true>(prm, B, H, stream); break;
     case 1033: st = launch<16, 1, true>(prm, B, H, stream); break;
     case 1064: st = launch<32, 0, true>(prm, B, H, stream); break;
@@ -379,6 +397,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 1129: st = launch<64, 1, true>(prm, B, H, stream); break;
     case 1256: st = launch<128, 0, true>(prm, B, H, stream); break;
     case 1257: st = launch<128, 1, true>(prm, B, H, stream); break;
+    case 1096: st = launch<48, 0, true>(prm, B, H, stream); break;
+    case 1097: st = launch<48, 1, true>(prm, B, H, stream); break;
+    case 1160: st = launch<80, 0, true>(prm, B, H, stream); break;
+    case 1161: st = launch<80, 1, true>(prm, B, H, stream); break;
+    case 1192: st = launch<96, 0, true>(prm, B, H, stream); break;
+    case 1193: st = launch<96, 1, true>(prm, B, H, stream); break;
+    case 1224: st = launch<112, 0, true>(prm, B, H, stream); break;
+    case 1225: st = launch<112, 1, true>(prm, B, H, stream); break;
     case 66: st = launch<32, kE4M3, false>(prm, B, H, stream); break;
     case 130: st = launch<64, kE4M3, false>(prm, B, H, stream); break;
     case 258: st = launch<128, kE4M3, false>(prm, B, H, stream); break;
@@ -393,6 +419,14 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 129: return launch_combine<64, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
     case 256: return launch_combine<128, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
     case 257: return launch_combine<128, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 96: return launch_combine<48, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 97: return launch_combine<48, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 160: return launch_combine<80, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 161: return launch_combine<80, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 192: return launch_combine<96, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 193: return launch_combine<96, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 224: return launch_combine<112, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 225: return launch_combine<112, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
   }
   return FA_ERR_HEADDIM;
 }
@@ -444,7 +478,7 @@ extern "C" int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out
 
 extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {
   if (B < 1 || H < 1 || L_q < 0 || n_splits < 1 || n_splits > kMaxSplits) return 0;
-  if (D != 16 && D != 32 && D != 64 && D != 128) return 0;
+  if (!valid_fwd_d(D)) return 0;
   return ws_total_bytes(static_cast<int64_t>(B) * H * L_q, D, n_splits);
 }
 
@@ -650,7 +684,7 @@ extern "C" int fa_fwd_splitkv_static(const void *q, const void *k, const void *v
   // the size limit first, so that an oversized problem never reaches the GPU
   // (sizes fwd_impl would reject fall through to its own error codes)
   if (B >= 1 && H >= 1 && L_q >= 0 && L_q <= fa::kMaxSeq &&
-      (D == 16 || D == 32 || D == 64 || D == 128) &&
+      fa::valid_fwd_d(D) &&
       fa::ws_total_bytes(static_cast<int64_t>(B) * H * L_q, D, n_splits) >
           FA_STATIC_SCRATCH_BYTES)
     return FA_ERR_SCRATCH;
@@ -680,7 +714,7 @@ extern "C" const char *fa_status_string(int status) {
     case FA_OK: return "FA_OK";
     case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
     case FA_ERR_SHAPE: return "FA_ERR_SHAPE: bad sizes (B,H,H_kv>=1, L>=0, H%H_kv==0)";
-    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: D must be 16, 32, 64 or 128";
+    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: unsupported head dim D (see fa.h)";
     case FA_ERR_DTYPE: return "FA_ERR_DTYPE: dtype must be FA_F16 or FA_BF16";
     case FA_ERR_ALIGN: return "FA_ERR_ALIGN: q/k/v/out need 16-byte, lse 4-byte alignment";
     case FA_ERR_ARG: return "FA_ERR_ARG: scale must be finite and >= 0";

@@ -118,14 +118,23 @@ struct FwdParams {
 template <int D, int ES = 2>
 struct Geo {
   static constexpr int kRowBytes = D * ES;
-  static constexpr int kSwBytes = kRowBytes >= 128 ? 128 : kRowBytes;  // swizzle span
+  // swizzle span: the largest of 128 / 64 / 32 bytes dividing the row
+  static constexpr int kSwBytes = kRowBytes % 128 == 0 ? 128 : (kRowBytes % 64 == 0 ? 64 : 32);
   static constexpr int kBoxCols = kSwBytes / ES;                      // elements per box row
   static constexpr int kNumBox = kRowBytes / kSwBytes;                 // column boxes per tile
   static constexpr int kBoxBytes = kBM * kSwBytes;
   static constexpr int kTileBytes = kBM * kRowBytes;
   static_assert(kSwBytes >= 32, "rows of at least 32 bytes (a swizzle span)");
-  static constexpr int kSlotsK = kTileBytes >= 32768 ? 3 : (kTileBytes >= 16384 ? 4 : 8);
-  static constexpr int kSlotsV = kTileBytes >= 32768 ? 2 : (kTileBytes >= 16384 ? 4 : 8);
+  static_assert(kRowBytes % kSwBytes == 0, "whole swizzle atoms per row");
+  // ring depth: the tuned values for D = 16..128 powers of two; otherwise as
+  // many slots (up to 8) as the 224 KB shared-memory budget leaves beside Q
+  static constexpr bool kPow2 = (D & (D - 1)) == 0;
+  static constexpr int kFitSlots = (224 * 1024) / kTileBytes - 2 < 8
+                                       ? (224 * 1024) / kTileBytes - 2 : 8;
+  static constexpr int kSlotsK = kPow2 ? (kTileBytes >= 32768 ? 3 : (kTileBytes >= 16384 ? 4 : 8))
+                                       : (kFitSlots + 1) / 2;
+  static constexpr int kSlotsV = kPow2 ? (kTileBytes >= 32768 ? 2 : (kTileBytes >= 16384 ? 4 : 8))
+                                       : kFitSlots / 2;
   static constexpr int kSlots = kSlotsK + kSlotsV;
   static constexpr uint32_t kLayout = kSwBytes == 128 ? 2u : (kSwBytes == 64 ? 4u : 6u);
   static constexpr int kUnitsPerBoxRow = kSwBytes / 16;
@@ -252,6 +261,35 @@ __device__ __forceinline__ void apply_mask(float (&sv)[kBNc], const FwdParams &p
         sv[c] = fmaf(sv[c], sl2, c < n_cols ? m[c] * kLog2e : 0.0f);
     }
   }
+}
+
+// Visit the D TMEM columns of an O row in chunks of 32 (a 16-wide tail when
+// D is an odd multiple of 16): f(first column, width as an integral
+// constant).
+template <int D, typename F>
+__device__ __forceinline__ void for_o_chunks(F &&f) {
+#pragma unroll
+  for (int c = 0; c < D; c += 32) {
+    if (c + 32 <= D)
+      f(c, std::integral_constant<int, 32>{});
+    else
+      f(c, std::integral_constant<int, 16>{});
+  }
+}
+
+// O row *= alpha in TMEM.
+template <int D>
+__device__ __forceinline__ void scale_o_row(uint32_t tO, float alpha) {
+  for_o_chunks<D>([&](int c, auto w) {
+    constexpr int W = decltype(w)::value;
+    uint32_t o[W];
+    tmem_ld_cols<W>(tO + c, o);
+    tmem_wait_ld();
+    reg_dep(o);
+#pragma unroll
+    for (int u = 0; u < W; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+    tmem_st_cols<W>(tO + c, o);
+  });
 }
 
 // P of one half-row (64 keys) into 32-bit TMEM words: two 16-bit values a
@@ -718,28 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           if (warp_rescale && n > 0) {
             // O_t was completed up to block j-1 (PV_t(j-1) finished before
             // S_t(j) was issued); scale it by alpha row by row.
-            if constexpr (D >= 32) {
-#pragma unroll
-              for (int c = 0; c < D; c += 32) {
-                uint32_t o[32];
-                tmem_ld_x32(tO + c, o);
-                tmem_wait_ld();
-                reg_dep(o);
-#pragma unroll
-                for (int u = 0; u < 32; ++u)
-                  o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-                tmem_st_x32(tO + c, o);
-              }
-            } else {
-              uint32_t o[16];
-              tmem_ld_x16(tO, o);
-              tmem_wait_ld();
-              reg_dep(o);
-#pragma unroll
-              for (int u = 0; u < 16; ++u)
-                o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-              tmem_st_x16(tO, o);
-            }
+            scale_o_row<D>(tO, alpha);
           }
         };
 
@@ -794,20 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           if (ok) {
             store_p_half<DT>(tPs, 0, pk[0]);
             store_p_half<DT>(tPs, 1, pk[1]);
-            if (warp_rescale && n > 0) {
-              constexpr int kChunk = D >= 32 ? 32 : D;
-#pragma unroll
-              for (int c = 0; c < D; c += kChunk) {
-                uint32_t o[kChunk];
-                tmem_ld_cols<kChunk>(tO + c, o);
-                tmem_wait_ld();
-                reg_dep(o);
-#pragma unroll
-                for (int u = 0; u < kChunk; ++u)
-                  o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-                tmem_st_cols<kChunk>(tO + c, o);
-              }
-            }
+            if (warp_rescale && n > 0) scale_o_row<D>(tO, alpha);
           }
         } else {
         // Speculative pass (unmasked blocks, once every row has a reference
@@ -872,27 +876,26 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           const size_t row = static_cast<size_t>(split) * p.rows_total +
                              static_cast<size_t>(row_head) * p.L_q + i;
           float4 *dst = reinterpret_cast<float4 *>(p.ws_o + row * D);
-          constexpr int kChunk = D >= 32 ? 32 : D;
-#pragma unroll
-          for (int c = 0; c < D; c += kChunk) {
-            uint32_t o[kChunk];
+          for_o_chunks<D>([&](int c, auto w) {
+            constexpr int W = decltype(w)::value;
+            uint32_t o[W];
             if (n_blocks > 0) {
-              tmem_ld_cols<kChunk>(tO + c, o);
+              tmem_ld_cols<W>(tO + c, o);
               tmem_wait_ld();
               reg_dep(o);
             } else {
 #pragma unroll
-              for (int u = 0; u < kChunk; ++u) o[u] = 0u;
+              for (int u = 0; u < W; ++u) o[u] = 0u;
             }
             if (mine) {
 #pragma unroll
-              for (int u = 0; u < kChunk / 4; ++u)
+              for (int u = 0; u < W / 4; ++u)
                 dst[c / 4 + u] = make_float4(__uint_as_float(o[4 * u]),
                                              __uint_as_float(o[4 * u + 1]),
                                              __uint_as_float(o[4 * u + 2]),
                                              __uint_as_float(o[4 * u + 3]));
             }
-          }
+          });
           if (mine) p.ws_ml[row] = make_float2(l > 0.0f ? m_use : -INFINITY, l);
         }
       } else {
@@ -943,42 +946,24 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
       } else {
       if (ok) {
-        if constexpr (D >= 32) {
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            if (n_blocks > 0) {
-              tmem_ld_x32(tO + c, o);
-              tmem_wait_ld();
-              reg_dep(o);
-            } else {
-#pragma unroll
-              for (int u = 0; u < 32; ++u) o[u] = 0u;
-            }
-            uint32_t w[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-              w[u] = pack2<DT>(__uint_as_float(o[2 * u]) * inv_l,
-                               __uint_as_float(o[2 * u + 1]) * inv_l);
-            put_units(c, w, 4);
-          }
-        } else {
-          uint32_t o[16];
+        for_o_chunks<D>([&](int c, auto wd) {
+          constexpr int W = decltype(wd)::value;
+          uint32_t o[W];
           if (n_blocks > 0) {
-            tmem_ld_x16(tO, o);
+            tmem_ld_cols<W>(tO + c, o);
             tmem_wait_ld();
             reg_dep(o);
           } else {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) o[u] = 0u;
+            for (int u = 0; u < W; ++u) o[u] = 0u;
           }
-          uint32_t w[8];
+          uint32_t w[W / 2];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            w[u] = pack2<DT>(__uint_as_float(o[2 * u]) * inv_l,
-                             __uint_as_float(o[2 * u + 1]) * inv_l);
-          put_units(0, w, 2);
-        }
+          for (int u = 0; u < W / 2; ++u)
+            w[u] = pack2<kF8 ? 1 : DT>(__uint_as_float(o[2 * u]) * inv_l,
+                                       __uint_as_float(o[2 * u + 1]) * inv_l);
+          put_units(c, w, W / 8);
+        });
       }
       fence_proxy_async_smem();
       named_barrier_sync(1 + t, kBM);

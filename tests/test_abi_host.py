@@ -65,7 +65,7 @@ def _call(**kw):
     (dict(B=0), -2), (dict(H=0), -2), (dict(H_kv=0), -2), (dict(H=4, H_kv=3), -2),
     (dict(L_q=-1), -2), (dict(L_k=-5), -2), (dict(L_q=(1 << 30) + 1), -2),
     (dict(B=1 << 16, H=1 << 15, L_q=1 << 10), -2),
-    (dict(D=0), -3), (dict(D=48), -3), (dict(D=96), -3), (dict(D=256), -3),
+    (dict(D=0), -3), (dict(D=40), -3), (dict(D=8), -3), (dict(D=144), -3), (dict(D=256), -3),
     (dict(dtype=2), -4), (dict(dtype=-1), -4),
     (dict(q=24), -5), (dict(out=8), -5), (dict(v=4), -5), (dict(lse=2), -5),
     (dict(scale=-0.5), -6), (dict(scale=float("nan")), -6), (dict(scale=float("inf")), -6),
@@ -112,7 +112,8 @@ def test_splitkv_workspace_bytes(lib):
     rows, D, S = 2 * 4 * 8, 64, 3
     o = S * rows * D * 4
     assert fa.fa_splitkv_workspace_bytes(2, 4, 8, D, S) == ((o + 255) // 256) * 256 + S * rows * 8
-    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 48, S) == 0
+    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 40, S) == 0
+    assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 48, S) > 0          # any multiple of 16
     assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 64, 0) == 0
     assert fa.fa_splitkv_workspace_bytes(2, 4, 8, 64, 65) == 0
 
@@ -120,7 +121,7 @@ def test_splitkv_workspace_bytes(lib):
 @pytest.mark.parametrize("kw,code", [
     (dict(n_splits=0), -6), (dict(n_splits=65), -6), (dict(n_splits=-1), -6),
     (dict(ws=0), -1), (dict(ws=128), -5), (dict(ws_bytes=100), -9),
-    (dict(q=0), -1), (dict(D=48), -3), (dict(scale=-1.0), -6),
+    (dict(q=0), -1), (dict(D=40), -3), (dict(scale=-1.0), -6),
 ])
 def test_splitkv_argument_errors(lib, kw, code):
     assert _call_split(**kw) == code
@@ -213,7 +214,7 @@ def _call_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, smax=0, ssum=0, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(mtype=4), -6), (dict(mtype=-1), -6), (dict(sq=-1), -6), (dict(sb=-8), -6),
     (dict(mask=0), -1), (dict(smax=16, ssum=0), -1), (dict(smax=0, ssum=16), -1),
-    (dict(smax=18, ssum=16), -5), (dict(q=0), -1), (dict(D=48), -3),
+    (dict(smax=18, ssum=16), -5), (dict(q=0), -1), (dict(D=40), -3),
 ])
 def test_ex_argument_errors(lib, kw, code):
     assert _call_ex(**kw) == code

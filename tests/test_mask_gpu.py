@@ -126,3 +126,9 @@ def test_mask_matches_equivalent_causal():
     torch.cuda.synchronize()
     assert (o1.float() - o2.float()).abs().max().item() <= 2e-3
     assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+@pytest.mark.parametrize("D", [48, 112])
+def test_non_pow2_head_dim_with_mask(D):
+    w = _w(D=D, seed=7950 + D)
+    check_masked(w, _mask((1, w.H, w.L_q, w.L_k), "f32", 7960 + D))

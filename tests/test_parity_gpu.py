@@ -173,3 +173,27 @@ def test_gqa_packed_matches_repeated_heads():
     o2, l2 = run_gpu(q, k.repeat_interleave(4, dim=1), v.repeat_interleave(4, dim=1), wm)
     assert (o1.float() - o2.float()).abs().max().item() <= 2 * 3e-3 + 4e-3   # two gates
     assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+# ------------------------------------------------------------ non-power-of-two head dims
+# Rows of 96, 160, 192 and 224 bytes: 32-, 32-, 64- and 32-byte swizzle
+# atoms (3, 5, 3, 7 per row); O chunks with a 16-column tail.
+@pytest.mark.parametrize("D", [48, 80, 96, 112])
+@pytest.mark.parametrize("L", [1, 129, 300])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", [F16, BF16])
+def test_non_pow2_head_dims(D, L, causal, dtype):
+    check_full(_w(H=3, H_kv=3, L_q=L, L_k=L, D=D, causal=causal, dtype=dtype,
+                  seed=5300 + D + L), derived=True)
+
+
+@pytest.mark.parametrize("D", [48, 96])
+def test_non_pow2_gqa_packed_and_long(D):
+    check_full(_w(B=2, H=8, H_kv=2, L_q=20, L_k=1500, D=D, seed=5400 + D))
+    check_full(_w(B=1, H=2, H_kv=2, L_q=2000, L_k=2000, D=D, causal=True, seed=5410 + D),
+               derived=True)
+
+
+@pytest.mark.parametrize("D", [80, 112])
+def test_non_pow2_split_kv(D):
+    check_full(_w(B=1, H=4, H_kv=4, L_q=3, L_k=3000, D=D, seed=5500 + D), n_splits=5)
