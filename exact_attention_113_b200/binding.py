@@ -25,7 +25,7 @@ STATUS = {
 }
 FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
 EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
-           "fa_fwd_splitkv",
+           "fa_fwd_host", "fa_fwd_host_workspace_bytes", "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_splitkv_workspace_bytes",
            "fa_status_string", "fa_version")
 # size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
@@ -66,6 +66,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f = ctypes.c_float
         lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, i, i, vp]
         lib.fa_fwd_fp8.restype = i
+        lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, i, vp,
+                                    ctypes.c_size_t, i, vp]
+        lib.fa_fwd_host.restype = i
+        lib.fa_fwd_host_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        lib.fa_fwd_host_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float,
                                        i, i, i, i, i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_splitkv.restype = i
@@ -114,6 +119,18 @@ def fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, des
     return load().fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, float(scale),
                              float(descale_q), float(descale_k), float(descale_v), int(causal),
                              int(window_left), int(window_right), stream)
+
+
+def fa_fwd_host(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                window_right, dtype, workspace, workspace_bytes, n_chunks, stream) -> int:
+    """The host-buffer (pipelined) C entry point, unchanged."""
+    return load().fa_fwd_host(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, float(scale),
+                              int(causal), int(window_left), int(window_right), int(dtype),
+                              workspace, int(workspace_bytes), int(n_chunks), stream)
+
+
+def fa_fwd_host_workspace_bytes(B, H, H_kv, L_q, L_k, D, n_chunks) -> int:
+    return int(load().fa_fwd_host_workspace_bytes(B, H, H_kv, L_q, L_k, D, n_chunks))
 
 
 def mask_layout(mask, B, H, L_q, L_k):
@@ -392,4 +409,45 @@ def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1
                         window_right, stream.cuda_stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd_fp8")
+    return out, lse
+
+
+def flash_fwd_host(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
+                   out=None, lse=None, n_chunks=8, workspace=None, device=None, stream=None):
+    """Exact attention forward on host (CPU, preferably pinned) tensors
+    through fa_fwd_host: chunked copies in, kernels, copies out, overlapped.
+    Returns (out, lse) as host tensors, valid once ``stream`` (default: the
+    device's current stream) is synchronised.  The device workspace is
+    allocated here with torch unless given."""
+    import torch
+
+    B, H, L_q, D = q.shape
+    _, H_kv, L_k, _ = k.shape
+    if q.is_cuda or k.is_cuda or v.is_cuda:
+        raise ValueError("flash_fwd_host takes host tensors")
+    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share dtype float16 or bfloat16")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    dtype = FA_F16 if q.dtype == torch.float16 else FA_BF16
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    pin = q.is_pinned()
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=pin)
+    if lse is None:
+        lse = torch.empty((B, H, L_q), dtype=torch.float32, pin_memory=pin)
+    if workspace is None:
+        nbytes = fa_fwd_host_workspace_bytes(B, H, H_kv, L_q, L_k, D, n_chunks)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        st = fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr(), B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                         window_right, dtype, workspace.data_ptr(), workspace.numel(), n_chunks,
+                         stream.cuda_stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_host")
     return out, lse

@@ -493,6 +493,144 @@ extern "C" int fa_fwd_splitkv(const void *q, const void *k, const void *v, void 
 }
 
 // ---------------------------------------------------------------------------
+// Forward on host buffers, pipelined: the K/V-head groups are cut into
+// n_chunks contiguous ranges (whole GQA groups: a range of K/V heads is a
+// contiguous range of query heads); chunk c's inputs are copied in on one
+// stream, computed on the caller's stream and copied out on a third, into
+// and out of two device slots taken from the caller's workspace, so that
+// the copies of neighbouring chunks overlap the kernel.
+namespace fa {
+namespace {
+struct HostPlan {
+  int64_t groups, per;              // K/V-head groups, groups per chunk
+  size_t q_b, kv_b, o_b, lse_b;     // bytes of one slot's buffers
+  size_t slot_b;
+};
+HostPlan host_plan(int B, int H, int H_kv, int L_q, int L_k, int D, int n_chunks) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  HostPlan hp;
+  hp.groups = static_cast<int64_t>(B) * H_kv;
+  hp.per = (hp.groups + n_chunks - 1) / n_chunks;
+  const int64_t g = H / H_kv;
+  hp.q_b = up(static_cast<size_t>(hp.per * g) * L_q * D * 2);
+  hp.kv_b = up(static_cast<size_t>(hp.per) * L_k * D * 2);
+  hp.o_b = hp.q_b;
+  hp.lse_b = up(static_cast<size_t>(hp.per * g) * L_q * sizeof(float));
+  hp.slot_b = hp.q_b + 2 * hp.kv_b + hp.o_b + hp.lse_b;
+  return hp;
+}
+
+// Per device: the copy streams and the events that order the pipeline.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t in_ready[2], comp_done[2], out_done[2];
+  bool ready = false;
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+
+int host_pipe(HostPipe **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe &hp = g_pipe[dev];
+  if (!hp.ready) {
+    if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess)
+      return FA_ERR_CUDA;
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&hp.in_ready[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&hp.comp_done[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&hp.out_done[i], cudaEventDisableTiming) != cudaSuccess)
+        return FA_ERR_CUDA;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return FA_OK;
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" size_t fa_fwd_host_workspace_bytes(int B, int H, int H_kv, int L_q, int L_k, int D,
+                                              int n_chunks) {
+  if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || L_q < 0 || L_k < 0 ||
+      L_q > fa::kMaxSeq || L_k > fa::kMaxSeq || n_chunks < 1 || !fa::valid_fwd_d(D))
+    return 0;
+  return 2 * fa::host_plan(B, H, H_kv, L_q, L_k, D, n_chunks).slot_b;
+}
+
+extern "C" int fa_fwd_host(const void *q, const void *k, const void *v, void *out, float *lse,
+                           int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                           int causal, int window_left, int window_right, int dtype,
+                           void *workspace, size_t workspace_bytes, int n_chunks,
+                           cudaStream_t stream) {
+  using namespace fa;
+  if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || H % H_kv != 0) return FA_ERR_SHAPE;
+  if (L_q > kMaxSeq || L_k > kMaxSeq) return FA_ERR_SHAPE;
+  if (!valid_fwd_d(D)) return FA_ERR_HEADDIM;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (n_chunks < 1) return FA_ERR_ARG;
+  if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+  if (L_q == 0) return FA_OK;
+  if (!q || !out || (L_k > 0 && (!k || !v)) || !workspace) return FA_ERR_NULL;
+  if (!aligned(workspace, 256)) return FA_ERR_ALIGN;
+  const HostPlan hp = host_plan(B, H, H_kv, L_q, L_k, D, n_chunks);
+  if (workspace_bytes < 2 * hp.slot_b) return FA_ERR_WORKSPACE;
+  HostPipe *pp = nullptr;
+  int st = host_pipe(&pp);
+  if (st != FA_OK) return st;
+  const int64_t g = H / H_kv;
+  const size_t qrow = static_cast<size_t>(L_q) * D * 2, kvrow = static_cast<size_t>(L_k) * D * 2;
+  const size_t lrow = static_cast<size_t>(L_q) * sizeof(float);
+  // the first chunk's copies wait for work the caller queued before this call
+  if (cudaEventRecord(pp->comp_done[0], stream) != cudaSuccess ||
+      cudaStreamWaitEvent(pp->h2d, pp->comp_done[0], 0) != cudaSuccess)
+    return FA_ERR_CUDA;
+  int n_used = 0;
+  for (int64_t g0 = 0; g0 < hp.groups; g0 += hp.per, ++n_used) {
+    const int slot = n_used & 1;
+    const int64_t ng = std::min(hp.per, hp.groups - g0);   // K/V heads in this chunk
+    char *base = static_cast<char *>(workspace) + slot * hp.slot_b;
+    char *dq = base, *dk = dq + hp.q_b, *dv = dk + hp.kv_b, *dout = dv + hp.kv_b;
+    float *dlse = reinterpret_cast<float *>(dout + hp.o_b);
+    bool ok = true;
+    // inputs in (after the slot's previous chunk has been copied out)
+    if (n_used >= 2) ok = ok && cudaStreamWaitEvent(pp->h2d, pp->out_done[slot], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(dq, static_cast<const char *>(q) + g0 * g * qrow, ng * g * qrow,
+                               cudaMemcpyHostToDevice, pp->h2d) == cudaSuccess;
+    if (L_k > 0) {
+      ok = ok && cudaMemcpyAsync(dk, static_cast<const char *>(k) + g0 * kvrow, ng * kvrow,
+                                 cudaMemcpyHostToDevice, pp->h2d) == cudaSuccess;
+      ok = ok && cudaMemcpyAsync(dv, static_cast<const char *>(v) + g0 * kvrow, ng * kvrow,
+                                 cudaMemcpyHostToDevice, pp->h2d) == cudaSuccess;
+    }
+    ok = ok && cudaEventRecord(pp->in_ready[slot], pp->h2d) == cudaSuccess;
+    // compute on the caller's stream: the chunk is one batch of ng*g heads
+    ok = ok && cudaStreamWaitEvent(stream, pp->in_ready[slot], 0) == cudaSuccess;
+    if (!ok) return FA_ERR_CUDA;
+    st = fwd_impl(dq, dk, dv, dout, lse ? dlse : nullptr, 1, static_cast<int>(ng * g),
+                  static_cast<int>(ng), L_q, L_k, D, scale, causal, window_left, window_right,
+                  dtype, 0, nullptr, 0, nullptr, stream);
+    if (st != FA_OK) return st;
+    ok = cudaEventRecord(pp->comp_done[slot], stream) == cudaSuccess;
+    // results out
+    ok = ok && cudaStreamWaitEvent(pp->d2h, pp->comp_done[slot], 0) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(static_cast<char *>(out) + g0 * g * qrow, dout, ng * g * qrow,
+                               cudaMemcpyDeviceToHost, pp->d2h) == cudaSuccess;
+    if (lse)
+      ok = ok && cudaMemcpyAsync(reinterpret_cast<char *>(lse) + g0 * g * lrow, dlse,
+                                 ng * g * lrow, cudaMemcpyDeviceToHost, pp->d2h) == cudaSuccess;
+    ok = ok && cudaEventRecord(pp->out_done[slot], pp->d2h) == cudaSuccess;
+    if (!ok) return FA_ERR_CUDA;
+  }
+  // the caller's stream sees the whole call: wait for the last copies out
+  for (int i = 0; i < std::min(n_used, 2); ++i)
+    if (cudaStreamWaitEvent(stream, pp->out_done[(n_used - 1 - i) & 1], 0) != cudaSuccess)
+      return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Backward.  Workspace: dQ accumulator [B*H][L_q][D] fp32, then lse2 and
 // delta [B*H][L_q_pad] fp32 (L_q_pad = L_q rounded up to 128), each part at
 // a 256-byte boundary.

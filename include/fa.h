@@ -155,6 +155,37 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *ls
                int window_right, cudaStream_t stream);
 
 /*
+ * fa_fwd_host_workspace_bytes -- bytes of device workspace fa_fwd_host
+ * needs (0 if the sizes are invalid): two slots, each holding one chunk's
+ * q, k, v, out and lse.
+ */
+size_t fa_fwd_host_workspace_bytes(int B, int H, int H_kv, int L_q, int L_k, int D,
+                                   int n_chunks);
+
+/*
+ * fa_fwd_host -- fa_fwd on HOST buffers (pinned memory lets the copies run
+ * asynchronously and overlap; pageable memory works but serialises them).
+ * The B*H_kv key/value heads (with their query heads) are cut into
+ * n_chunks contiguous ranges; chunk c's q, k, v are copied in on a copy
+ * stream, its forward runs on `stream`, its out and lse are copied back on
+ * a second copy stream, each chunk through one of two device slots in
+ * `workspace`, so the copies in both directions overlap the kernels of
+ * neighbouring chunks.  Arguments as fa_fwd except:
+ *   q, k, v, out, lse  HOST pointers, same layouts (lse may be NULL)
+ *   workspace          device, 256-byte aligned, at least
+ *                      fa_fwd_host_workspace_bytes(...) bytes
+ *   n_chunks           >= 1 (FA_ERR_ARG otherwise)
+ * Returns after enqueueing; `stream` is ordered after the last copy out, so
+ * synchronising it makes out and lse valid.  The copy streams and events
+ * are created by the first call on each device (make it before any stream
+ * capture); calls on one device must not overlap.
+ */
+int fa_fwd_host(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
+                int window_left, int window_right, int dtype, void *workspace,
+                size_t workspace_bytes, int n_chunks, cudaStream_t stream);
+
+/*
  * fa_splitkv_workspace_bytes -- bytes of device workspace fa_fwd_splitkv
  * needs for these sizes (0 if the sizes are invalid): B*H*L_q*n_splits rows
  * of a D-wide fp32 partial output plus an (m, l) pair each.

@@ -242,3 +242,34 @@ def test_16bit_entries_refuse_the_fp8_code(lib):
     # dtype 2 is internal to fa_fwd_fp8
     assert _call(dtype=2) == -4
     assert _call_split(dtype=2) == -4
+
+
+# ------------------------------------------------------------ host-buffer entry
+def _call_host(ws=256, ws_bytes=1 << 40, n_chunks=4, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_host(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"], a["H_kv"],
+                          a["L_q"], a["L_k"], a["D"], a["scale"], a["causal"], a["wl"], a["wr"],
+                          a["dtype"], ws, ws_bytes, n_chunks, None)
+
+
+def test_host_workspace_bytes(lib):
+    # two slots of one chunk: ceil(B*H_kv / n_chunks) K/V heads and their
+    # query heads; q, k, v, out in the element type, lse fp32, 256-aligned parts
+    up = lambda x: (x + 255) // 256 * 256
+    B, H, H_kv, L_q, L_k, D, n = 2, 8, 2, 100, 300, 64, 3
+    per = -(-(B * H_kv) // n)
+    slot = 2 * up(per * 4 * L_q * D * 2) + 2 * up(per * L_k * D * 2) + up(per * 4 * L_q * 4)
+    assert fa.fa_fwd_host_workspace_bytes(B, H, H_kv, L_q, L_k, D, n) == 2 * slot
+    assert fa.fa_fwd_host_workspace_bytes(B, H, H_kv, L_q, L_k, 40, n) == 0
+    assert fa.fa_fwd_host_workspace_bytes(B, H, 3, L_q, L_k, D, n) == 0
+    assert fa.fa_fwd_host_workspace_bytes(B, H, H_kv, L_q, L_k, D, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_chunks=0), -6), (dict(ws=0), -1), (dict(ws=128), -5), (dict(ws_bytes=100), -9),
+    (dict(D=40), -3), (dict(dtype=2), -4), (dict(q=0), -1), (dict(H=4, H_kv=3), -2),
+    (dict(scale=float("nan")), -6),
+])
+def test_host_argument_errors(lib, kw, code):
+    assert _call_host(**kw) == code
