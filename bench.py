@@ -62,8 +62,10 @@ UNIT = "TFLOPS"
 BWD_FLOP_FACTOR = 2.5      # backward: S, dP, dV, dK, dQ = 5 GEMMs vs the forward's 2
 DEFAULT_WORKLOAD = W.ROOFLINE.name
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fa_fwd_roofline_b4h48l8192d128_ncu.md")
+# the forward kernel's device code (the ncu summary is valid while it is
+# unchanged; the host-side launch code lives in fa_api.cu)
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_113_b200", "csrc", f)
-                  for f in ("fa_fwd_kernel.cuh", "sm100.cuh", "fa_api.cu")]
+                  for f in ("fa_fwd_kernel.cuh", "sm100.cuh")]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
