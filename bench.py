@@ -60,6 +60,10 @@ METRIC = "attention fwd TFLOPS (and % of B200 fp16 tensor peak) vs seq len"
 METRIC_BWD = "attention bwd TFLOPS (five GEMMs: 2.5x the forward's FLOPs)"
 UNIT = "TFLOPS"
 BWD_FLOP_FACTOR = 2.5      # backward: S, dP, dV, dK, dQ = 5 GEMMs vs the forward's 2
+# MUFU ex2 rate per SM and clock: 8 clk per warp instruction per sub-partition
+# (measured with a one-CTA microbenchmark on this GPU), 4 sub-partitions
+MUFU_EX2_PER_CLK_SM = 16.0
+SM_COUNT = 148
 DEFAULT_WORKLOAD = W.ROOFLINE.name
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fa_fwd_roofline_b4h48l8192d128_ncu.md")
 # the forward kernel's device code (the ncu summary is valid while it is
@@ -382,6 +386,9 @@ def run_ours(args, w: W.Workload):
     if n_splits:
         roofline["timed"] = (f"whole step: split-KV launch ({n_splits} key slices) "
                              "plus merge launch")
+    clocks = clk.summary()
+    exp_bound = exp_roof(w, avg_launch_s, clocks.get("sm_mhz") or clocks.get("sm_max_mhz"),
+                         bwd)
 
     # ---- end to end through host buffers (pinned), rank-local
     e2e = None
@@ -456,7 +463,8 @@ def run_ours(args, w: W.Workload):
         "data": "synthetic (seeded N(0,%g) inputs, per-rank seeds)" % w.std,
         "config": workload_config(w, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "clocks": clk.summary(), "gpu_launches": args.steps * launches_per_step,
+        "clocks": clocks, "gpu_launches": args.steps * launches_per_step,
+        "exp_bound": exp_bound,
         "pct_of_tensor_peak": round(100.0 * value / world / peak, 2),
         "launch_ms": {"min": round(min(launch_ms), 4), "median": round(statistics.median(launch_ms), 4),
                       "max": round(max(launch_ms), 4)},
@@ -469,6 +477,19 @@ def run_ours(args, w: W.Workload):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def exp_roof(w: W.Workload, launch_s: float, sm_mhz, bwd: bool = False) -> dict:
+    """The third roof: one exponential per visible (query, key) pair (the
+    backward recomputes them once more) against MUFU's ex2 rate at the
+    sampled SM clock."""
+    mhz = float(sm_mhz) if sm_mhz else 1965.0
+    exps = float(w.B * w.H * visible_pairs_per_head(w))
+    per_clk_sm = exps / (launch_s * mhz * 1e6 * SM_COUNT)
+    return {"exps_per_launch": exps, "achieved_per_clk_per_sm": round(per_clk_sm, 3),
+            "peak_per_clk_per_sm": MUFU_EX2_PER_CLK_SM,
+            "frac": round(per_clk_sm / MUFU_EX2_PER_CLK_SM, 4), "sm_mhz_used": mhz,
+            "note": "backward: P recomputed once" if bwd else "forward"}
 
 
 def resolve_splits(arg: str, w: W.Workload, sm_count: int = 148) -> int:

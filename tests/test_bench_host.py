@@ -104,3 +104,13 @@ def test_resolve_splits():
     assert bench.resolve_splits("0", w) == 0
     assert bench.resolve_splits("5", w) == 5
     assert 1 <= bench.resolve_splits("auto", w) <= 64
+
+
+def test_exp_roof_closed_form():
+    # B4 H48 L8192 non-causal: 4*48*8192^2 exponentials; at 1 GHz over 1 ms
+    w = W.ROOFLINE
+    r = bench.exp_roof(w, 1e-3, 1000.0)
+    exps = 4 * 48 * 8192 * 8192
+    assert r["exps_per_launch"] == exps
+    assert abs(r["achieved_per_clk_per_sm"] - round(exps / (1e-3 * 1e9 * 148), 3)) < 1e-9
+    assert abs(r["frac"] - round(exps / (1e-3 * 1e9 * 148) / 16.0, 4)) < 1e-9
