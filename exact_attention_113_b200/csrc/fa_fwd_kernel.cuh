@@ -143,7 +143,7 @@ struct Geo {
   // In unmasked blocks one column pair in kPolyPeriod takes 2^x from the FMA
   // pipe (exp2_poly2) instead of MUFU: the MUFU rate (16/clk/SM) alone needs
   // as many cycles per block as the D=128 tensor work.
-  static constexpr int kPolyPeriod = 1 << 20;  // (tuned below)
+  static constexpr int kPolyPeriod = 1 << 20;  // off; the kernel picks kPoly
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kTileBytes;
@@ -319,6 +319,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   constexpr int kES = kF8 ? 1 : 2;
   constexpr int kKStep = 32 / kES;             // K of one MMA instruction (32 bytes)
   using G = Geo<D, kES>;
+  // One column pair in kPoly takes 2^x from the FMA pipe (unmasked blocks).
+  // Measured: +4 % for fp8 at D = 128, where the tensor work per block halves
+  // and MUFU becomes the limit; 10-25 % slower at D <= 64, whose softmax
+  // threads are bound by their own instruction stream; neutral otherwise.
+  constexpr int kPoly = (kF8 && D == 128) ? 8 : G::kPolyPeriod;
   constexpr int kSlots = G::kSlots;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -734,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                     __ffma2_rn(make_float2(sv[half * 64 + c], sv[half * 64 + c + 1]), sl2v, negm);
                 const int pair = (half * 64 + c) >> 1;
                 float2 pp;
-                if (decltype(poly_ok)::value && (pair % G::kPolyPeriod) == G::kPolyPeriod - 1)
+                if (decltype(poly_ok)::value && (pair % kPoly) == kPoly - 1)
                   pp = exp2_poly2(x);
                 else
                   pp = make_float2(ex2(x.x), ex2(x.y));
@@ -794,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             const int pair = c >> 1;
             const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2v, negm);
             float2 pp;
-            if (full && (pair % G::kPolyPeriod) == G::kPolyPeriod - 1)
+            if (full && (pair % kPoly) == kPoly - 1)
               pp = exp2_poly2(x);
             else
               pp = make_float2(ex2(x.x), ex2(x.y));
@@ -833,7 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             mx[pair & 3] = fmax3(mx[pair & 3], s[c], s[c + 1]);
             const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2v, negm);
             float2 pp;
-            if ((pair % G::kPolyPeriod) == G::kPolyPeriod - 1)
+            if ((pair % kPoly) == kPoly - 1)
               pp = exp2_poly2(x);
             else
               pp = make_float2(ex2(x.x), ex2(x.y));
