@@ -124,6 +124,11 @@ class Oracle:
             dp, dp, dp, dp, i64, i64, i64, i64, i64, i64, ctypes.c_double, ctypes.c_int,
             i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
         lib.oracle_attention_bwd_f64.restype = ctypes.c_int
+        lib.oracle_attention_bwd_f64_ex.argtypes = [
+            dp, dp, dp, dp, i64, i64, i64, i64, i64, i64, ctypes.c_double, ctypes.c_int,
+            i64, i64, ctypes.c_void_p, ctypes.c_int, i64, i64, i64,
+            dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.oracle_attention_bwd_f64_ex.restype = ctypes.c_int
         self.lib = lib
         self._tables = {}
 
@@ -316,20 +321,24 @@ class Oracle:
         return out, lse
 
     def attention_bwd_f64(self, q, k, v, dout, scale, causal=False, window_left=-1,
-                          window_right=-1, delta_err=None, with_abs=False, n_threads=0):
+                          window_right=-1, delta_err=None, with_abs=False, n_threads=0,
+                          mask=None):
         """Gradients of sum(dout * O) on float64 arrays: returns (dq, dk, dv),
         or (dq, dk, dv, dq_abs, dk_abs, dv_abs) with ``with_abs`` (the error
-        scales documented in attention_ref.c; ``delta_err`` [B,H,L_q])."""
+        scales documented in attention_ref.c; ``delta_err`` [B,H,L_q]).
+        ``mask``: as attention_rows_ex."""
         q, k, v, dout = self._f64(q), self._f64(k), self._f64(v), self._f64(dout)
         B, H, L_q, D = q.shape
         _, H_kv, L_k, _ = k.shape
+        m, mtype, sb, sh, sq = self.mask_args(mask, B, H, L_q, L_k)
         dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
         absb = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)] if with_abs else None
         de = None if delta_err is None else self._f64(delta_err).reshape(B, H, L_q)
         c = ctypes.c_double
-        rc = self.lib.oracle_attention_bwd_f64(
+        rc = self.lib.oracle_attention_bwd_f64_ex(
             _ptr(q, c), _ptr(k, c), _ptr(v, c), _ptr(dout, c), B, H, H_kv, L_q, L_k, D,
             float(scale), int(bool(causal)), int(window_left), int(window_right),
+            m.ctypes.data_as(ctypes.c_void_p) if m is not None else None, mtype, sb, sh, sq,
             _ptr(dq, c), _ptr(dk, c), _ptr(dv, c), _ptr(de, c) if de is not None else None,
             _ptr(absb[0], c) if with_abs else None, _ptr(absb[1], c) if with_abs else None,
             _ptr(absb[2], c) if with_abs else None, int(n_threads))
@@ -340,11 +349,11 @@ class Oracle:
         return dq, dk, dv
 
     def attention_bwd(self, q, k, v, dout, dtype, scale, causal=False, window_left=-1,
-                      window_right=-1, delta_err=None, with_abs=False):
+                      window_right=-1, delta_err=None, with_abs=False, mask=None):
         """attention_bwd_f64 on fp16/bf16 bit patterns (decoded exactly)."""
         dec = [self.decode(x, dtype) for x in (q, k, v, dout)]
         return self.attention_bwd_f64(*dec, scale, causal, window_left, window_right,
-                                      delta_err, with_abs)
+                                      delta_err, with_abs, mask=mask)
 
 
 _default = None

@@ -543,16 +543,19 @@ int oracle_attention_f64(const double *q, const double *k, const double *v,
  * Threads run over (b, K/V head) so that each owns its dk / dv rows.
  * Returns the number of threads used, or a negative value on bad input.
  */
-int oracle_attention_bwd_f64(const double *q, const double *k, const double *v,
-                             const double *dout, int64_t B, int64_t H,
-                             int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
-                             double scale, int causal, int64_t wl, int64_t wr,
-                             double *dq, double *dk, double *dv,
-                             const double *delta_err, double *dq_abs,
-                             double *dk_abs, double *dv_abs, int n_threads)
+static int bwd_core(const double *q, const double *k, const double *v,
+                    const double *dout, int64_t B, int64_t H, int64_t H_kv,
+                    int64_t L_q, int64_t L_k, int64_t D, double scale,
+                    int causal, int64_t wl, int64_t wr, const void *mask,
+                    int mask_type, int64_t stride_b, int64_t stride_h,
+                    int64_t stride_q, double *dq, double *dk, double *dv,
+                    const double *delta_err, double *dq_abs, double *dk_abs,
+                    double *dv_abs, int n_threads)
 {
     if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1 ||
         H % H_kv != 0)
+        return -1;
+    if (mask_type < 0 || mask_type > 3 || (mask_type != 0 && mask == NULL))
         return -1;
     const int64_t group = H / H_kv;
     int used = 1;
@@ -592,10 +595,15 @@ int oracle_attention_bwd_f64(const double *q, const double *k, const double *v,
                     const double *doi = dout + row * D;
                     /* recompute P_i (plain safe softmax of the scaled row) */
                     for (int64_t j = 0; j < L_k; j++) {
-                        if (!visible(i, j, L_k, causal, wl, wr)) { s[j] = -INFINITY; continue; }
+                        int hidden = 0;
+                        double bias = 0.0;
+                        if (mask_type != 0)
+                            bias = mask_value(mask, mask_type, b * stride_b + h * stride_h +
+                                                                   i * stride_q + j, &hidden);
+                        if (hidden || !visible(i, j, L_k, causal, wl, wr)) { s[j] = -INFINITY; continue; }
                         double acc = 0.0;
                         for (int64_t d = 0; d < D; d++) acc += qi[d] * kp[j * D + d];
-                        s[j] = scale * acc;
+                        s[j] = scale * acc + bias;
                     }
                     double m, den;
                     oracle_safe_softmax(s, L_k, p, &den, &m);
@@ -639,3 +647,33 @@ int oracle_attention_bwd_f64(const double *q, const double *k, const double *v,
     return used;
 }
 
+/* The backward without a mask, and with one (read as the forward reads it,
+ * see mask_value): P is the softmax of scale q.k + mask with hidden keys
+ * removed; the mask is a constant, so the gradients keep their form. */
+int oracle_attention_bwd_f64(const double *q, const double *k, const double *v,
+                             const double *dout, int64_t B, int64_t H,
+                             int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
+                             double scale, int causal, int64_t wl, int64_t wr,
+                             double *dq, double *dk, double *dv,
+                             const double *delta_err, double *dq_abs,
+                             double *dk_abs, double *dv_abs, int n_threads)
+{
+    return bwd_core(q, k, v, dout, B, H, H_kv, L_q, L_k, D, scale, causal, wl, wr,
+                    NULL, 0, 0, 0, 0, dq, dk, dv, delta_err, dq_abs, dk_abs, dv_abs,
+                    n_threads);
+}
+
+int oracle_attention_bwd_f64_ex(const double *q, const double *k, const double *v,
+                                const double *dout, int64_t B, int64_t H,
+                                int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
+                                double scale, int causal, int64_t wl, int64_t wr,
+                                const void *mask, int mask_type, int64_t stride_b,
+                                int64_t stride_h, int64_t stride_q, double *dq,
+                                double *dk, double *dv, const double *delta_err,
+                                double *dq_abs, double *dk_abs, double *dv_abs,
+                                int n_threads)
+{
+    return bwd_core(q, k, v, dout, B, H, H_kv, L_q, L_k, D, scale, causal, wl, wr,
+                    mask, mask_type, stride_b, stride_h, stride_q, dq, dk, dv,
+                    delta_err, dq_abs, dk_abs, dv_abs, n_threads);
+}

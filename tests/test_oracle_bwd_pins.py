@@ -197,3 +197,72 @@ def test_module_level_entries():
     assert np.array_equal(oracle.attention_bwd_f64(q, k, v, do, 0.7)[0],
                           oracle.get().attention_bwd_f64(q, k, v, do, 0.7)[0])
     assert callable(oracle.attention_bwd) and callable(oracle.attention_f64)
+
+
+# ------------------------------------------------------------ with a mask
+def test_masked_backward_finite_differences(orc):
+    # an additive mask is a constant: the gradient of the masked forward
+    c = CASES[0]
+    q, k, v, do = _inputs(c, 13)
+    rng = np.random.default_rng(14)
+    m = rng.uniform(-2, 2, size=(1, c["H"], c["L_q"], c["L_k"])).astype(np.float32)
+    m[0, 0, 1, :3] = -np.inf                                         # hidden keys
+    dq, dk, dv = orc.attention_bwd_f64(q, k, v, do, 0.7, mask=m)
+
+    def f(qq, kk, vv):
+        return float((_masked_forward(qq, kk, vv, m) * do).sum())
+
+    eps = 1e-5
+    for idx, (x, g) in enumerate(((q, dq), (k, dk), (v, dv))):
+        for flat in np.random.default_rng(15).choice(x.size, size=12, replace=False):
+            pos = np.unravel_index(flat, x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[pos] += eps
+            xm[pos] -= eps
+            a, b = [q, k, v], [q, k, v]
+            a[idx], b[idx] = xp, xm
+            fd = (f(*a) - f(*b)) / (2 * eps)
+            assert abs(fd - g[pos]) <= 1e-7 * (1 + abs(g[pos])), (idx, pos, fd, g[pos])
+
+
+def _masked_forward(q, k, v, m):
+    # fp64 forward with an additive mask (numpy; the same rule written out)
+    H, H_kv = q.shape[1], k.shape[1]
+    kk = np.repeat(k, H // H_kv, axis=1)
+    vv = np.repeat(v, H // H_kv, axis=1)
+    s = 0.7 * q @ kk.transpose(0, 1, 3, 2) + m.astype(np.float64)
+    mx = s.max(-1, keepdims=True)
+    e = np.exp(s - mx)
+    return (e / e.sum(-1, keepdims=True)) @ vv
+
+
+def test_masked_backward_matches_torch_autograd(orc):
+    c = CASES[2]
+    q, k, v, do = _inputs(c, 16)
+    rng = np.random.default_rng(17)
+    hide = rng.uniform(size=(c["B"], 1, c["L_q"], c["L_k"])) < 0.3
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    kk = tk.repeat_interleave(c["H"] // c["H_kv"], dim=1)
+    vv = tv.repeat_interleave(c["H"] // c["H_kv"], dim=1)
+    i = torch.arange(c["L_q"]).view(-1, 1)
+    j = torch.arange(c["L_k"]).view(1, -1)
+    vis = (j >= i - c["wl"]) & (j <= i + c["wr"]) & ~torch.tensor(hide)
+    s = (0.7 * tq @ kk.transpose(-1, -2)).masked_fill(~vis, float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    p = torch.where(vis.any(dim=-1, keepdim=True), p, torch.zeros_like(p))
+    (p @ vv).backward(torch.tensor(do))
+    dq, dk, dv = orc.attention_bwd_f64(q, k, v, do, 0.7, False, c["wl"], c["wr"], mask=hide)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_causal_pattern_mask_equals_causal_backward(orc):
+    c = CASES[1]
+    q, k, v, do = _inputs(c, 18)
+    i = np.arange(c["L_q"])[:, None]
+    j = np.arange(c["L_k"])[None, :]
+    g1 = orc.attention_bwd_f64(q, k, v, do, 0.7, True)
+    g2 = orc.attention_bwd_f64(q, k, v, do, 0.7, False, mask=(j > i)[None, None])
+    for a, b in zip(g1, g2):
+        assert np.array_equal(a, b)

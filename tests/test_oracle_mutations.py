@@ -63,6 +63,9 @@ MUTATIONS = {
     "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);                /* subnormal: m * 2^-9 */",
                              "v = ldexp((double)m, -10);"),
     "e4m3_nan_missed": ("if (e == 0xf && m == 0x7)", "if (e == 0xf && m == 0x8)"),
+    "bwd_mask_bias_dropped": ("s[j] = scale * acc + bias;", "s[j] = scale * acc;"),
+    "bwd_mask_row_stride_ignored": ("h * stride_h +\n                                                                   i * stride_q + j, &hidden);",
+                                    "h * stride_h +\n                                                                   j, &hidden);"),
     # mask and statistics
     "mask_bool_inverted": ("*hidden = ((const uint8_t *)mask)[idx] != 0;",
                            "*hidden = ((const uint8_t *)mask)[idx] == 0;"),
@@ -105,6 +108,9 @@ def _battery(orc):
     for dt in (F16, BF16):
         yield lambda dt=dt: bwd_pins.test_bit_pattern_entry_decodes_exactly(orc, dt)
     yield lambda: bwd_pins.test_error_scales(orc)
+    yield lambda: bwd_pins.test_masked_backward_finite_differences(orc)
+    yield lambda: bwd_pins.test_masked_backward_matches_torch_autograd(orc)
+    yield lambda: bwd_pins.test_causal_pattern_mask_equals_causal_backward(orc)
     yield lambda: fp8_pins.test_decode_every_code_matches_torch(orc)
     yield lambda: fp8_pins.test_decode_closed_points(orc)
     yield lambda: fp8_pins.test_attention_on_e4m3_equals_fp16_of_same_values(orc)
