@@ -24,7 +24,7 @@ STATUS = {
     -8: "FA_ERR_TIMEOUT", -9: "FA_ERR_WORKSPACE", -10: "FA_ERR_SCRATCH",
 }
 FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
-EXPORTS = ("fa_bwd", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
+EXPORTS = ("fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
            "fa_fwd_host", "fa_fwd_host_workspace_bytes", "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_splitkv_workspace_bytes",
            "fa_status_string", "fa_version")
@@ -80,6 +80,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
                                ctypes.c_float, i, i, i, i, vp, ctypes.c_size_t, vp]
         lib.fa_bwd.restype = i
+        lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, ctypes.c_longlong,
+                                  ctypes.c_longlong, ctypes.c_longlong, i, i, i, i, i, i,
+                                  ctypes.c_float, i, i, i, i, vp, ctypes.c_size_t, vp]
+        lib.fa_bwd_ex.restype = i
         lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
         lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -180,6 +184,17 @@ def fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, H_kv, L_q, L_k, D, scale, 
     return load().fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, H_kv, L_q, L_k, D,
                          float(scale), int(causal), int(window_left), int(window_right),
                          int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, mask, mask_type, mask_stride_b,
+              mask_stride_h, mask_stride_q, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+              window_right, dtype, workspace, workspace_bytes, stream) -> int:
+    """The masked backward C entry point, unchanged."""
+    return load().fa_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, mask, int(mask_type),
+                            int(mask_stride_b), int(mask_stride_h), int(mask_stride_q), B, H,
+                            H_kv, L_q, L_k, D, float(scale), int(causal), int(window_left),
+                            int(window_right), int(dtype), workspace, int(workspace_bytes),
+                            stream)
 
 
 def fa_bwd_workspace_bytes(B, H, L_q, D) -> int:
@@ -335,12 +350,14 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
 
 
 def flash_bwd(q, k, v, out, dout, lse, scale=None, causal=False, window_left=-1,
-              window_right=-1, dq=None, dk=None, dv=None, workspace=None, stream=None):
+              window_right=-1, dq=None, dk=None, dv=None, workspace=None, stream=None,
+              mask=None):
     """Exact attention backward on CUDA tensors: returns (dq, dk, dv).
 
     q, out, dout: [B, H, L_q, D]; k, v: [B, H_kv, L_k, D]; lse: [B, H, L_q]
     fp32 from the forward (same scale and mask).  The workspace is allocated
-    here with torch unless given (a uint8 CUDA tensor, 256-byte aligned)."""
+    here with torch unless given (a uint8 CUDA tensor, 256-byte aligned).
+    ``mask``: the forward's attention mask (as flash_fwd), through fa_bwd_ex."""
     import torch
 
     B, H, L_q, D = q.shape
@@ -368,12 +385,25 @@ def flash_bwd(q, k, v, out, dout, lse, scale=None, causal=False, window_left=-1,
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
-        st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
-                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv,
-                    L_q, L_k, D, scale, causal, window_left, window_right, dtype,
-                    workspace.data_ptr(), workspace.numel(), stream.cuda_stream)
+        if mask is None:
+            st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                        dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                        dv.data_ptr(), B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
+                        window_right, dtype, workspace.data_ptr(), workspace.numel(),
+                        stream.cuda_stream)
+            where = "fa_bwd"
+        else:
+            if not mask.is_cuda or mask.device != q.device:
+                raise ValueError("mask must be on q's device")
+            mtype, sb, sh, sq = mask_layout(mask, B, H, L_q, L_k)
+            st = fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                           dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                           dv.data_ptr(), mask.data_ptr(), mtype, sb, sh, sq, B, H, H_kv, L_q,
+                           L_k, D, scale, causal, window_left, window_right, dtype,
+                           workspace.data_ptr(), workspace.numel(), stream.cuda_stream)
+            where = "fa_bwd_ex"
     if st != FA_OK:
-        raise FaError(st, "fa_bwd")
+        raise FaError(st, where)
     return dq, dk, dv
 
 

@@ -650,11 +650,11 @@ BwdWs bwd_ws(int64_t BH, int64_t L_q, int D) {
   return w;
 }
 
-template <int D, int DT>
+template <int D, int DT, bool kMask>
 int launch_bwd(const BwdParams &prm, const void *out, const void *dout, const float *lse,
                void *dq, int B, int H, cudaStream_t stream) {
   using BG = BwdGeo<D>;
-  auto kern = fa_bwd_kernel<D, DT>;
+  auto kern = fa_bwd_kernel<D, DT, kMask>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   static bool configured[64] = {};
@@ -691,12 +691,14 @@ extern "C" size_t fa_bwd_workspace_bytes(int B, int H, int L_q, int D) {
   return fa::bwd_ws(static_cast<int64_t>(B) * H, L_q, D).total;
 }
 
-extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *out,
-                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
-                      int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
-                      int window_left, int window_right, int dtype, void *workspace,
-                      size_t workspace_bytes, cudaStream_t stream) {
-  using namespace fa;
+namespace fa {
+namespace {
+// Shared body of fa_bwd and fa_bwd_ex (mask == nullptr: no mask).
+int bwd_impl(const void *q, const void *k, const void *v, const void *out, const void *dout,
+             const float *lse, void *dq, void *dk, void *dv, int B, int H, int H_kv, int L_q,
+             int L_k, int D, float scale, int causal, int window_left, int window_right,
+             int dtype, const FwdExtras *mx, void *workspace, size_t workspace_bytes,
+             cudaStream_t stream) {
   if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0) return FA_ERR_SHAPE;
   if (H % H_kv != 0) return FA_ERR_SHAPE;
   if (L_q > kMaxSeq || L_k > kMaxSeq) return FA_ERR_SHAPE;
@@ -714,6 +716,12 @@ extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *o
       !aligned(lse, 4) || !aligned(workspace, 256))
     return FA_ERR_ALIGN;
   if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
+  const bool masked = mx != nullptr && mx->type != FA_MASK_NONE;
+  if (mx != nullptr) {
+    if (mx->type < FA_MASK_NONE || mx->type > FA_MASK_F32) return FA_ERR_ARG;
+    if (mx->sb < 0 || mx->sh < 0 || mx->sq < 0) return FA_ERR_ARG;
+    if (masked && nq && nk && !mx->mask) return FA_ERR_NULL;
+  }
   const int64_t BH = static_cast<int64_t>(B) * H;
   const BwdWs ws = bwd_ws(BH, L_q, D);
   if (nq && nk && workspace_bytes < ws.total) return FA_ERR_WORKSPACE;
@@ -761,6 +769,13 @@ extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *o
   prm.delta = reinterpret_cast<const float *>(wsb + ws.delta_off);
   prm.dk = dk;
   prm.dv = dv;
+  if (masked) {
+    prm.mask = mx->mask;
+    prm.mask_type = mx->type;
+    prm.mask_sb = mx->sb;
+    prm.mask_sh = mx->sh;
+    prm.mask_sq = mx->sq;
+  }
   const int box_cols = D * 2 >= 128 ? 64 : D;
   if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
@@ -768,17 +783,55 @@ extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *o
       !encode_map(&prm.tm_do, dout, dtype, B * H, L_q, D, box_cols) ||
       !encode_map_f32(&prm.tm_dq, prm.dq_acc, B * H, L_q, D, D >= 32 ? 32 : 16))
     return FA_ERR_CUDA;
-  switch (D * 2 + dtype) {
-    case 32: return launch_bwd<16, 0>(prm, out, dout, lse, dq, B, H, stream);
-    case 33: return launch_bwd<16, 1>(prm, out, dout, lse, dq, B, H, stream);
-    case 64: return launch_bwd<32, 0>(prm, out, dout, lse, dq, B, H, stream);
-    case 65: return launch_bwd<32, 1>(prm, out, dout, lse, dq, B, H, stream);
-    case 128: return launch_bwd<64, 0>(prm, out, dout, lse, dq, B, H, stream);
-    case 129: return launch_bwd<64, 1>(prm, out, dout, lse, dq, B, H, stream);
-    case 256: return launch_bwd<128, 0>(prm, out, dout, lse, dq, B, H, stream);
-    case 257: return launch_bwd<128, 1>(prm, out, dout, lse, dq, B, H, stream);
+  switch (D * 2 + dtype + (masked ? 1000 : 0)) {
+    case 32: return launch_bwd<16, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 33: return launch_bwd<16, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 64: return launch_bwd<32, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 65: return launch_bwd<32, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 128: return launch_bwd<64, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 129: return launch_bwd<64, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 256: return launch_bwd<128, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 257: return launch_bwd<128, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 1032: return launch_bwd<16, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1033: return launch_bwd<16, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1064: return launch_bwd<32, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1065: return launch_bwd<32, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1128: return launch_bwd<64, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1129: return launch_bwd<64, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1256: return launch_bwd<128, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1257: return launch_bwd<128, 1, true>(prm, out, dout, lse, dq, B, H, stream);
   }
   return FA_ERR_HEADDIM;
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_bwd(const void *q, const void *k, const void *v, const void *out,
+                      const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                      int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
+                      int window_left, int window_right, int dtype, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream) {
+  return fa::bwd_impl(q, k, v, out, dout, lse, dq, dk, dv, B, H, H_kv, L_q, L_k, D, scale,
+                      causal, window_left, window_right, dtype, nullptr, workspace,
+                      workspace_bytes, stream);
+}
+
+extern "C" int fa_bwd_ex(const void *q, const void *k, const void *v, const void *out,
+                         const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                         const void *mask, int mask_type, long long mask_stride_b,
+                         long long mask_stride_h, long long mask_stride_q, int B, int H,
+                         int H_kv, int L_q, int L_k, int D, float scale, int causal,
+                         int window_left, int window_right, int dtype, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+  fa::FwdExtras mx;
+  mx.mask = mask;
+  mx.type = mask_type;
+  mx.sb = mask_stride_b;
+  mx.sh = mask_stride_h;
+  mx.sq = mask_stride_q;
+  return fa::bwd_impl(q, k, v, out, dout, lse, dq, dk, dv, B, H, H_kv, L_q, L_k, D, scale,
+                      causal, window_left, window_right, dtype, &mx, workspace,
+                      workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

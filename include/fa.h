@@ -254,6 +254,21 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *out, const v
            int dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fa_bwd_ex -- fa_bwd for a forward that used an attention mask (fa_fwd_ex):
+ * P is recomputed with the same mask (same arguments, same reading: a
+ * nonzero bool hides the key, a float is added to the scaled score; element
+ * (b, h, i, j) at mask[b*mask_stride_b + h*mask_stride_h + i*mask_stride_q
+ * + j]).  The mask itself gets no gradient.  Other arguments and errors as
+ * fa_bwd; FA_ERR_ARG for a bad mask_type or a negative stride.
+ */
+int fa_bwd_ex(const void *q, const void *k, const void *v, const void *out, const void *dout,
+              const float *lse, void *dq, void *dk, void *dv, const void *mask, int mask_type,
+              long long mask_stride_b, long long mask_stride_h, long long mask_stride_q, int B,
+              int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
+              int window_left, int window_right, int dtype, void *workspace,
+              size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * fa_fwd_splitkv_static -- fa_fwd_splitkv with no workspace argument: the
  * partials live in a fixed scratch array inside the library (static device
  * memory, FA_STATIC_SCRATCH_BYTES per device).  The pages have no

@@ -273,3 +273,20 @@ def test_host_workspace_bytes(lib):
 ])
 def test_host_argument_errors(lib, kw, code):
     assert _call_host(**kw) == code
+
+
+def _call_bwd_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, **kw):
+    a = dict(BWD_GOOD)
+    a.update(kw)
+    return fa.fa_bwd_ex(a["q"], a["k"], a["v"], a["out"], a["dout"], a["lse"], a["dq"], a["dk"],
+                        a["dv"], mask, mtype, sb, sh, sq, a["B"], a["H"], a["H_kv"], a["L_q"],
+                        a["L_k"], a["D"], a["scale"], a["causal"], a["wl"], a["wr"], a["dtype"],
+                        a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mtype=4), -6), (dict(sq=-1), -6), (dict(mask=0), -1), (dict(D=48), -3),
+    (dict(q=0), -1), (dict(ws_bytes=10), -9),
+])
+def test_bwd_ex_argument_errors(lib, kw, code):
+    assert _call_bwd_ex(**kw) == code

@@ -42,22 +42,29 @@ def _w(**kw):
     return Workload(**base)
 
 
-def _oracle_forward(w, q, k, v):
-    out, lse, _ = oracle.attention_rows(to_bits(q), to_bits(k), to_bits(v), w.dtype,
-                                        w.softmax_scale, w.causal, w.window_left,
-                                        w.window_right)
+def _oracle_forward(w, q, k, v, mask=None):
+    out, lse, _, _ = oracle.attention_rows_ex(to_bits(q), to_bits(k), to_bits(v), w.dtype,
+                                              w.softmax_scale, w.causal, w.window_left,
+                                              w.window_right, mask=mask)
     return out.reshape(w.B, w.H, w.L_q, w.D), lse.reshape(w.B, w.H, w.L_q)
 
 
-def check_bwd(w: Workload, o_lse_from_gpu: bool = False):
+def check_bwd(w: Workload, o_lse_from_gpu: bool = False, mask=None):
+    """``mask``: a CPU torch mask (bool / float16 / float32, broadcastable
+    to [B, H, L_q, L_k]) used by the forward and the backward."""
     import exact_attention_113_b200 as fa
     q, k, v = make_qkv(w)
     do = make_dout(w)
-    o_exact, lse_exact = _oracle_forward(w, q, k, v)
+    mnp = None if mask is None else mask.numpy()
+    md = None if mask is None else mask.cuda()
+    o_exact, lse_exact = _oracle_forward(w, q, k, v, mnp)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     if o_lse_from_gpu:
         out, lse = fa.flash_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal,
-                                window_left=w.window_left, window_right=w.window_right)
+                                window_left=w.window_left, window_right=w.window_right)[:2] \
+            if mask is None else \
+            fa.flash_fwd(qd, kd, vd, scale=w.softmax_scale, causal=w.causal,
+                         window_left=w.window_left, window_right=w.window_right, mask=md)[:2]
     else:
         out = torch.from_numpy(o_exact).to(TORCH_DTYPE[w.dtype]).cuda()
         lse = torch.from_numpy(lse_exact).float().cuda()
@@ -65,7 +72,8 @@ def check_bwd(w: Workload, o_lse_from_gpu: bool = False):
     dk = torch.full_like(kd, float("nan"))
     dv = torch.full_like(vd, float("nan"))
     fa.flash_bwd(qd, kd, vd, out, dod, lse, scale=w.softmax_scale, causal=w.causal,
-                 window_left=w.window_left, window_right=w.window_right, dq=dq, dk=dk, dv=dv)
+                 window_left=w.window_left, window_right=w.window_right, dq=dq, dk=dk, dv=dv,
+                 mask=md)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0, "device watchdog fired"
 
@@ -75,7 +83,7 @@ def check_bwd(w: Workload, o_lse_from_gpu: bool = False):
     e = (np.abs(do64) * (np.abs(o_in - o_exact) + 2.0 ** -23 * np.abs(o_in))).sum(-1)
     dq_r, dk_r, dv_r, dq_a, dk_a, dv_a = oracle.attention_bwd(
         to_bits(q), to_bits(k), to_bits(v), to_bits(do), w.dtype, w.softmax_scale, w.causal,
-        w.window_left, w.window_right, delta_err=e / (2 * u), with_abs=True)
+        w.window_left, w.window_right, delta_err=e / (2 * u), with_abs=True, mask=mnp)
     group = w.H // w.H_kv
     sub = 2.0 ** -25 if w.dtype == F16 else 0.0
     stats = {}
@@ -162,3 +170,32 @@ def test_empty():
     dq, dk, dv = fa.flash_bwd(q, k, k, q, q, lse)
     torch.cuda.synchronize()
     assert torch.all(dq == 0) and dk.numel() == 0
+
+
+# ------------------------------------------------------------ with a mask
+def _mask(shape, kind, seed, p_hide=0.3):
+    g = torch.Generator().manual_seed(seed)
+    if kind == "bool":
+        return torch.rand(shape, generator=g) < p_hide
+    x = torch.randn(shape, generator=g)
+    x = torch.where(torch.rand(shape, generator=g) < p_hide, torch.tensor(float("-inf")), x)
+    return x.to(torch.float16 if kind == "f16" else torch.float32)
+
+
+@pytest.mark.parametrize("kind", ["bool", "f16", "f32"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_masked(kind, D):
+    w = _w(B=2, H=4, H_kv=2, L_q=300, L_k=333, D=D, dtype=BF16, seed=6900 + D)
+    check_bwd(w, mask=_mask((w.B, w.H, w.L_q, w.L_k), kind, 6910 + D))
+
+
+@pytest.mark.parametrize("shape", ["qk", "key_padding"])
+def test_masked_broadcast_and_causal(shape):
+    w = _w(B=2, H=4, H_kv=4, L_q=257, L_k=257, D=32, causal=True, dtype=F16, seed=6950)
+    dims = (1, 1, w.L_q, w.L_k) if shape == "qk" else (w.B, 1, 1, w.L_k)
+    check_bwd(w, mask=_mask(dims, "f32", 6951))
+
+
+def test_masked_end_to_end_with_gpu_forward():
+    w = _w(B=1, H=4, H_kv=2, L_q=500, L_k=500, D=128, dtype=BF16, seed=6960)
+    check_bwd(w, o_lse_from_gpu=True, mask=_mask((w.B, w.H, w.L_q, w.L_k), "bool", 6961))
