@@ -687,7 +687,7 @@ int launch_bwd(const BwdParams &prm, const void *out, const void *dout, const fl
 
 extern "C" size_t fa_bwd_workspace_bytes(int B, int H, int L_q, int D) {
   if (B < 1 || H < 1 || L_q < 0 || L_q > fa::kMaxSeq) return 0;
-  if (D != 16 && D != 32 && D != 64 && D != 128) return 0;
+  if (!fa::valid_fwd_d(D)) return 0;
   return fa::bwd_ws(static_cast<int64_t>(B) * H, L_q, D).total;
 }
 
@@ -705,7 +705,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *out, const
   if (static_cast<int64_t>(B) * H_kv * ((static_cast<int64_t>(L_k) + 127) / 128) >
       (1ll << 31) - 1)
     return FA_ERR_SHAPE;
-  if (D != 16 && D != 32 && D != 64 && D != 128) return FA_ERR_HEADDIM;
+  if (!valid_fwd_d(D)) return FA_ERR_HEADDIM;
   if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   const bool nq = L_q > 0, nk = L_k > 0;
   if ((nq && (!q || !out || !dout || !dq)) || (nk && (!k || !v || !dk || !dv)) ||
@@ -776,12 +776,12 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *out, const
     prm.mask_sh = mx->sh;
     prm.mask_sq = mx->sq;
   }
-  const int box_cols = D * 2 >= 128 ? 64 : D;
+  const int box_cols = sw_span(D, 2) / 2;
   if (!encode_map(&prm.tm_q, q, dtype, B * H, L_q, D, box_cols) ||
       !encode_map(&prm.tm_k, k, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_v, v, dtype, B * H_kv, L_k, D, box_cols) ||
       !encode_map(&prm.tm_do, dout, dtype, B * H, L_q, D, box_cols) ||
-      !encode_map_f32(&prm.tm_dq, prm.dq_acc, B * H, L_q, D, D >= 32 ? 32 : 16))
+      !encode_map_f32(&prm.tm_dq, prm.dq_acc, B * H, L_q, D, D % 32 == 0 ? 32 : 16))
     return FA_ERR_CUDA;
   switch (D * 2 + dtype + (masked ? 1000 : 0)) {
     case 32: return launch_bwd<16, 0, false>(prm, out, dout, lse, dq, B, H, stream);
@@ -792,6 +792,14 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *out, const
     case 129: return launch_bwd<64, 1, false>(prm, out, dout, lse, dq, B, H, stream);
     case 256: return launch_bwd<128, 0, false>(prm, out, dout, lse, dq, B, H, stream);
     case 257: return launch_bwd<128, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 96: return launch_bwd<48, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 97: return launch_bwd<48, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 160: return launch_bwd<80, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 161: return launch_bwd<80, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 192: return launch_bwd<96, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 193: return launch_bwd<96, 1, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 224: return launch_bwd<112, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 225: return launch_bwd<112, 1, false>(prm, out, dout, lse, dq, B, H, stream);
     case 1032: return launch_bwd<16, 0, true>(prm, out, dout, lse, dq, B, H, stream);
     case 1033: return launch_bwd<16, 1, true>(prm, out, dout, lse, dq, B, H, stream);
     case 1064: return launch_bwd<32, 0, true>(prm, out, dout, lse, dq, B, H, stream);
@@ -800,6 +808,14 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *out, const
     case 1129: return launch_bwd<64, 1, true>(prm, out, dout, lse, dq, B, H, stream);
     case 1256: return launch_bwd<128, 0, true>(prm, out, dout, lse, dq, B, H, stream);
     case 1257: return launch_bwd<128, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1096: return launch_bwd<48, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1097: return launch_bwd<48, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1160: return launch_bwd<80, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1161: return launch_bwd<80, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1192: return launch_bwd<96, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1193: return launch_bwd<96, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1224: return launch_bwd<112, 0, true>(prm, out, dout, lse, dq, B, H, stream);
+    case 1225: return launch_bwd<112, 1, true>(prm, out, dout, lse, dq, B, H, stream);
   }
   return FA_ERR_HEADDIM;
 }

@@ -84,12 +84,17 @@ struct BwdGeo {
   static constexpr int kDsBytes = 2 * kDsBoxBytes;
   // dO is single-buffered at D = 128 (its last reader, dV of the step, runs
   // early) to make room for the dQ staging buffer
-  static constexpr int kDoStages = D == 128 ? 1 : 2;
-  // dQ staging: two fp32 boxes of [128 rows][kDqBoxCols], 64 columns a round
-  static constexpr int kDqBoxCols = D >= 32 ? 32 : D;
+  // (D >= 112: K, V, 2 x Q, dS and the dQ staging leave room for one dO)
+  static constexpr int kDoStages = D >= 112 ? 1 : 2;
+  // dQ staging: up to 32 KB of fp32 boxes of [128 rows][kDqBoxCols] a round
+  // (32 columns, 128-byte swizzle; 16 columns, 64-byte swizzle when D is an
+  // odd multiple of 16); the last round may hold fewer boxes
+  static constexpr int kDqBoxCols = D % 32 == 0 ? 32 : 16;
   static constexpr int kDqBoxBytes = 128 * kDqBoxCols * 4;
-  static constexpr int kDqBoxes = D >= 64 ? 2 : 1;        // boxes per round
-  static constexpr int kDqRounds = D / (kDqBoxCols * kDqBoxes);
+  static constexpr int kDqTotalBoxes = D / kDqBoxCols;
+  static constexpr int kDqBoxes = (32768 / kDqBoxBytes) < kDqTotalBoxes
+                                      ? (32768 / kDqBoxBytes) : kDqTotalBoxes;   // per round
+  static constexpr int kDqRounds = (kDqTotalBoxes + kDqBoxes - 1) / kDqBoxes;
   static constexpr int kDqSwBytes = kDqBoxCols * 4;       // 128 (SW128) or 64 (SW64)
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
@@ -538,28 +543,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       const uint32_t tAcc = tmem + lane_base + 256u + (wg ? D : 0);
       uint8_t *dst = static_cast<uint8_t *>(wg ? p.dk : p.dv) +
                      (static_cast<size_t>(bh_kv) * p.L_k + j) * D * 2;
-      constexpr int kChunk = D >= 32 ? 32 : D;
-#pragma unroll
-      for (int c = 0; c < D; c += kChunk) {
-        uint32_t o[kChunk];
+      for_o_chunks<D>([&](int c, auto wd) {   // 32-column chunks, 16-column tail
+        constexpr int W = decltype(wd)::value;
+        uint32_t o[W];
         if (n_steps > 0) {
-          tmem_ld_cols<kChunk>(tAcc + c, o);
+          tmem_ld_cols<W>(tAcc + c, o);
           tmem_wait_ld();
           reg_dep(o);
         } else {
 #pragma unroll
-          for (int u = 0; u < kChunk; ++u) o[u] = 0u;
+          for (int u = 0; u < W; ++u) o[u] = 0u;
         }
         if (j < p.L_k) {
 #pragma unroll
-          for (int u = 0; u < kChunk / 8; ++u)
+          for (int u = 0; u < W / 8; ++u)
             *reinterpret_cast<uint4 *>(dst + (c + 8 * u) * 2) = make_uint4(
                 pack2<DT>(__uint_as_float(o[8 * u]), __uint_as_float(o[8 * u + 1])),
                 pack2<DT>(__uint_as_float(o[8 * u + 2]), __uint_as_float(o[8 * u + 3])),
                 pack2<DT>(__uint_as_float(o[8 * u + 4]), __uint_as_float(o[8 * u + 5])),
                 pack2<DT>(__uint_as_float(o[8 * u + 6]), __uint_as_float(o[8 * u + 7])));
         }
-      }
+      });
     }
   } else {
     // =================================================== dQ drain (warps 12-15)
@@ -582,11 +586,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 #pragma unroll
       for (int rd = 0; rd < BG::kDqRounds; ++rd) {
         uint32_t v[BG::kDqBoxes][BG::kDqBoxCols];
+        // boxes of this round (the last round may have fewer)
+        constexpr int kLast = BG::kDqTotalBoxes - (BG::kDqRounds - 1) * BG::kDqBoxes;
+        const int nbox = rd == BG::kDqRounds - 1 ? kLast : BG::kDqBoxes;
         if (ok) {
 #pragma unroll
           for (int bx = 0; bx < BG::kDqBoxes; ++bx)
-            tmem_ld_cols<BG::kDqBoxCols>(
-                tDQ + (rd * BG::kDqBoxes + bx) * BG::kDqBoxCols, v[bx]);
+            if (bx < nbox)
+              tmem_ld_cols<BG::kDqBoxCols>(
+                  tDQ + (rd * BG::kDqBoxes + bx) * BG::kDqBoxCols, v[bx]);
           tmem_wait_ld();
 #pragma unroll
           for (int bx = 0; bx < BG::kDqBoxes; ++bx) reg_dep(v[bx]);
@@ -600,19 +608,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         if (ok) {
 #pragma unroll
           for (int bx = 0; bx < BG::kDqBoxes; ++bx)
+            if (bx < nbox)
 #pragma unroll
-            for (int u = 0; u < kUnits; ++u)
-              *reinterpret_cast<uint4 *>(stage + bx * BG::kDqBoxBytes + r * BG::kDqSwBytes +
-                                         ((u ^ sw) << 4)) =
-                  make_uint4(v[bx][4 * u], v[bx][4 * u + 1], v[bx][4 * u + 2], v[bx][4 * u + 3]);
+              for (int u = 0; u < kUnits; ++u)
+                *reinterpret_cast<uint4 *>(stage + bx * BG::kDqBoxBytes + r * BG::kDqSwBytes +
+                                           ((u ^ sw) << 4)) =
+                    make_uint4(v[bx][4 * u], v[bx][4 * u + 1], v[bx][4 * u + 2],
+                               v[bx][4 * u + 3]);
         }
         fence_proxy_async_smem();
         named_barrier_sync(2, 128);
         if (leader && ok) {
 #pragma unroll
           for (int bx = 0; bx < BG::kDqBoxes; ++bx)
-            tma_reduce_add_3d(&p.tm_dq, smem_u32(stage + bx * BG::kDqBoxBytes),
-                              (rd * BG::kDqBoxes + bx) * BG::kDqBoxCols, q0, bh);
+            if (bx < nbox)
+              tma_reduce_add_3d(&p.tm_dq, smem_u32(stage + bx * BG::kDqBoxBytes),
+                                (rd * BG::kDqBoxes + bx) * BG::kDqBoxCols, q0, bh);
           bulk_commit_group();
         }
       }

@@ -55,7 +55,7 @@ typedef enum {
                              or a size whose byte extent overflows */
     FA_ERR_HEADDIM = -3,  /* D not supported: the 16-bit forward entries take
                              any multiple of 16 in [16, 128]; fa_fwd_fp8
-                             takes 32, 64, 128; fa_bwd 16, 32, 64, 128 */
+                             takes 32, 64, 128 */
     FA_ERR_DTYPE = -4,    /* dtype not FA_F16 / FA_BF16 */
     FA_ERR_ALIGN = -5,    /* q, k, v, out not 16-byte aligned, or lse not
                              4-byte aligned */

@@ -187,14 +187,15 @@ def test_bwd_workspace_bytes(lib):
     B, H, L_q, D = 2, 3, 130, 64
     want = up(B * H * L_q * D * 4) + 2 * up(B * H * 256 * 4)
     assert fa.fa_bwd_workspace_bytes(B, H, L_q, D) == want
-    assert fa.fa_bwd_workspace_bytes(B, H, L_q, 48) == 0
+    assert fa.fa_bwd_workspace_bytes(B, H, L_q, 40) == 0
+    assert fa.fa_bwd_workspace_bytes(B, H, L_q, 48) > 0          # any multiple of 16
     assert fa.fa_bwd_workspace_bytes(0, H, L_q, 64) == 0
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(q=0), -1), (dict(dout=0), -1), (dict(lse=0), -1), (dict(dk=0), -1), (dict(ws=0), -1),
     (dict(B=0), -2), (dict(H=4, H_kv=3), -2), (dict(L_k=-1), -2),
-    (dict(D=48), -3), (dict(dtype=2), -4),
+    (dict(D=40), -3), (dict(D=144), -3), (dict(dtype=2), -4),
     (dict(dq=8), -5), (dict(lse=2), -5), (dict(ws=128), -5),
     (dict(scale=float("nan")), -6), (dict(ws_bytes=1000), -9),
 ])
@@ -285,7 +286,7 @@ def _call_bwd_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, **kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(mtype=4), -6), (dict(sq=-1), -6), (dict(mask=0), -1), (dict(D=48), -3),
+    (dict(mtype=4), -6), (dict(sq=-1), -6), (dict(mask=0), -1), (dict(D=40), -3),
     (dict(q=0), -1), (dict(ws_bytes=10), -9),
 ])
 def test_bwd_ex_argument_errors(lib, kw, code):

@@ -199,3 +199,18 @@ def test_masked_broadcast_and_causal(shape):
 def test_masked_end_to_end_with_gpu_forward():
     w = _w(B=1, H=4, H_kv=2, L_q=500, L_k=500, D=128, dtype=BF16, seed=6960)
     check_bwd(w, o_lse_from_gpu=True, mask=_mask((w.B, w.H, w.L_q, w.L_k), "bool", 6961))
+
+
+# ------------------------------------------------------------ non-power-of-two head dims
+# 16-column fp32 dQ boxes (64-byte swizzle) when D is an odd multiple of 16,
+# a partial last drain round (D = 80, 96, 112), one dO stage at D = 112
+@pytest.mark.parametrize("D", [48, 80, 96, 112])
+@pytest.mark.parametrize("causal", [False, True])
+def test_non_pow2_head_dims(D, causal):
+    check_bwd(_w(B=1, H=4, H_kv=2, L_q=300, L_k=300, D=D, causal=causal, dtype=BF16,
+                 seed=7100 + D))
+
+
+def test_non_pow2_with_mask():
+    w = _w(B=1, H=2, H_kv=2, L_q=257, L_k=333, D=80, dtype=F16, seed=7200)
+    check_bwd(w, mask=_mask((1, 1, w.L_q, w.L_k), "f32", 7201))
