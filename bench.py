@@ -25,6 +25,11 @@ the dQ conversion); the metric counts 2.5x the forward's FLOPs.
 output); its roofline peak is the measured bf16 rate x 2 (the nominal
 fp8 / bf16 ratio of the tensor cores).
 
+--sweep prints one line per named workload (tiny, GPT-2, memory-table,
+the B4 H48 sequence sweep, the GQA window, the roofline point; the decoding
+shapes through fa_fwd_splitkv): % of the tensor peak, of the exp bound and,
+for the memory-bound ones, of HBM.  Not the driver's single-line run.
+
 --splits S (or auto) times fa_fwd_splitkv instead: one split-KV launch plus
 one merge launch per step, for the decoding workloads (a few query rows, a
 long key/value cache), whose roofline is HBM bandwidth rather than the
@@ -587,6 +592,8 @@ def main(argv=None):
                     help="time fa_fwd_fp8 on the inputs converted to E4M3")
     ap.add_argument("--splits", default="0",
                     help="key slices for fa_fwd_splitkv (0: plain fa_fwd; auto)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per named workload (kernel timing only)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -596,6 +603,17 @@ def main(argv=None):
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
+    if args.sweep and args.impl == "ours":
+        import gc
+        named = W.TINY + [W.GPT2] + W.MEMTABLE + W.SWEEP + [W.GQA_WINDOW, W.ROOFLINE]
+        for wk in named + W.DECODE:
+            sub = argparse.Namespace(**vars(args))
+            sub.skip_cpu_baseline = True
+            sub.skip_e2e = True
+            sub.splits = "auto" if wk in W.DECODE else "0"
+            run_ours(sub, wk)
+            gc.collect()
+        return
     w = W.ALL[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
