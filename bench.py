@@ -373,8 +373,15 @@ def run_ours(args, w: W.Workload):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     if bwd or roofline_bound(w, peak, hbm) == "tensor":
         achieved = fm * algorithmic_flops(w) / avg_launch_s / 1e12
+        sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        if fp8:
+            sustained *= 2.0
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    # the same against the power-capped rate of a seconds-long
+                    # cuBLAS loop (this bench's steps also run back to back)
+                    "peak_sustained": sustained,
+                    "frac_of_sustained": round(achieved / sustained, 4),
                     "traffic": profiled_traffic() if w.name == W.ROOFLINE.name else None,
                     "peak_source": (f"{peak_kind} cuBLAS bf16 burst x 2 (nominal fp8 ratio)" if fp8
                                     else f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)")}
