@@ -26,8 +26,8 @@ STATUS = {
 FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
 EXPORTS = ("fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
            "fa_fwd_host", "fa_fwd_host_workspace_bytes", "fa_fwd_splitkv",
-           "fa_fwd_splitkv_static", "fa_get_device_status", "fa_splitkv_workspace_bytes",
-           "fa_status_string", "fa_version")
+           "fa_fwd_splitkv_static", "fa_get_device_status", "fa_selftest_wait_timeout",
+           "fa_splitkv_workspace_bytes", "fa_status_string", "fa_version")
 # size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -90,6 +90,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_get_device_status.argtypes = [vp]
         lib.fa_get_device_status.restype = i
+        lib.fa_selftest_wait_timeout.argtypes = [vp, vp]
+        lib.fa_selftest_wait_timeout.restype = i
         lib.fa_status_string.argtypes = [i]
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_version.argtypes = []
@@ -235,6 +237,30 @@ def choose_splits(B, H, L_q, L_k, sm_count=148, H_kv=None) -> int:
 
 def fa_get_device_status(stream=None) -> int:
     return load().fa_get_device_status(stream)
+
+
+def fa_selftest_wait_timeout(result, stream=None) -> int:
+    """The C entry point: `result` is a device pointer to 6 ints."""
+    return load().fa_selftest_wait_timeout(result, stream)
+
+
+def selftest_wait_timeout(device=None) -> dict:
+    """Run the watchdog self-test on `device` (about 1 s of one SM) and
+    return its six result fields plus the device status read afterwards."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    with torch.cuda.device(dev):
+        res = torch.full((6,), -1, dtype=torch.int32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+        st = fa_selftest_wait_timeout(res.data_ptr(), stream.cuda_stream)
+        if st != 0:
+            raise FaError(st, "fa_selftest_wait_timeout")
+        status = fa_get_device_status(stream.cuda_stream)
+        r = [int(x) for x in res.cpu()]
+    keys = ("done_ok", "never_ok", "abort_flag", "wait_ms", "follower_ok", "follower_ms")
+    out = dict(zip(keys, r))
+    out["status"] = status
+    return out
 
 
 def status_string(status: int) -> str:

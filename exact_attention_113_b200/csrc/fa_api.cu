@@ -113,10 +113,10 @@ __global__ void fill_kernel(float *p, size_t n, float value) {
   for (; i < n; i += stride) p[i] = value;
 }
 
-template <int D, int DT, bool kMask>
-int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
-  using G = Geo<D>;
-  auto kern = fa_fwd_kernel<D, DT, kMask>;
+template <int D, int DT, bool kMask, bool kHalfS>
+int launch_kernel(const FwdParams &prm, int B, int H, cudaStream_t stream) {
+  using G = Geo<D, DT == 2 ? 1 : 2>;
+  auto kern = fa_fwd_kernel<D, DT, kMask, kHalfS>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   static bool configured[64] = {};
@@ -136,6 +136,16 @@ int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
             1, 1);
   kern<<<grid, kThreads, G::kSmemBytes, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// D > 64 with one query tile per CTA takes the half-S schedule (16-bit
+// inputs); everything else the kernel's default for its head dim.
+template <int D, int DT, bool kMask>
+int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
+  if constexpr (D > 64 && DT != 2) {
+    if (prm.tiles == 1) return launch_kernel<D, DT, kMask, true>(prm, B, H, stream);
+  }
+  return launch_kernel<D, DT, kMask, false>(prm, B, H, stream);
 }
 
 // Split-KV workspace: partial O [n_splits][rows][D] fp32, then (m, l)
@@ -901,6 +911,55 @@ extern "C" int fa_fwd_splitkv_static(const void *q, const void *k, const void *v
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
                   window_right, dtype, n_splits, scratch, FA_STATIC_SCRATCH_BYTES, nullptr,
                   stream);
+}
+
+namespace fa {
+// Watchdog self-test: the library's bounded waits (sm100.cuh) on a phase
+// that completes and on one that nothing completes; see the header.
+__global__ void __launch_bounds__(64, 1) wait_selftest_kernel(int *result) {
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar[0]), 1);
+    mbar_init(smem_u32(&bar[1]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int *flag = &abort_flag;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp == 0) {
+    if (elect_one()) mbar_arrive(smem_u32(&bar[0]));
+    __syncwarp();
+    const bool done = mbar_wait_warp(smem_u32(&bar[0]), 0, flag);
+    const unsigned long long t0 = globaltimer_ns();
+    const bool never = mbar_wait_warp(smem_u32(&bar[1]), 0, flag);
+    const unsigned long long t1 = globaltimer_ns();
+    if (lane == 0) {
+      result[0] = done ? 1 : 0;
+      result[1] = never ? 1 : 0;
+      result[2] = *flag;
+      result[3] = static_cast<int>((t1 - t0) / 1000000ull);
+    }
+  } else {
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kWaitLimitNs / 2) __nanosleep(1000);
+    const unsigned long long t1 = globaltimer_ns();
+    const bool never = mbar_wait_warp(smem_u32(&bar[1]), 0, flag);
+    const unsigned long long t2 = globaltimer_ns();
+    if (lane == 0) {
+      result[4] = never ? 1 : 0;
+      result[5] = static_cast<int>((t2 - t1) / 1000000ull);
+    }
+  }
+}
+}  // namespace fa
+
+extern "C" int fa_selftest_wait_timeout(int *result, cudaStream_t stream) {
+  if (result == nullptr) return FA_ERR_NULL;
+  fa::wait_selftest_kernel<<<1, 64, 0, stream>>>(result);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 extern "C" int fa_get_device_status(cudaStream_t stream) {

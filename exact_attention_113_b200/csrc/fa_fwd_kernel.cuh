@@ -18,20 +18,34 @@
 //   warp  11    idle
 // Each softmax thread owns one query row, which is one TMEM lane.
 // Registers: launched at kLaunchRegs per thread; the third warpgroup gives
-// back down to kSmallRegs and the two softmax warpgroups grow to kBigRegs:
-//   2*128*kBigRegs + 128*kSmallRegs <= 384*kLaunchRegs (64512 <= 64512).
+// back down to RegSplit::kSmall and the two softmax warpgroups grow to
+// RegSplit::kBig: 2*128*kBig + 128*kSmall = 384*kLaunchRegs (64512).
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D).  P_t (fp16/bf16, two per 32-bit column) is read by the
 // PV MMA straight from TMEM.
 //
-// D = 128 (TMEM full): P_t is written over the first 64 columns of S_t, and
-// the two query tiles ping-pong.  MMA issue order per K/V block j:
+// D > 64, two query tiles (TMEM full): P_t is written over the first 64
+// columns of S_t, and the two tiles ping-pong.  MMA issue order per K/V
+// block j:
 //   S0(j), PV1(j-1), S1(j), PV0(j)
 // so that while softmax warpgroup 0 works on S0(j), the tensor pipe runs
 // PV1(j-1) and S1(j), and the other way round.  S_t(j+1) is issued after
 // PV_t(j), which reads P_t from the same TMEM columns; tcgen05 MMAs issued by
 // one thread execute in issue order.
+//
+// D > 64, one query tile (kHalfS; problems with fewer query tiles than SMs,
+// decoding): with no second tile to ping-pong with, S_t is computed in two
+// 64-key halves and P_t is written over the second half, columns [64, 128).
+// Per block j the MMA issuer runs
+//   S_t(j) keys [0, 64)     once the softmax holds S_t(j-1) (s_free),
+//   PV_t(j-1)               once P_t(j-1) is in TMEM (p_full),
+//   S_t(j) keys [64, 128)   into the columns PV_t(j-1) has just read,
+// so the softmax of block j starts on the first half while the tensor pipe
+// still runs PV_t(j-1) and the second half.  (With two tiles this schedule
+// measured 11-15 % slower than the ping-pong: the N = 64 halves and the two
+// softmax warpgroups competing for the exp unit cost more than the shorter
+// chain saves.)
 //
 // D <= 64 (room to spare): P_t has its own columns [384 + 64t, 448 + 64t).
 // The softmax frees S_t as soon as it holds the row in registers and its
@@ -58,10 +72,17 @@ constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kBN = 128;        // keys per K/V block
 constexpr int kThreads = 384;
 constexpr uint32_t kLaunchRegs = 168;   // 65536 / 384, rounded down to 8
-constexpr uint32_t kBigRegs = 224;
-constexpr uint32_t kSmallRegs = 56;
-static_assert(2 * 128 * kBigRegs + 128 * kSmallRegs <= kThreads * kLaunchRegs,
-              "register split must fit in the launch allocation");
+// Softmax / other-warpgroup register split per instance: the half-S issuer
+// keeps more state than 56 registers hold (fewest spills measured with
+// ptxas -v for each choice).
+template <int D, int DT, bool kHalfS>
+struct RegSplit {
+  static constexpr uint32_t kBig = !kHalfS ? 224 : (D < 128 ? 216 : (DT == 2 ? 224 : 208));
+  static constexpr uint32_t kSmall = (kThreads * kLaunchRegs - 2 * 128 * kBig) / 128;
+  static_assert(kSmall % 8 == 0 && kSmall >= 24, "setmaxnreg takes multiples of 8");
+  static_assert(2 * 128 * kBig + 128 * kSmall <= kThreads * kLaunchRegs,
+                "register split must fit in the launch allocation");
+};
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;     // Q and K
 constexpr int kLoadWarpV = 10;   // V
@@ -163,13 +184,14 @@ struct Bars {
   uint64_t q_full[2];
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
-  uint64_t s_full[2];
-  uint64_t s_free[2];    // split-P schedule: softmax holds S_t in registers
+  uint64_t s_full[2];     // S_t complete (half-S: keys [64, 128) of S_t)
+  uint64_t s_free[2];     // softmax holds S_t in registers
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  uint64_t s_lo_full[2];  // half-S: keys [0, 64) of S_t complete
 };
 
 // Key range [lo, hi) in blocks for query rows [first, last] of one tile.
@@ -312,9 +334,11 @@ __device__ __forceinline__ void store_p_half(uint32_t base, int half, const uint
     tmem_st_x32(base + 32u * half, pk);
 }
 
-template <int D, int DT, bool kMask>
+template <int D, int DT, bool kMask, bool kHalfS>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
-  // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 inputs (bf16 output)
+  // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 inputs (bf16 output).  kHalfS: the
+  // half-S schedule (D > 64, one query tile per CTA).
+  static_assert(!kHalfS || D > 64, "half-S schedule is for D > 64");
   constexpr bool kF8 = DT == 2;
   constexpr int kES = kF8 ? 1 : 2;
   constexpr int kKStep = 32 / kES;             // K of one MMA instruction (32 bytes)
@@ -325,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   // threads are bound by their own instruction stream; neutral otherwise.
   constexpr int kPoly = (kF8 && D == 128) ? 8 : G::kPolyPeriod;
   constexpr int kSlots = G::kSlots;
+  static_assert(sizeof(Bars<kSlots>) <= G::kBarBytes, "barrier block");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -395,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&bars->q_full[t]), 1);
       mbar_init(smem_u32(&bars->s_full[t]), 1);
+      if (kHalfS) mbar_init(smem_u32(&bars->s_lo_full[t]), 1);
       mbar_init(smem_u32(&bars->s_free[t]), kBM);
       mbar_init(smem_u32(&bars->p_full[t]), kBM);
       mbar_init(smem_u32(&bars->pv_done[t]), 1);
@@ -427,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 
   if (warp >= 8) {
   // ===================================================== warpgroup 2
-  regs_dec<kSmallRegs>();
+  regs_dec<RegSplit<D, DT, kHalfS>::kSmall>();
   if (warp == kLoadWarp || warp == kLoadWarpV) {
     // =================================================== TMA producers
     // Warp 9 loads Q and the K ring, warp 10 the V ring.  The whole warp
@@ -514,7 +540,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       };
       auto issue_pv = [&](int t, int slot) {
         const uint32_t vlo = desc_lo(sRing + slot * G::kTileBytes, G::kBoxBytes);
-        const uint32_t a_tmem = tmem + (G::kSplitP ? 384u + (t ? 64u : 0u) : (t ? 128u : 0u));
+        // P_t: own columns (D <= 64), S_t columns [64, 128) (half-S) or
+        // [0, 64) (ping-pong)
+        const uint32_t a_tmem =
+            tmem + (G::kSplitP ? 384u + (t ? 64u : 0u)
+                               : (t ? 128u : 0u) + (kHalfS ? 64u : 0u));
         const uint32_t d_tmem = tmem + 256u + (t ? D : 0u);
         const bool first = (t ? npv1 : npv0) == 0;
         if (elect_one()) {
@@ -580,7 +610,71 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             commit(smem_u32(&bars->empty[vslot(q - 1)]));
           }
         }
+      } else if constexpr (kHalfS) {
+        // Per tile and block j: S_t(j) keys [0, 64) as soon as the softmax
+        // holds S_t(j-1) in registers (s_free), then PV_t(j-1) once P_t(j-1)
+        // is in TMEM (p_full), then S_t(j) keys [64, 128) into the columns
+        // that PV_t(j-1) has just read P from (MMAs of one thread run in
+        // issue order).
+        int ns0 = 0, ns1 = 0;
+        constexpr uint32_t kIdescHalf =
+            kF8 ? make_idesc_e4m3(kBM, kBN / 2, 0, 0) : make_idesc_f16(kBM, kBN / 2, DT, 0, 0);
+        auto issue_s_half = [&](int t, int slot, int h) {
+          const uint32_t qlo = t ? q_lo1 : q_lo0;
+          const uint32_t klo =
+              desc_lo(sRing + slot * G::kTileBytes + h * (kBN / 2) * G::kSwBytes, 16);
+          const uint32_t d_tmem = tmem + (t ? 128u : 0u) + (h ? 64u : 0u);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / kKStep; ++kk) {
+              const int byte = kk * 32;
+              const uint32_t off =
+                  ((byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes)) >> 4;
+              mma_ss_t<kF8>(d_tmem, desc_join(qlo + off, kHi), desc_join(klo + off, kHi),
+                            kIdescHalf, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(smem_u32(h ? &bars->s_full[t] : &bars->s_lo_full[t]));
+          }
+          __syncwarp();
+        };
+        auto tile_step = [&](int t, int j, int q) -> bool {
+          const bool cur = j < hi && in(t, j);
+          if (cur) {
+            const int ns = t ? ns1 : ns0;
+            if (ns > 0) {
+              if (!mbar_wait_warp(smem_u32(&bars->s_free[t]), (ns - 1) & 1, abort_flag))
+                return false;
+              tc_fence_after_sync();
+            }
+            issue_s_half(t, kslot(q), 0);
+          }
+          if (j > lo && in(t, j - 1)) {
+            if (!mbar_wait_warp(smem_u32(&bars->full[vslot(q - 1)]), vpar(q - 1), abort_flag) ||
+                !mbar_wait_warp(smem_u32(&bars->p_full[t]), (t ? npv1 : npv0) & 1, abort_flag))
+              return false;
+            tc_fence_after_sync();
+            issue_pv(t, vslot(q - 1));
+          }
+          if (cur) {
+            issue_s_half(t, kslot(q), 1);
+            if (t) ++ns1; else ++ns0;
+          }
+          return true;
+        };
+        for (int j = lo; j <= hi && ok; ++j) {
+          const int q = j - lo;
+          if (j < hi) {
+            ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+          }
+          ok = tile_step(0, j, q) && tile_step(1, j, q);
+          if (!ok) break;
+          if (j < hi) commit(smem_u32(&bars->empty[kslot(q)]));
+          if (j > lo) commit(smem_u32(&bars->empty[vslot(q - 1)]));
+        }
       } else {
+      // D > 64, two tiles: ping-pong
       for (int j = lo; j < hi && ok; ++j) {
         const int q = j - lo;
         ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
@@ -627,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   }
   } else {
     // =================================================== softmax / epilogue
-    regs_inc<kBigRegs>();
+    regs_inc<RegSplit<D, DT, kHalfS>::kBig>();
     const int t = warp >> 2;             // query tile of this warpgroup
     const int r = tid & 127;             // row within the tile = TMEM lane
     // this tile's scalars (selected, so that nothing is indexed at run time)
@@ -665,7 +759,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     if (trows > 0) {
       for (int n = 0; n < n_blocks; ++n) {
         const int j = tlo + n;
-        ok = mbar_wait_warp(smem_u32(&bars->s_full[t]), n & 1, abort_flag);
+        ok = mbar_wait_warp(
+            smem_u32(kHalfS ? &bars->s_lo_full[t] : &bars->s_full[t]), n & 1, abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
 
@@ -818,8 +913,119 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             store_p_half<DT>(tPs, 1, pk[1]);
             if (warp_rescale && n > 0) scale_o_row<D>(tO, alpha);
           }
+        } else if constexpr (kHalfS) {
+          // D > 64, one tile: the block in two 64-key halves.  Keys [0, 64) arrive
+          // first (s_lo_full) and their exponentials run while the tensor
+          // pipe does PV_t(j-1) and keys [64, 128) (s_full).  Each half takes
+          // its maximum first, then the conditional rescale, then P.  P_t is
+          // stored over columns [64, 128) of S_t once both halves are in
+          // registers; S_t is freed for the next block's first half then.
+          float alpha = 1.0f;
+          bool rescaled = false;
+          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          uint32_t pk[2][32];
+          auto load_half = [&](int h, float (&sv)[kBN / 2]) {
+            uint32_t sr[2][32];
+            tmem_ld_x32(tS + 64 * h, sr[0]);
+            tmem_ld_x32(tS + 64 * h + 32, sr[1]);
+            tmem_wait_ld();
+            reg_dep(sr[0]);
+            reg_dep(sr[1]);
+#pragma unroll
+            for (int c = 0; c < kBN / 2; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
+            const int k0 = j * kBN + 64 * h;   // key of column 0
+            if (!full) {
+              const int lo_c = row_lo - k0;
+              const int hi_c = row_hi - k0;
+#pragma unroll
+              for (int c = 0; c < kBN / 2; ++c)
+                if (c < lo_c || c > hi_c) sv[c] = -INFINITY;
+            }
+            if constexpr (kMask)
+              apply_mask(sv, p, mask_row + static_cast<long long>(k0), min(kBN / 2, p.L_k - k0),
+                         r_loc < trows, p.scale_log2);
+          };
+          // half maximum (four chains of 3-input maxima), in scaled log2 units
+          auto half_max = [&](const float (&sv)[kBN / 2]) -> float {
+            float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+            for (int c = 4; c < kBN / 2 - 4; c += 8)
+#pragma unroll
+              for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
+            const float m = fmax3(fmax3(mx[0], mx[1], sv[kBN / 2 - 4]),
+                                  fmax3(mx[2], mx[3], sv[kBN / 2 - 3]),
+                                  fmaxf(sv[kBN / 2 - 2], sv[kBN / 2 - 1]));
+            return m == -INFINITY ? -INFINITY : m * sl2;
+          };
+          // conditional rescale against a half's maximum; true if this warp
+          // moved its reference
+          auto raise = [&](float m_new) -> bool {
+            m_true = fmaxf(m_true, m_new);
+            if (!__any_sync(0xffffffffu, m_new > m_use + kRescaleThreshold)) return false;
+            const float m_upd = fmaxf(m_use, m_new);
+            const float a = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
+            m_use = m_upd;
+            l *= a;
+            alpha *= a;
+            rescaled = true;
+            return true;
+          };
+          auto exp_half = [&](const float (&sv)[kBN / 2], uint32_t (&pkh)[32], auto poly_ok) {
+            const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
+            const float2 negm = make_float2(-m_sub, -m_sub);
+#pragma unroll
+            for (int c = 0; c < kBN / 2; c += 2) {
+              const int pair = c >> 1;
+              const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2v, negm);
+              float2 pp;
+              if (decltype(poly_ok)::value && (pair % kPoly) == kPoly - 1)
+                pp = exp2_poly2(x);
+              else
+                pp = make_float2(ex2(x.x), ex2(x.y));
+              // l sums the unrounded fp32 weights
+              ls[pair & 1] = __fadd2_rn(ls[pair & 1], pp);
+              put_p<DT>(pkh, pair, pp.x, pp.y);
+            }
+          };
+          auto exp_any = [&](const float (&sv)[kBN / 2], uint32_t (&pkh)[32]) {
+            // masked entries are -inf: only MUFU's ex2 turns them into exact 0
+            if (full)
+              exp_half(sv, pkh, std::true_type{});
+            else
+              exp_half(sv, pkh, std::false_type{});
+          };
+          {
+            float sv[kBN / 2];
+            load_half(0, sv);
+            raise(half_max(sv));
+            exp_any(sv, pk[0]);
+          }
+          // keys [64, 128): issued after PV_t(j-1), so O_t holds blocks < j
+          // and P_t(j-1) has been read once this wait returns
+          ok = mbar_wait_warp(smem_u32(&bars->s_full[t]), n & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after_sync();
+          {
+            float sv[kBN / 2];
+            load_half(1, sv);
+            if (raise(half_max(sv))) {
+              // the first half's P used the old reference: redo it from
+              // S_t keys [0, 64), still in TMEM until s_free
+              float s0[kBN / 2];
+              load_half(0, s0);
+              ls[0] = ls[1] = make_float2(0.f, 0.f);
+              exp_any(s0, pk[0]);
+            }
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&bars->s_free[t]));
+            store_p_half<DT>(tS + 64, 0, pk[0]);
+            exp_any(sv, pk[1]);
+          }
+          l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+          if (rescaled && n > 0) scale_o_row<D>(tO, alpha);
+          store_p_half<DT>(tS + 64, 1, pk[1]);
         } else {
-        // Speculative pass (unmasked blocks, once every row has a reference
+        // D > 64, two tiles.  Speculative pass (unmasked blocks, once every row has a reference
         // max): P = 2^(s*scale*log2e - m_use) against the current reference
         // while the block max is reduced alongside, so that the exponentials
         // do not wait for the max.  If some row's max grew by more than 2^8

@@ -308,6 +308,31 @@ int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out
  */
 int fa_get_device_status(cudaStream_t stream);
 
+/*
+ * fa_selftest_wait_timeout -- exercise the device-side watchdog that every
+ * kernel of this library relies on.  The pages have no counterpart; this
+ * entry point exists so that the failure path can be tested on a GPU
+ * without faulting it.  It enqueues one CTA of two warps on `stream`:
+ *   warp 0 waits on an mbarrier phase that completes (one arrival), then on
+ *          one that nothing completes; that wait gives up after the
+ *          library's wait limit (1 s), raises the CTA's abort flag and sets
+ *          the device status word, and the warp returns;
+ *   warp 1 sleeps 0.5 s, then waits on the same never-completed phase and
+ *          must give up as soon as warp 0 raises the abort flag, before its
+ *          own limit.
+ * `result` (device memory, 6 ints, written by the kernel):
+ *   [0] 1 if the completed wait returned success, [1] 1 if the abandoned
+ *   wait returned success (expected 0), [2] the abort flag afterwards
+ *   (expected 1), [3] warp 0's abandoned wait in ms (about 1000), [4] 1 if
+ *   warp 1's wait returned success (expected 0), [5] warp 1's wait in ms
+ *   (about 500).
+ * The kernel occupies one SM for about 1 s.  Afterwards
+ * fa_get_device_status(stream) returns FA_ERR_TIMEOUT once (and clears
+ * it); the context stays usable.  Returns FA_ERR_NULL for a NULL result,
+ * FA_ERR_CUDA if the launch fails, else FA_OK.
+ */
+int fa_selftest_wait_timeout(int *result, cudaStream_t stream);
+
 /* fa_status_string -- a static, human-readable name for a status code. */
 const char *fa_status_string(int status);
 

@@ -291,3 +291,8 @@ def _call_bwd_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, **kw):
 ])
 def test_bwd_ex_argument_errors(lib, kw, code):
     assert _call_bwd_ex(**kw) == code
+
+
+def test_watchdog_selftest_rejects_null(lib):
+    # returns before any CUDA call
+    assert fa.fa_selftest_wait_timeout(None, None) == -1

@@ -1,0 +1,67 @@
+"""Both forward schedules for head dims above 64, against the fp64 oracle.
+
+At D > 64 the accumulators fill TMEM and the kernel has two schedules:
+  two query tiles per CTA that ping-pong on the tensor pipe, taken when the
+  problem has more 128-row query tiles than the GPU has SMs (148 on B200);
+  the half-S schedule, one tile per CTA, where S is computed in two 64-key
+  halves and P overwrites the second half, taken for fewer tiles than SMs
+  (short problems, decoding).
+The host picks by the tile count, so every case is sized on one side of that
+line: TWO = B 2 x H 40 at L_q 300 is 240 tiles (ping-pong), ONE = B 1 x H 3 is
+9 tiles (half-S).  Large-variance inputs (std 3: scaled scores of spread ~9,
+~13 in log2 units) make the running maximum move past the rescale threshold
+inside blocks, including between a block's two halves, which is the rare
+path of the half-S softmax (P of the first half recomputed)."""
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_113_b200.inputs import BF16, F16, Workload
+from tests.parity import check_full
+from tests.test_mask_gpu import _mask, check_masked
+
+pytestmark = pytest.mark.gpu
+
+TWO = dict(B=2, H=40, H_kv=40)
+ONE = dict(B=1, H=3, H_kv=3)
+
+
+def _w(shape, **kw):
+    base = dict(name="sched", L_q=300, L_k=300, D=128, dtype=F16, seed=9000)
+    base.update(TWO if shape == "two" else ONE)
+    base.update(kw)
+    return Workload(**base)
+
+
+@pytest.mark.parametrize("shape", ["two", "one"])
+@pytest.mark.parametrize("D", [80, 96, 112, 128])
+@pytest.mark.parametrize("dtype", [F16, BF16])
+@pytest.mark.parametrize("causal", [False, True])
+def test_both_schedules(shape, D, dtype, causal):
+    check_full(_w(shape, D=D, dtype=dtype, causal=causal, seed=9000 + D + 7 * dtype + causal),
+               derived=True)
+
+
+@pytest.mark.parametrize("shape", ["two", "one"])
+@pytest.mark.parametrize("D", [96, 128])
+def test_rescale_heavy(shape, D):
+    check_full(_w(shape, D=D, L_q=400, L_k=900, std=3.0, seed=9100 + D), derived=True)
+
+
+@pytest.mark.parametrize("shape", ["two", "one"])
+def test_gqa_window(shape):
+    kw = dict(H_kv=8) if shape == "two" else dict(H=6, H_kv=3)
+    check_full(_w(shape, L_q=500, L_k=700, causal=True, window_left=150, window_right=0,
+                  seed=9200, **kw), derived=True)
+
+
+@pytest.mark.parametrize("shape", ["two", "one"])
+@pytest.mark.parametrize("D,kind", [(128, "bool"), (96, "f32")])
+def test_masked(shape, D, kind):
+    w = _w(shape, D=D, L_k=333, seed=9300 + D)
+    check_masked(w, _mask((w.B, w.H, w.L_q, w.L_k), kind, 9400 + D))
+
+
+@pytest.mark.parametrize("shape", ["two", "one"])
+def test_split_kv(shape):
+    check_full(_w(shape, L_q=300, L_k=1000, seed=9500), n_splits=3, derived=True)
