@@ -23,7 +23,9 @@ the dQ conversion); the metric counts 2.5x the forward's FLOPs.
 
 --fp8 times fa_fwd_fp8 on the workload's inputs converted to E4M3 (bf16
 output); its roofline peak is the measured bf16 rate x 2 (the nominal
-fp8 / bf16 ratio of the tensor cores).
+fp8 / bf16 ratio of the tensor cores).  With --splits it times
+fa_fwd_fp8_splitkv (an fp8 key/value cache; HBM-bound decodes count the
+inputs at one byte per element).
 
 --sweep prints one line per named workload (tiny, GPT-2, memory-table,
 the B4 H48 sequence sweep, the GQA window, the roofline point; the decoding
@@ -328,7 +330,7 @@ def run_ours(args, w: W.Workload):
         def step():
             fa.flash_fwd_fp8(q, k, v, scale=w.softmax_scale, causal=w.causal,
                              window_left=w.window_left, window_right=w.window_right,
-                             out=out, lse=lse, stream=stream)
+                             out=out, lse=lse, stream=stream, n_splits=n_splits, workspace=ws)
     else:
         def step():
             fa.flash_fwd(q, k, v, scale=w.softmax_scale, causal=w.causal,
@@ -371,7 +373,8 @@ def run_ours(args, w: W.Workload):
     if fp8:
         peak *= 2.0                 # nominal fp8 / bf16 dense ratio
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    if bwd or roofline_bound(w, peak, hbm) == "tensor":
+    in_bytes = 1 if fp8 else 2
+    if bwd or roofline_bound(w, peak, hbm, in_bytes) == "tensor":
         achieved = fm * algorithmic_flops(w) / avg_launch_s / 1e12
         sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         if fp8:
@@ -386,12 +389,12 @@ def run_ours(args, w: W.Workload):
                     "peak_source": (f"{peak_kind} cuBLAS bf16 burst x 2 (nominal fp8 ratio)" if fp8
                                     else f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)")}
     else:
-        achieved = min_hbm_bytes(w) / avg_launch_s / 1e9
+        achieved = min_hbm_bytes(w, in_bytes) / avg_launch_s / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                     "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
                     "peak_source": f"{peak_kind} HBM copy bandwidth"}
     roofline.update({"algorithmic_flop_per_launch": fm * algorithmic_flops(w),
-                     "min_hbm_bytes_per_launch": min_hbm_bytes(w)})
+                     "min_hbm_bytes_per_launch": min_hbm_bytes(w, in_bytes)})
     if bwd:
         roofline["traffic"] = None
         roofline["timed"] = "whole step: prep, gradient kernel and dQ conversion launches"
@@ -512,19 +515,20 @@ def resolve_splits(arg: str, w: W.Workload, sm_count: int = 148) -> int:
     return int(arg)
 
 
-def roofline_bound(w: W.Workload, tflops: float, gbs: float) -> str:
+def roofline_bound(w: W.Workload, tflops: float, gbs: float, in_bytes: int = 2) -> str:
     """Whichever of the tensor pipe and HBM takes longer for the workload's
     algorithmic FLOPs and minimum bytes."""
     t_tensor = algorithmic_flops(w) / (tflops * 1e12)
-    t_hbm = min_hbm_bytes(w) / (gbs * 1e9)
+    t_hbm = min_hbm_bytes(w, in_bytes) / (gbs * 1e9)
     return "tensor" if t_tensor >= t_hbm else "hbm"
 
 
-def min_hbm_bytes(w: W.Workload) -> int:
-    """Q, K, V read once, O written once (2 B/elem), lse written (4 B/row)."""
-    qo = 2 * w.B * w.H * w.L_q * w.D * 2
-    kv = 2 * w.B * w.H_kv * w.L_k * w.D * 2
-    return qo + kv + 4 * w.B * w.H * w.L_q
+def min_hbm_bytes(w: W.Workload, in_bytes: int = 2) -> int:
+    """Q, K, V read once (in_bytes per element: 2, or 1 for E4M3 codes), O
+    written once (2 B/elem: fp16 / bf16), lse written (4 B/row)."""
+    q = w.B * w.H * w.L_q * w.D
+    kv = 2 * w.B * w.H_kv * w.L_k * w.D
+    return (q + kv) * in_bytes + q * 2 + 4 * w.B * w.H * w.L_q
 
 
 def workload_config(w: W.Workload, world: int) -> dict:

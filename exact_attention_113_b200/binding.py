@@ -25,6 +25,7 @@ STATUS = {
 }
 FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
 EXPORTS = ("fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
+           "fa_fwd_fp8_splitkv",
            "fa_fwd_host", "fa_fwd_host_workspace_bytes", "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_selftest_wait_timeout",
            "fa_splitkv_workspace_bytes", "fa_status_string", "fa_version")
@@ -66,6 +67,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f = ctypes.c_float
         lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, i, i, vp]
         lib.fa_fwd_fp8.restype = i
+        lib.fa_fwd_fp8_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, i,
+                                           i, i, vp, ctypes.c_size_t, vp]
+        lib.fa_fwd_fp8_splitkv.restype = i
         lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, i, vp,
                                     ctypes.c_size_t, i, vp]
         lib.fa_fwd_host.restype = i
@@ -125,6 +129,16 @@ def fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, des
     return load().fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, float(scale),
                              float(descale_q), float(descale_k), float(descale_v), int(causal),
                              int(window_left), int(window_right), stream)
+
+
+def fa_fwd_fp8_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q,
+                       descale_k, descale_v, causal, window_left, window_right, n_splits,
+                       workspace, workspace_bytes, stream) -> int:
+    """The fp8 (E4M3) split-KV C entry point, unchanged."""
+    return load().fa_fwd_fp8_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, float(scale),
+                                     float(descale_q), float(descale_k), float(descale_v),
+                                     int(causal), int(window_left), int(window_right),
+                                     int(n_splits), workspace, int(workspace_bytes), stream)
 
 
 def fa_fwd_host(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
@@ -435,10 +449,13 @@ def flash_bwd(q, k, v, out, dout, lse, scale=None, causal=False, window_left=-1,
 
 def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1.0,
                   causal=False, window_left=-1, window_right=-1, return_lse=True, out=None,
-                  lse=None, stream=None):
+                  lse=None, stream=None, n_splits=0, workspace=None):
     """Exact attention forward on fp8 E4M3 CUDA tensors (torch.float8_e4m3fn
     or uint8 codes), q [B, H, L_q, D], k, v [B, H_kv, L_k, D]; real values are
-    code * descale.  Returns (out bf16 [B, H, L_q, D], lse or None)."""
+    code * descale.  Returns (out bf16 [B, H, L_q, D], lse or None).
+    ``n_splits`` > 0 (or "auto") goes through fa_fwd_fp8_splitkv with that
+    many key slices; the workspace is allocated here with torch unless
+    given (a uint8 CUDA tensor, 256-byte aligned)."""
     import torch
 
     B, H, L_q, D = q.shape
@@ -458,13 +475,29 @@ def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1
         lse = None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    if n_splits == "auto":
+        n_splits = choose_splits(B, H, L_q, L_k,
+                                 torch.cuda.get_device_properties(q.device).multi_processor_count,
+                                 H_kv=H_kv)
     with torch.cuda.device(q.device):
-        st = fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                        lse.data_ptr() if lse is not None else None, B, H, H_kv, L_q, L_k, D,
-                        scale, descale_q, descale_k, descale_v, causal, window_left,
-                        window_right, stream.cuda_stream)
+        if not n_splits:
+            st = fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            lse.data_ptr() if lse is not None else None, B, H, H_kv, L_q, L_k,
+                            D, scale, descale_q, descale_k, descale_v, causal, window_left,
+                            window_right, stream.cuda_stream)
+            where = "fa_fwd_fp8"
+        else:
+            need = fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits)
+            if workspace is None:
+                workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+            st = fa_fwd_fp8_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None, B, H, H_kv,
+                                    L_q, L_k, D, scale, descale_q, descale_k, descale_v, causal,
+                                    window_left, window_right, n_splits, workspace.data_ptr(),
+                                    workspace.numel(), stream.cuda_stream)
+            where = "fa_fwd_fp8_splitkv"
     if st != FA_OK:
-        raise FaError(st, "fa_fwd_fp8")
+        raise FaError(st, where)
     return out, lse
 
 

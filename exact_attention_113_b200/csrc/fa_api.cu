@@ -138,11 +138,11 @@ int launch_kernel(const FwdParams &prm, int B, int H, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// D > 64 with one query tile per CTA takes the half-S schedule (16-bit
-// inputs); everything else the kernel's default for its head dim.
+// D > 64 with one query tile per CTA takes the half-S schedule; everything
+// else the kernel's default for its head dim.
 template <int D, int DT, bool kMask>
 int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
-  if constexpr (D > 64 && DT != 2) {
+  if constexpr (D > 64) {
     if (prm.tiles == 1) return launch_kernel<D, DT, kMask, true>(prm, B, H, stream);
   }
   return launch_kernel<D, DT, kMask, false>(prm, B, H, stream);
@@ -161,13 +161,15 @@ size_t ws_total_bytes(int64_t rows, int D, int n_splits) {
 }
 
 // Merge the key slices of every row: m = max_s m_s, w_s = 2^(m_s - m),
-// O = sum_s w_s O_s / sum_s w_s l_s, lse = (m + log2 l) ln 2.  One warp per
-// row; the slices' partial sums are exact softmax pieces of the same row
-// (online-softmax merge of "FlashAttention算法原理与性能优化实战" §1.2.2).
+// O = oscale * sum_s w_s O_s / sum_s w_s l_s, lse = (m + log2 l) ln 2.  One
+// warp per row; the slices' partial sums are exact softmax pieces of the
+// same row (online-softmax merge of "FlashAttention算法原理与性能优化实战"
+// §1.2.2).  DT: 0 fp16 / 1 bf16 output, 2 (fp8 inputs) bf16 output; oscale
+// is descale_v for fp8 inputs, else 1.
 template <int D, int DT>
 __global__ void __launch_bounds__(256) fa_combine_kernel(const float *ws_o, const float2 *ws_ml,
                                                          void *out, float *lse, int n_splits,
-                                                         long long rows_total) {
+                                                         long long rows_total, float oscale) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows_total) return;
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *ws_o, cons
       }
     }
   }
-  const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+  const float inv_l = l > 0.0f ? oscale / l : 0.0f;
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
     const int d = lane + 32 * u;
@@ -209,10 +211,10 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *ws_o, cons
 
 template <int D, int DT>
 int launch_combine(const float *ws_o, const float2 *ws_ml, void *out, float *lse, int n_splits,
-                   long long rows_total, cudaStream_t stream) {
+                   long long rows_total, cudaStream_t stream, float oscale = 1.0f) {
   const unsigned blocks = static_cast<unsigned>((rows_total + 7) / 8);
   fa_combine_kernel<D, DT><<<blocks, 256, 0, stream>>>(ws_o, ws_ml, out, lse, n_splits,
-                                                       rows_total);
+                                                       rows_total, oscale);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -270,8 +272,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     if ((mx->smax == nullptr) != (mx->ssum == nullptr)) return FA_ERR_NULL;
     if (L_q > 0 && (!aligned(mx->smax, 4) || !aligned(mx->ssum, 4))) return FA_ERR_ALIGN;
   }
-  // fp8 inputs only through fa_fwd_fp8: no key slices, no mask
-  if (dtype == kE4M3 && (n_splits != 0 || masked)) return FA_ERR_DTYPE;
+  // fp8 inputs only through fa_fwd_fp8 / fa_fwd_fp8_splitkv: no mask
+  if (dtype == kE4M3 && masked) return FA_ERR_DTYPE;
   const int64_t rows_total = static_cast<int64_t>(B) * H * L_q;
   if (n_splits != 0) {
     if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
@@ -437,6 +439,9 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 193: return launch_combine<96, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
     case 224: return launch_combine<112, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
     case 225: return launch_combine<112, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
+    case 66: return launch_combine<32, kE4M3>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream, prm.descale_v);
+    case 130: return launch_combine<64, kE4M3>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream, prm.descale_v);
+    case 258: return launch_combine<128, kE4M3>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream, prm.descale_v);
   }
   return FA_ERR_HEADDIM;
 }
@@ -471,19 +476,43 @@ extern "C" int fa_fwd_ex(const void *q, const void *k, const void *v, void *out,
                   window_right, dtype, 0, nullptr, 0, &mx, stream);
 }
 
-extern "C" int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse,
-                          int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
-                          float descale_q, float descale_k, float descale_v, int causal,
-                          int window_left, int window_right, cudaStream_t stream) {
+namespace fa {
+namespace {
+int fp8_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+             int H_kv, int L_q, int L_k, int D, float scale, float descale_q, float descale_k,
+             float descale_v, int causal, int window_left, int window_right, int n_splits,
+             void *workspace, size_t workspace_bytes, cudaStream_t stream) {
   for (float d : {descale_q, descale_k, descale_v})
     if (!std::isfinite(d) || d < 0.0f) return FA_ERR_ARG;
   if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
   const float s = scale * descale_q * descale_k;   // the scores' full scale
   if (!std::isfinite(s)) return FA_ERR_ARG;
-  fa::FwdExtras ex;
+  FwdExtras ex;
   ex.descale_v = descale_v;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, s, causal, window_left,
-                  window_right, fa::kE4M3, 0, nullptr, 0, &ex, stream);
+                  window_right, kE4M3, n_splits, workspace, workspace_bytes, &ex, stream);
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse,
+                          int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                          float descale_q, float descale_k, float descale_v, int causal,
+                          int window_left, int window_right, cudaStream_t stream) {
+  return fa::fp8_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
+                      descale_v, causal, window_left, window_right, 0, nullptr, 0, stream);
+}
+
+extern "C" int fa_fwd_fp8_splitkv(const void *q, const void *k, const void *v, void *out,
+                                  float *lse, int B, int H, int H_kv, int L_q, int L_k, int D,
+                                  float scale, float descale_q, float descale_k,
+                                  float descale_v, int causal, int window_left,
+                                  int window_right, int n_splits, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
+  if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
+  return fa::fp8_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
+                      descale_v, causal, window_left, window_right, n_splits, workspace,
+                      workspace_bytes, stream);
 }
 
 extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {
@@ -498,6 +527,7 @@ extern "C" int fa_fwd_splitkv(const void *q, const void *k, const void *v, void 
                               int dtype, int n_splits, void *workspace, size_t workspace_bytes,
                               cudaStream_t stream) {
   if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, causal, window_left,
                   window_right, dtype, n_splits, workspace, workspace_bytes, nullptr, stream);
 }
@@ -898,6 +928,7 @@ extern "C" int fa_fwd_splitkv_static(const void *q, const void *k, const void *v
                                      int window_right, int dtype, int n_splits,
                                      cudaStream_t stream) {
   if (n_splits < 1 || n_splits > fa::kMaxSplits) return FA_ERR_ARG;
+  if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   // the size limit first, so that an oversized problem never reaches the GPU
   // (sizes fwd_impl would reject fall through to its own error codes)
   if (B >= 1 && H >= 1 && L_q >= 0 && L_q <= fa::kMaxSeq &&

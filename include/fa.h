@@ -215,6 +215,21 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float
                    cudaStream_t stream);
 
 /*
+ * fa_fwd_fp8_splitkv -- fa_fwd_fp8 computed in key slices as
+ * fa_fwd_splitkv does (decoding over an fp8 key/value cache).  The slices'
+ * partial outputs are fp32 in units of the V codes; the merge applies
+ * descale_v and writes bf16.  Arguments as fa_fwd_fp8, plus n_splits,
+ * workspace and workspace_bytes as fa_fwd_splitkv (the workspace size is
+ * fa_splitkv_workspace_bytes(B, H, L_q, D, n_splits), the same as for
+ * 16-bit inputs).  D must be 32, 64 or 128 (FA_ERR_HEADDIM otherwise).
+ */
+int fa_fwd_fp8_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
+                       int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                       float descale_q, float descale_k, float descale_v, int causal,
+                       int window_left, int window_right, int n_splits, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * fa_bwd_workspace_bytes -- bytes of device workspace fa_bwd needs (0 if
  * the sizes are invalid): an fp32 dQ accumulator [B, H, L_q, D] and two
  * fp32 row vectors [B, H, roundup(L_q, 128)].

@@ -240,9 +240,34 @@ def test_fp8_argument_errors(lib, kw, code):
 
 
 def test_16bit_entries_refuse_the_fp8_code(lib):
-    # dtype 2 is internal to fa_fwd_fp8
+    # dtype 2 is internal to fa_fwd_fp8 / fa_fwd_fp8_splitkv
     assert _call(dtype=2) == -4
     assert _call_split(dtype=2) == -4
+    assert _call_static(dtype=2) == -4
+
+
+def _call_fp8_split(dq=1.0, dk=1.0, dv=1.0, n_splits=2, ws=256, ws_bytes=None, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    if ws_bytes is None:
+        ws_bytes = fa.fa_splitkv_workspace_bytes(a["B"], a["H"], a["L_q"], a["D"],
+                                                 max(1, min(64, n_splits)))
+    return fa.fa_fwd_fp8_splitkv(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["H"],
+                                 a["H_kv"], a["L_q"], a["L_k"], a["D"], a["scale"], dq, dk, dv,
+                                 a["causal"], a["wl"], a["wr"], n_splits, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_splits=0), -6), (dict(n_splits=65), -6), (dict(ws=0), -1), (dict(ws=128), -5),
+    (dict(ws_bytes=100), -9), (dict(D=16), -3), (dict(D=48), -3), (dict(q=0), -1),
+    (dict(q=8), -5), (dict(dq=-1.0), -6), (dict(dv=float("nan")), -6), (dict(scale=-1.0), -6),
+])
+def test_fp8_splitkv_argument_errors(lib, kw, code):
+    assert _call_fp8_split(**kw) == code
+
+
+def test_fp8_splitkv_empty_queries_is_a_no_op(lib):
+    assert _call_fp8_split(L_q=0, ws=0) == 0
 
 
 # ------------------------------------------------------------ host-buffer entry

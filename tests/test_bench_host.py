@@ -97,6 +97,10 @@ def test_roofline_bound_by_workload():
     w = W.DECODE[0]
     kv = 2 * w.B * w.H_kv * w.L_k * w.D * 2
     assert kv < bench.min_hbm_bytes(w) < kv * 1.01
+    # an fp8 cache is read at one byte per element; the bf16 output stays 2
+    assert kv // 2 < bench.min_hbm_bytes(w, 1) < kv // 2 * 1.01
+    q = w.B * w.H * w.L_q * w.D
+    assert bench.min_hbm_bytes(w) - bench.min_hbm_bytes(w, 1) == q + kv // 2
 
 
 def test_resolve_splits():

@@ -31,14 +31,20 @@ def _w(**kw):
     return Workload(**base)
 
 
-def check_fp8(w, descale=(1.0, 1.0, 1.0)):
+def check_fp8(w, descale=(1.0, 1.0, 1.0), n_splits=0):
     import exact_attention_113_b200 as fa
     dq, dk, dv = descale
     q, k, v = make_qkv_fp8(w)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
+    ws = None
+    if n_splits:
+        # NaN-filled: a partial the merge reads but no slice wrote poisons its row
+        nb = fa.fa_splitkv_workspace_bytes(w.B, w.H, w.L_q, w.D, n_splits)
+        ws = torch.full((nb // 4,), float("nan"), dtype=torch.float32,
+                        device="cuda").view(torch.uint8)
     out, lse = fa.flash_fwd_fp8(qd, kd, vd, scale=w.softmax_scale, descale_q=dq, descale_k=dk,
                                 descale_v=dv, causal=w.causal, window_left=w.window_left,
-                                window_right=w.window_right)
+                                window_right=w.window_right, n_splits=n_splits, workspace=ws)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
     s_eff = w.softmax_scale * dq * dk
@@ -86,3 +92,51 @@ def test_fp8_gqa_and_packing(H, H_kv, L_q):
 
 def test_fp8_window():
     check_fp8(_w(L_q=500, L_k=500, D=64, causal=True, window_left=100, seed=8400))
+
+
+# ------------------------------------------------------------ split-KV (fp8 cache)
+# fa_fwd_fp8_splitkv: the key range in slices, merged with descale_v into
+# bf16; the same gate as the single pass (the slices only reorder the fp32
+# sums).
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("n_splits", [1, 3, 8])
+def test_fp8_splitkv_decode(D, n_splits):
+    check_fp8(_w(B=2, H=8, H_kv=2, L_q=1, L_k=3000, D=D, seed=8500 + D), n_splits=n_splits)
+
+
+@pytest.mark.parametrize("L_q,causal", [(16, False), (300, True)])
+def test_fp8_splitkv_tiles(L_q, causal):
+    check_fp8(_w(B=1, H=4, H_kv=4, L_q=L_q, L_k=2500, D=128, causal=causal, seed=8600 + L_q),
+              descale=(0.5, 2.0, 0.25), n_splits=5)
+
+
+def test_fp8_splitkv_more_slices_than_blocks_and_window():
+    check_fp8(_w(B=1, H=2, H_kv=1, L_q=3, L_k=200, D=64, seed=8700), n_splits=9)
+    check_fp8(_w(B=1, H=4, H_kv=2, L_q=200, L_k=1200, D=128, causal=True, window_left=300,
+                 seed=8710), n_splits=4)
+
+
+def test_fp8_splitkv_matches_single_pass():
+    import exact_attention_113_b200 as fa
+    w = _w(B=2, H=16, H_kv=4, L_q=1, L_k=8192, D=128, seed=8800)
+    q, k, v = (t.cuda() for t in make_qkv_fp8(w))
+    o1, l1 = fa.flash_fwd_fp8(q, k, v, descale_v=0.5)
+    o2, l2 = fa.flash_fwd_fp8(q, k, v, descale_v=0.5, n_splits="auto")
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status() == 0
+    # both bf16 roundings of nearly the same fp32 value
+    assert (o1.float() - o2.float()).abs().max().item() <= 2 * 2.0 ** -8
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+# ------------------------------------------------------------ both D = 128 schedules
+# One query tile per CTA (fewer 128-row tiles than SMs) takes the half-S
+# schedule, more tiles the two-tile ping-pong: B 2 x H 40 at L_q 300 is 240
+# tiles (ping-pong), B 1 x H 3 is 9 (half-S).  std 3 moves the running max
+# past the rescale threshold inside blocks.
+@pytest.mark.parametrize("shape", ["two", "one"])
+@pytest.mark.parametrize("causal,std", [(False, 1.0), (True, 1.0), (False, 3.0)])
+def test_fp8_both_schedules(shape, causal, std):
+    hw = dict(B=2, H=40, H_kv=40) if shape == "two" else dict(B=1, H=3, H_kv=3)
+    check_fp8(_w(L_q=300, L_k=400, D=128, causal=causal, std=std,
+                 seed=8900 + int(causal) + int(std), **hw))
