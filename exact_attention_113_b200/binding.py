@@ -25,7 +25,7 @@ STATUS = {
 }
 FA_MASK_NONE, FA_MASK_BOOL, FA_MASK_F16, FA_MASK_F32 = 0, 1, 2, 3
 EXPORTS = ("fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex", "fa_fwd_fp8",
-           "fa_fwd_fp8_splitkv",
+           "fa_fwd_fp8_ex", "fa_fwd_fp8_splitkv",
            "fa_fwd_host", "fa_fwd_host_workspace_bytes", "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_selftest_wait_timeout",
            "fa_splitkv_workspace_bytes", "fa_status_string", "fa_version")
@@ -67,6 +67,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f = ctypes.c_float
         lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, i, i, vp]
         lib.fa_fwd_fp8.restype = i
+        lib.fa_fwd_fp8_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, ll, ll, ll, i, i, i, i,
+                                      i, i, f, f, f, f, i, i, i, vp]
+        lib.fa_fwd_fp8_ex.restype = i
         lib.fa_fwd_fp8_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, i,
                                            i, i, vp, ctypes.c_size_t, vp]
         lib.fa_fwd_fp8_splitkv.restype = i
@@ -129,6 +132,17 @@ def fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, des
     return load().fa_fwd_fp8(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, float(scale),
                              float(descale_q), float(descale_k), float(descale_v), int(causal),
                              int(window_left), int(window_right), stream)
+
+
+def fa_fwd_fp8_ex(q, k, v, out, lse, smax, ssum, mask, mask_type, mask_stride_b, mask_stride_h,
+                  mask_stride_q, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
+                  descale_v, causal, window_left, window_right, stream) -> int:
+    """The fp8 (E4M3) C entry point with mask and statistics, unchanged."""
+    return load().fa_fwd_fp8_ex(q, k, v, out, lse, smax, ssum, mask, int(mask_type),
+                                int(mask_stride_b), int(mask_stride_h), int(mask_stride_q), B, H,
+                                H_kv, L_q, L_k, D, float(scale), float(descale_q),
+                                float(descale_k), float(descale_v), int(causal),
+                                int(window_left), int(window_right), stream)
 
 
 def fa_fwd_fp8_splitkv(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q,
@@ -449,13 +463,16 @@ def flash_bwd(q, k, v, out, dout, lse, scale=None, causal=False, window_left=-1,
 
 def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1.0,
                   causal=False, window_left=-1, window_right=-1, return_lse=True, out=None,
-                  lse=None, stream=None, n_splits=0, workspace=None):
+                  lse=None, stream=None, n_splits=0, workspace=None, mask=None,
+                  return_softmax_stats=False):
     """Exact attention forward on fp8 E4M3 CUDA tensors (torch.float8_e4m3fn
     or uint8 codes), q [B, H, L_q, D], k, v [B, H_kv, L_k, D]; real values are
     code * descale.  Returns (out bf16 [B, H, L_q, D], lse or None).
     ``n_splits`` > 0 (or "auto") goes through fa_fwd_fp8_splitkv with that
     many key slices; the workspace is allocated here with torch unless
-    given (a uint8 CUDA tensor, 256-byte aligned)."""
+    given (a uint8 CUDA tensor, 256-byte aligned).  ``mask`` and
+    ``return_softmax_stats`` as in flash_fwd (through fa_fwd_fp8_ex; the
+    result is then (out, lse, softmax_max, softmax_sum))."""
     import torch
 
     B, H, L_q, D = q.shape
@@ -475,6 +492,28 @@ def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1
         lse = None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    if mask is not None or return_softmax_stats:
+        if n_splits:
+            raise ValueError("mask / softmax statistics are not available with n_splits")
+        mtype, sb, sh, sq = (FA_MASK_NONE, 0, 0, 0) if mask is None else \
+            mask_layout(mask, B, H, L_q, L_k)
+        if mask is not None and (not mask.is_cuda or mask.device != q.device):
+            raise ValueError("mask must be on q's device")
+        smax = ssum = None
+        if return_softmax_stats:
+            smax = torch.empty((B, H, L_q), dtype=torch.float32, device=q.device)
+            ssum = torch.empty_like(smax)
+        with torch.cuda.device(q.device):
+            st = fa_fwd_fp8_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr() if lse is not None else None,
+                               smax.data_ptr() if smax is not None else None,
+                               ssum.data_ptr() if ssum is not None else None,
+                               mask.data_ptr() if mask is not None else None, mtype, sb, sh, sq,
+                               B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k, descale_v,
+                               causal, window_left, window_right, stream.cuda_stream)
+        if st != FA_OK:
+            raise FaError(st, "fa_fwd_fp8_ex")
+        return out, lse, smax, ssum
     if n_splits == "auto":
         n_splits = choose_splits(B, H, L_q, L_k,
                                  torch.cuda.get_device_properties(q.device).multi_processor_count,

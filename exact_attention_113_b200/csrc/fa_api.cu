@@ -272,8 +272,6 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     if ((mx->smax == nullptr) != (mx->ssum == nullptr)) return FA_ERR_NULL;
     if (L_q > 0 && (!aligned(mx->smax, 4) || !aligned(mx->ssum, 4))) return FA_ERR_ALIGN;
   }
-  // fp8 inputs only through fa_fwd_fp8 / fa_fwd_fp8_splitkv: no mask
-  if (dtype == kE4M3 && masked) return FA_ERR_DTYPE;
   const int64_t rows_total = static_cast<int64_t>(B) * H * L_q;
   if (n_splits != 0) {
     if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
@@ -420,6 +418,9 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 66: st = launch<32, kE4M3, false>(prm, B, H, stream); break;
     case 130: st = launch<64, kE4M3, false>(prm, B, H, stream); break;
     case 258: st = launch<128, kE4M3, false>(prm, B, H, stream); break;
+    case 1066: st = launch<32, kE4M3, true>(prm, B, H, stream); break;
+    case 1130: st = launch<64, kE4M3, true>(prm, B, H, stream); break;
+    case 1258: st = launch<128, kE4M3, true>(prm, B, H, stream); break;
   }
   if (st != FA_OK || n_splits == 0) return st;
   switch (D * 2 + dtype) {
@@ -478,16 +479,17 @@ extern "C" int fa_fwd_ex(const void *q, const void *k, const void *v, void *out,
 
 namespace fa {
 namespace {
+// fp8 entries: descales checked and folded (q, k into the scores' scale; v
+// into the extras); `ex` carries fa_fwd_fp8_ex's mask and statistics.
 int fp8_impl(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
              int H_kv, int L_q, int L_k, int D, float scale, float descale_q, float descale_k,
              float descale_v, int causal, int window_left, int window_right, int n_splits,
-             void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+             void *workspace, size_t workspace_bytes, FwdExtras ex, cudaStream_t stream) {
   for (float d : {descale_q, descale_k, descale_v})
     if (!std::isfinite(d) || d < 0.0f) return FA_ERR_ARG;
   if (!std::isfinite(scale) || scale < 0.0f) return FA_ERR_ARG;
   const float s = scale * descale_q * descale_k;   // the scores' full scale
   if (!std::isfinite(s)) return FA_ERR_ARG;
-  FwdExtras ex;
   ex.descale_v = descale_v;
   return fwd_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, s, causal, window_left,
                   window_right, kE4M3, n_splits, workspace, workspace_bytes, &ex, stream);
@@ -500,7 +502,27 @@ extern "C" int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out
                           float descale_q, float descale_k, float descale_v, int causal,
                           int window_left, int window_right, cudaStream_t stream) {
   return fa::fp8_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
-                      descale_v, causal, window_left, window_right, 0, nullptr, 0, stream);
+                      descale_v, causal, window_left, window_right, 0, nullptr, 0,
+                      fa::FwdExtras{}, stream);
+}
+
+extern "C" int fa_fwd_fp8_ex(const void *q, const void *k, const void *v, void *out,
+                             float *lse, float *softmax_max, float *softmax_sum,
+                             const void *mask, int mask_type, long long mask_stride_b,
+                             long long mask_stride_h, long long mask_stride_q, int B, int H,
+                             int H_kv, int L_q, int L_k, int D, float scale, float descale_q,
+                             float descale_k, float descale_v, int causal, int window_left,
+                             int window_right, cudaStream_t stream) {
+  fa::FwdExtras mx;
+  mx.mask = mask;
+  mx.type = mask_type;
+  mx.sb = mask_stride_b;
+  mx.sh = mask_stride_h;
+  mx.sq = mask_stride_q;
+  mx.smax = softmax_max;
+  mx.ssum = softmax_sum;
+  return fa::fp8_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
+                      descale_v, causal, window_left, window_right, 0, nullptr, 0, mx, stream);
 }
 
 extern "C" int fa_fwd_fp8_splitkv(const void *q, const void *k, const void *v, void *out,
@@ -512,7 +534,7 @@ extern "C" int fa_fwd_fp8_splitkv(const void *q, const void *k, const void *v, v
   if (n_splits < 1 || n_splits > kMaxSplits) return FA_ERR_ARG;
   return fa::fp8_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
                       descale_v, causal, window_left, window_right, n_splits, workspace,
-                      workspace_bytes, stream);
+                      workspace_bytes, fa::FwdExtras{}, stream);
 }
 
 extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {

@@ -215,6 +215,20 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float
                    cudaStream_t stream);
 
 /*
+ * fa_fwd_fp8_ex -- fa_fwd_fp8 with fa_fwd_ex's optional attention mask and
+ * softmax statistics (same layouts and meaning; the mask's values are added
+ * to the full-scale scores scale * descale_q * descale_k * q_i . k_j, and
+ * softmax_max / softmax_sum refer to those scores).  Errors as fa_fwd_fp8
+ * and fa_fwd_ex.
+ */
+int fa_fwd_fp8_ex(const void *q, const void *k, const void *v, void *out, float *lse,
+                  float *softmax_max, float *softmax_sum, const void *mask, int mask_type,
+                  long long mask_stride_b, long long mask_stride_h, long long mask_stride_q,
+                  int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
+                  float descale_q, float descale_k, float descale_v, int causal,
+                  int window_left, int window_right, cudaStream_t stream);
+
+/*
  * fa_fwd_fp8_splitkv -- fa_fwd_fp8 computed in key slices as
  * fa_fwd_splitkv does (decoding over an fp8 key/value cache).  The slices'
  * partial outputs are fp32 in units of the V codes; the merge applies

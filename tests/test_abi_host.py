@@ -239,6 +239,24 @@ def test_fp8_argument_errors(lib, kw, code):
     assert _call_fp8(**kw) == code
 
 
+def _call_fp8_ex(mask=16, mtype=1, sb=0, sh=0, sq=8, smax=0, ssum=0, dq=1.0, dk=1.0, dv=1.0,
+                 **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_fp8_ex(a["q"], a["k"], a["v"], a["out"], a["lse"], smax, ssum, mask, mtype,
+                            sb, sh, sq, a["B"], a["H"], a["H_kv"], a["L_q"], a["L_k"], a["D"],
+                            a["scale"], dq, dk, dv, a["causal"], a["wl"], a["wr"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mtype=4), -6), (dict(sq=-1), -6), (dict(mask=0), -1), (dict(smax=16, ssum=0), -1),
+    (dict(smax=18, ssum=16), -5), (dict(D=48), -3), (dict(D=16), -3), (dict(dk=-2.0), -6),
+    (dict(q=8), -5),
+])
+def test_fp8_ex_argument_errors(lib, kw, code):
+    assert _call_fp8_ex(**kw) == code
+
+
 def test_16bit_entries_refuse_the_fp8_code(lib):
     # dtype 2 is internal to fa_fwd_fp8 / fa_fwd_fp8_splitkv
     assert _call(dtype=2) == -4

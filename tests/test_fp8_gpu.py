@@ -31,7 +31,7 @@ def _w(**kw):
     return Workload(**base)
 
 
-def check_fp8(w, descale=(1.0, 1.0, 1.0), n_splits=0):
+def check_fp8(w, descale=(1.0, 1.0, 1.0), n_splits=0, mask=None, stats=False):
     import exact_attention_113_b200 as fa
     dq, dk, dv = descale
     q, k, v = make_qkv_fp8(w)
@@ -42,15 +42,19 @@ def check_fp8(w, descale=(1.0, 1.0, 1.0), n_splits=0):
         nb = fa.fa_splitkv_workspace_bytes(w.B, w.H, w.L_q, w.D, n_splits)
         ws = torch.full((nb // 4,), float("nan"), dtype=torch.float32,
                         device="cuda").view(torch.uint8)
-    out, lse = fa.flash_fwd_fp8(qd, kd, vd, scale=w.softmax_scale, descale_q=dq, descale_k=dk,
-                                descale_v=dv, causal=w.causal, window_left=w.window_left,
-                                window_right=w.window_right, n_splits=n_splits, workspace=ws)
+    kw = {}
+    if mask is not None or stats:
+        kw = dict(mask=None if mask is None else mask.cuda(), return_softmax_stats=stats)
+    res = fa.flash_fwd_fp8(qd, kd, vd, scale=w.softmax_scale, descale_q=dq, descale_k=dk,
+                           descale_v=dv, causal=w.causal, window_left=w.window_left,
+                           window_right=w.window_right, n_splits=n_splits, workspace=ws, **kw)
+    out, lse = res[0], res[1]
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
     s_eff = w.softmax_scale * dq * dk
-    ref, ref_lse, _, ssum, wabs = oracle.attention_rows_ex(
+    ref, ref_lse, ref_max, ssum, wabs = oracle.attention_rows_ex(
         to_bits(q), to_bits(k), to_bits(v), E4M3, s_eff, w.causal, w.window_left,
-        w.window_right, with_wabs=True)
+        w.window_right, mask=None if mask is None else mask.numpy(), with_wabs=True)
     ref = ref * dv
     wabs = wabs * dv
     vabs = np.abs(v.float().double().numpy()).sum(axis=2) * dv       # [B, H_kv, D]
@@ -67,6 +71,14 @@ def check_fp8(w, descale=(1.0, 1.0, 1.0), n_splits=0):
     inf = np.isneginf(ref_lse)
     assert np.array_equal(np.isneginf(gl), inf)
     assert np.abs(gl[~inf] - ref_lse[~inf]).max(initial=0) <= 1e-3
+    if stats:
+        gm = res[2].cpu().numpy().reshape(-1).astype(np.float64)
+        gs = res[3].cpu().numpy().reshape(-1).astype(np.float64)
+        minf = np.isneginf(ref_max)
+        assert np.array_equal(np.isneginf(gm), minf)
+        assert np.all(gs[minf] == 0)
+        assert np.abs(gm[~minf] - ref_max[~minf]).max(initial=0) <= 1e-3
+        assert np.all(np.abs(gs[~minf] - ssum[~minf]) <= 1e-3 * ssum[~minf])
     return float(err.max())
 
 
@@ -140,3 +152,25 @@ def test_fp8_both_schedules(shape, causal, std):
     hw = dict(B=2, H=40, H_kv=40) if shape == "two" else dict(B=1, H=3, H_kv=3)
     check_fp8(_w(L_q=300, L_k=400, D=128, causal=causal, std=std,
                  seed=8900 + int(causal) + int(std), **hw))
+
+
+# ------------------------------------------------------------ mask and statistics
+# fa_fwd_fp8_ex: the 16-bit mask semantics on the full-scale fp8 scores.
+@pytest.mark.parametrize("shape", ["two", "one"])
+@pytest.mark.parametrize("D,kind", [(128, "bool"), (64, "f32"), (32, "f16")])
+def test_fp8_mask_and_stats(shape, D, kind):
+    from tests.test_mask_gpu import _mask
+    hw = dict(B=2, H=40, H_kv=40) if shape == "two" else dict(B=2, H=4, H_kv=2)
+    w = _w(L_q=300, L_k=333, D=D, seed=9600 + D, **hw)
+    check_fp8(w, descale=(0.5, 2.0, 0.25), mask=_mask((w.B, w.H, w.L_q, w.L_k), kind, 9700 + D),
+              stats=True)
+
+
+def test_fp8_broadcast_mask_with_causal():
+    from tests.test_mask_gpu import _mask
+    w = _w(B=2, H=4, H_kv=4, L_q=260, L_k=260, D=128, causal=True, seed=9800)
+    check_fp8(w, mask=_mask((1, 1, 1, w.L_k), "bool", 9801), stats=True)
+
+
+def test_fp8_stats_without_mask():
+    check_fp8(_w(L_q=200, L_k=500, D=64, seed=9900), stats=True)
