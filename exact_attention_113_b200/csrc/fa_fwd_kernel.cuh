@@ -47,6 +47,14 @@
 // softmax warpgroups competing for the exp unit cost more than the shorter
 // chain saves.)
 //
+// D <= 64, one query tile (kDual): the second softmax warpgroup would be
+// idle, so the two warpgroups split every block's keys: warpgroup h takes
+// keys [64h, 64h + 64) of S0 with its own running max and sum, its own P_h
+// (columns [384 + 64h, 416 + 64h)) and its own O_h (the O0 / O1 slots); the
+// MMA issuer runs S(j) once both hold S(j-1), then PV_0(j-1) and PV_1(j-1)
+// over the two key halves.  The epilogue merges the two (m, l, O) like two
+// key slices.
+//
 // D <= 64 (room to spare): P_t has its own columns [384 + 64t, 448 + 64t).
 // The softmax frees S_t as soon as it holds the row in registers and its
 // maximum (barrier s_free), so S_t(j+1) is computed while block j's
@@ -334,11 +342,13 @@ __device__ __forceinline__ void store_p_half(uint32_t base, int half, const uint
     tmem_st_x32(base + 32u * half, pk);
 }
 
-template <int D, int DT, bool kMask, bool kHalfS>
+template <int D, int DT, bool kMask, bool kHalfS, bool kDual = false>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 inputs (bf16 output).  kHalfS: the
-  // half-S schedule (D > 64, one query tile per CTA).
+  // half-S schedule (D > 64, one query tile per CTA).  kDual: one query
+  // tile, its keys split between the two softmax warpgroups (D <= 64).
   static_assert(!kHalfS || D > 64, "half-S schedule is for D > 64");
+  static_assert(!kDual || (D <= 64 && !kHalfS && DT != 2), "dual softmax is for 16-bit D <= 64");
   constexpr bool kF8 = DT == 2;
   constexpr int kES = kF8 ? 1 : 2;
   constexpr int kKStep = 32 / kES;             // K of one MMA instruction (32 bytes)
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       mbar_init(smem_u32(&bars->q_full[t]), 1);
       mbar_init(smem_u32(&bars->s_full[t]), 1);
       if (kHalfS) mbar_init(smem_u32(&bars->s_lo_full[t]), 1);
-      mbar_init(smem_u32(&bars->s_free[t]), kBM);
+      mbar_init(smem_u32(&bars->s_free[t]), (kDual && t == 0) ? 2 * kBM : kBM);
       mbar_init(smem_u32(&bars->p_full[t]), kBM);
       mbar_init(smem_u32(&bars->pv_done[t]), 1);
     }
@@ -569,7 +579,62 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       auto kpar = [&](int q) { return static_cast<uint32_t>((q / G::kSlotsK) & 1); };
       auto vpar = [&](int q) { return static_cast<uint32_t>((q / G::kSlotsV) & 1); };
 
-      if constexpr (G::kSplitP) {
+      if constexpr (kDual) {
+        // One query tile, two softmax warpgroups: S(j) once both hold
+        // S(j-1) in registers (s_free, 256 arrivals); then, once P_h(j-1)
+        // of half h (keys [64h, 64h + 64)) is in TMEM, O_h += P_h V_h into
+        // that half's own accumulator.
+        int ns = 0;
+        auto issue_pv_h = [&](int h, int slot) {
+          const uint32_t vlo = desc_lo(sRing + slot * G::kTileBytes, G::kBoxBytes);
+          const uint32_t a_tmem = tmem + 384u + (h ? 64u : 0u);
+          const uint32_t d_tmem = tmem + 256u + (h ? D : 0u);
+          const bool first = (h ? npv1 : npv0) == 0;
+          constexpr int kHalfSteps = kBN / kKStep / 2;
+          if (elect_one()) {
+#pragma unroll
+            for (int u = 0; u < kHalfSteps; ++u) {
+              const int kk = h * kHalfSteps + u;
+              mma_ts_t<kF8>(d_tmem, a_tmem + u * 8,
+                            desc_join(vlo + ((kk * kKStep * G::kSwBytes) >> 4), kHi), kIdescPV,
+                            (!first || u > 0) ? 1u : 0u);
+            }
+            tc_commit(smem_u32(&bars->pv_done[h]));
+          }
+          __syncwarp();
+          if (h) ++npv1; else ++npv0;
+        };
+        for (int j = lo; j <= hi && ok; ++j) {
+          const int q = j - lo;
+          if (j < hi) {
+            ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (ns > 0) {
+              ok = mbar_wait_warp(smem_u32(&bars->s_free[0]), (ns - 1) & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after_sync();
+            }
+            issue_s(0, kslot(q));
+            ++ns;
+            commit(smem_u32(&bars->empty[kslot(q)]));
+          }
+          if (j > lo) {
+            ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q - 1)]), vpar(q - 1), abort_flag);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              ok = ok && mbar_wait_warp(smem_u32(&bars->p_full[h]), (h ? npv1 : npv0) & 1,
+                                        abort_flag);
+              if (ok) {
+                tc_fence_after_sync();
+                issue_pv_h(h, vslot(q - 1));
+              }
+            }
+            if (!ok) break;
+            commit(smem_u32(&bars->empty[vslot(q - 1)]));
+          }
+        }
+      } else if constexpr (G::kSplitP) {
         // S0(j), S1(j), PV0(j-1), PV1(j-1): S_t(j) waits only until the
         // softmax of tile t holds S_t(j-1) in registers (s_free)
         int ns0 = 0, ns1 = 0;
@@ -722,15 +787,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   } else {
     // =================================================== softmax / epilogue
     regs_inc<RegSplit<D, DT, kHalfS>::kBig>();
-    const int t = warp >> 2;             // query tile of this warpgroup
+    // warpgroup t: the softmax of query tile t, or (kDual) of keys
+    // [64t, 64t + 64) of every block of tile 0
+    const int t = warp >> 2;
+    const int tt = kDual ? 0 : t;        // query tile of this warpgroup
     const int r = tid & 127;             // row within the tile = TMEM lane
     // this tile's scalars (selected, so that nothing is indexed at run time)
-    const int tq0 = t ? q0[1] : q0[0];
-    const int trows = t ? rows[1] : rows[0];
-    const int tlo = t ? rng[1].lo : rng[0].lo;
-    const int n_blocks = t ? rng[1].hi - rng[1].lo : rng[0].hi - rng[0].lo;
+    const int tq0 = tt ? q0[1] : q0[0];
+    const int trows = tt ? rows[1] : rows[0];
+    const int tlo = tt ? rng[1].lo : rng[0].lo;
+    const int n_blocks = tt ? rng[1].hi - rng[1].lo : rng[0].hi - rng[0].lo;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + t * 128u;
+    // S columns this warpgroup reads; O_t and P_t are its own (kDual: the
+    // second tile's slots hold the second key half's)
+    const uint32_t tS = tmem + lane_base + (kDual ? 64u * t : t * 128u);
     const uint32_t tO = tmem + lane_base + 256u + t * D;
     const uint32_t tPs = tmem + lane_base + 384u + t * 64u;   // split-P: P_t columns
     // packed tiles: row r is query position r % tile_q of head bh + r / tile_q
@@ -760,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       for (int n = 0; n < n_blocks; ++n) {
         const int j = tlo + n;
         ok = mbar_wait_warp(
-            smem_u32(kHalfS ? &bars->s_lo_full[t] : &bars->s_full[t]), n & 1, abort_flag);
+            smem_u32(kHalfS ? &bars->s_lo_full[t] : &bars->s_full[tt]), n & 1, abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
 
@@ -792,6 +862,80 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         };
         const float2 sl2v = make_float2(sl2, sl2);
 
+        // 64-key helpers of the half-S and dual schedules
+        float alpha = 1.0f;
+        bool rescaled = false;
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // 64 keys of the row from TMEM address taddr, key k0 first
+        auto load64 = [&](uint32_t taddr, int k0, float (&sv)[kBN / 2]) {
+          uint32_t sr[2][32];
+          tmem_ld_x32(taddr, sr[0]);
+          tmem_ld_x32(taddr + 32, sr[1]);
+          tmem_wait_ld();
+          reg_dep(sr[0]);
+          reg_dep(sr[1]);
+#pragma unroll
+          for (int c = 0; c < kBN / 2; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
+          if (!full) {
+            const int lo_c = row_lo - k0;
+            const int hi_c = row_hi - k0;
+#pragma unroll
+            for (int c = 0; c < kBN / 2; ++c)
+              if (c < lo_c || c > hi_c) sv[c] = -INFINITY;
+          }
+          if constexpr (kMask)
+            apply_mask(sv, p, mask_row + static_cast<long long>(k0), min(kBN / 2, p.L_k - k0),
+                       r_loc < trows, p.scale_log2);
+        };
+        // half maximum (four chains of 3-input maxima), in scaled log2 units
+        auto half_max = [&](const float (&sv)[kBN / 2]) -> float {
+          float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+          for (int c = 4; c < kBN / 2 - 4; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
+          const float m = fmax3(fmax3(mx[0], mx[1], sv[kBN / 2 - 4]),
+                                fmax3(mx[2], mx[3], sv[kBN / 2 - 3]),
+                                fmaxf(sv[kBN / 2 - 2], sv[kBN / 2 - 1]));
+          return m == -INFINITY ? -INFINITY : m * sl2;
+        };
+        // conditional rescale against a half's maximum; true if this warp
+        // moved its reference
+        auto raise = [&](float m_new) -> bool {
+          m_true = fmaxf(m_true, m_new);
+          if (!__any_sync(0xffffffffu, m_new > m_use + kRescaleThreshold)) return false;
+          const float m_upd = fmaxf(m_use, m_new);
+          const float a = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
+          m_use = m_upd;
+          l *= a;
+          alpha *= a;
+          rescaled = true;
+          return true;
+        };
+        auto exp_half = [&](const float (&sv)[kBN / 2], uint32_t (&pkh)[32], auto poly_ok) {
+          const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
+          const float2 negm = make_float2(-m_sub, -m_sub);
+#pragma unroll
+          for (int c = 0; c < kBN / 2; c += 2) {
+            const int pair = c >> 1;
+            const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2v, negm);
+            float2 pp;
+            if (decltype(poly_ok)::value && (pair % kPoly) == kPoly - 1)
+              pp = exp2_poly2(x);
+            else
+              pp = make_float2(ex2(x.x), ex2(x.y));
+            // l sums the unrounded fp32 weights
+            ls[pair & 1] = __fadd2_rn(ls[pair & 1], pp);
+            put_p<DT>(pkh, pair, pp.x, pp.y);
+          }
+        };
+        auto exp_any = [&](const float (&sv)[kBN / 2], uint32_t (&pkh)[32]) {
+          // masked entries are -inf: only MUFU's ex2 turns them into exact 0
+          if (full)
+            exp_half(sv, pkh, std::true_type{});
+          else
+            exp_half(sv, pkh, std::false_type{});
+        };
         // exact pass: the row max first (four chains of 3-input maxima), then
         // the conditional rescale, then P; used for masked blocks, the first
         // block of a row, and whenever the speculative pass is dropped
@@ -860,7 +1004,29 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           }
         };
 
-        if constexpr (G::kSplitP) {
+        if constexpr (kDual) {
+          // keys [64t, 64t + 64) of this block: max first, then free S (both
+          // warpgroups arrive) for the next block's S MMA, then P_t
+          float sv[kBN / 2];
+          load64(tS, j * kBN + 64 * t, sv);
+          const float m_half = half_max(sv);
+          tc_fence_before_sync();
+          mbar_arrive(smem_u32(&bars->s_free[0]));
+          raise(m_half);
+          uint32_t pk[32];
+          exp_any(sv, pk);
+          l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+          // P_t and O_t are read / written by PV_t(j-1): wait for it
+          if (n > 0) {
+            const bool got = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n - 1) & 1, abort_flag);
+            ok = ok && got;
+            tc_fence_after_sync();
+          }
+          if (ok) {
+            store_p_half<DT>(tPs, 0, pk);
+            if (rescaled && n > 0) scale_o_row<D>(tO, alpha);
+          }
+        } else if constexpr (G::kSplitP) {
           // row max first, then free S_t for the next block's S MMA, then P
           float s[kBN];
           load_s(s);
@@ -920,83 +1086,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           // its maximum first, then the conditional rescale, then P.  P_t is
           // stored over columns [64, 128) of S_t once both halves are in
           // registers; S_t is freed for the next block's first half then.
-          float alpha = 1.0f;
-          bool rescaled = false;
-          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
           uint32_t pk[2][32];
-          auto load_half = [&](int h, float (&sv)[kBN / 2]) {
-            uint32_t sr[2][32];
-            tmem_ld_x32(tS + 64 * h, sr[0]);
-            tmem_ld_x32(tS + 64 * h + 32, sr[1]);
-            tmem_wait_ld();
-            reg_dep(sr[0]);
-            reg_dep(sr[1]);
-#pragma unroll
-            for (int c = 0; c < kBN / 2; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
-            const int k0 = j * kBN + 64 * h;   // key of column 0
-            if (!full) {
-              const int lo_c = row_lo - k0;
-              const int hi_c = row_hi - k0;
-#pragma unroll
-              for (int c = 0; c < kBN / 2; ++c)
-                if (c < lo_c || c > hi_c) sv[c] = -INFINITY;
-            }
-            if constexpr (kMask)
-              apply_mask(sv, p, mask_row + static_cast<long long>(k0), min(kBN / 2, p.L_k - k0),
-                         r_loc < trows, p.scale_log2);
-          };
-          // half maximum (four chains of 3-input maxima), in scaled log2 units
-          auto half_max = [&](const float (&sv)[kBN / 2]) -> float {
-            float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
-#pragma unroll
-            for (int c = 4; c < kBN / 2 - 4; c += 8)
-#pragma unroll
-              for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], sv[c + 2 * u], sv[c + 2 * u + 1]);
-            const float m = fmax3(fmax3(mx[0], mx[1], sv[kBN / 2 - 4]),
-                                  fmax3(mx[2], mx[3], sv[kBN / 2 - 3]),
-                                  fmaxf(sv[kBN / 2 - 2], sv[kBN / 2 - 1]));
-            return m == -INFINITY ? -INFINITY : m * sl2;
-          };
-          // conditional rescale against a half's maximum; true if this warp
-          // moved its reference
-          auto raise = [&](float m_new) -> bool {
-            m_true = fmaxf(m_true, m_new);
-            if (!__any_sync(0xffffffffu, m_new > m_use + kRescaleThreshold)) return false;
-            const float m_upd = fmaxf(m_use, m_new);
-            const float a = (m_upd == -INFINITY) ? 1.0f : ex2(m_use - m_upd);
-            m_use = m_upd;
-            l *= a;
-            alpha *= a;
-            rescaled = true;
-            return true;
-          };
-          auto exp_half = [&](const float (&sv)[kBN / 2], uint32_t (&pkh)[32], auto poly_ok) {
-            const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
-            const float2 negm = make_float2(-m_sub, -m_sub);
-#pragma unroll
-            for (int c = 0; c < kBN / 2; c += 2) {
-              const int pair = c >> 1;
-              const float2 x = __ffma2_rn(make_float2(sv[c], sv[c + 1]), sl2v, negm);
-              float2 pp;
-              if (decltype(poly_ok)::value && (pair % kPoly) == kPoly - 1)
-                pp = exp2_poly2(x);
-              else
-                pp = make_float2(ex2(x.x), ex2(x.y));
-              // l sums the unrounded fp32 weights
-              ls[pair & 1] = __fadd2_rn(ls[pair & 1], pp);
-              put_p<DT>(pkh, pair, pp.x, pp.y);
-            }
-          };
-          auto exp_any = [&](const float (&sv)[kBN / 2], uint32_t (&pkh)[32]) {
-            // masked entries are -inf: only MUFU's ex2 turns them into exact 0
-            if (full)
-              exp_half(sv, pkh, std::true_type{});
-            else
-              exp_half(sv, pkh, std::false_type{});
-          };
           {
             float sv[kBN / 2];
-            load_half(0, sv);
+            load64(tS, j * kBN, sv);
             raise(half_max(sv));
             exp_any(sv, pk[0]);
           }
@@ -1007,12 +1100,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           tc_fence_after_sync();
           {
             float sv[kBN / 2];
-            load_half(1, sv);
+            load64(tS + 64, j * kBN + 64, sv);
             if (raise(half_max(sv))) {
               // the first half's P used the old reference: redo it from
               // S_t keys [0, 64), still in TMEM until s_free
               float s0[kBN / 2];
-              load_half(0, s0);
+              load64(tS, j * kBN, s0);
               ls[0] = ls[1] = make_float2(0.f, 0.f);
               exp_any(s0, pk[0]);
             }
@@ -1078,7 +1171,59 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         ok = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n_blocks - 1) & 1, abort_flag);
         if (ok) tc_fence_after_sync();
       }
-      if (p.ws_o != nullptr) {
+      // kDual: the two key halves are two slices of the row.  Warpgroup 1
+      // hands its (m, l, exact max) to warpgroup 0 through shared memory (Q
+      // tile 1's slot, unused with one tile); warpgroup 0 merges them, as
+      // the split-KV merge does, and writes the row: O = wa O_0 + wb O_1.
+      float wa = 1.0f, wb = 0.0f;
+      if constexpr (kDual) {
+        float *xch = reinterpret_cast<float *>(smem + G::kOffQ + G::kTileBytes);
+        if (t == 1) {
+          xch[r] = m_use;
+          xch[kBM + r] = l;
+          xch[2 * kBM + r] = m_true;
+          xch[3 * kBM + r] = ok ? 1.0f : 0.0f;
+        }
+        tc_fence_before_sync();
+        named_barrier_sync(3, 2 * kBM);
+        tc_fence_after_sync();
+        if (t == 0) {
+          const float mb = xch[r], lb = xch[kBM + r], tb = xch[2 * kBM + r];
+          ok = ok && xch[3 * kBM + r] != 0.0f;   // uniform: the same rows' warp
+          const float m = fmaxf(m_use, mb);
+          wa = (m_use == -INFINITY) ? 0.0f : ex2(m_use - m);
+          wb = (mb == -INFINITY) ? 0.0f : ex2(mb - m);
+          l = wa * l + wb * lb;
+          m_use = m;
+          m_true = fmaxf(m_true, tb);
+        }
+      }
+      // O row chunk (columns [c, c + W)) into registers; kDual: merged
+      auto load_o = [&](int c, auto wd, auto &o) {
+        constexpr int W = decltype(wd)::value;
+        if (n_blocks > 0) {
+          tmem_ld_cols<W>(tO + c, o);
+          if constexpr (kDual) {
+            uint32_t ob[W];
+            tmem_ld_cols<W>(tO + D + c, ob);
+            tmem_wait_ld();
+            reg_dep(o);
+            reg_dep(ob);
+#pragma unroll
+            for (int u = 0; u < W; ++u)
+              o[u] = __float_as_uint(wa * __uint_as_float(o[u]) + wb * __uint_as_float(ob[u]));
+          } else {
+            tmem_wait_ld();
+            reg_dep(o);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < W; ++u) o[u] = 0u;
+        }
+      };
+      if (kDual && t == 1) {
+        // warpgroup 1 is done: warpgroup 0 writes the row
+      } else if (p.ws_o != nullptr) {
         // split-KV partial: unnormalised O (fp32) and (m, l) of this slice.
         // tcgen05.ld is warp-collective: every lane loads (ok and n_blocks
         // are warp-uniform), only the lanes of real rows store.
@@ -1090,14 +1235,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           for_o_chunks<D>([&](int c, auto w) {
             constexpr int W = decltype(w)::value;
             uint32_t o[W];
-            if (n_blocks > 0) {
-              tmem_ld_cols<W>(tO + c, o);
-              tmem_wait_ld();
-              reg_dep(o);
-            } else {
-#pragma unroll
-              for (int u = 0; u < W; ++u) o[u] = 0u;
-            }
+            load_o(c, w, o);
             if (mine) {
 #pragma unroll
               for (int u = 0; u < W / 4; ++u)
@@ -1160,14 +1298,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         for_o_chunks<D>([&](int c, auto wd) {
           constexpr int W = decltype(wd)::value;
           uint32_t o[W];
-          if (n_blocks > 0) {
-            tmem_ld_cols<W>(tO + c, o);
-            tmem_wait_ld();
-            reg_dep(o);
-          } else {
-#pragma unroll
-            for (int u = 0; u < W; ++u) o[u] = 0u;
-          }
+          load_o(c, wd, o);
           uint32_t w[W / 2];
 #pragma unroll
           for (int u = 0; u < W / 2; ++u)

@@ -1,14 +1,17 @@
-"""Both forward schedules for head dims above 64, against the fp64 oracle.
+"""Both forward schedules of every head dim, against the fp64 oracle.
 
-At D > 64 the accumulators fill TMEM and the kernel has two schedules:
-  two query tiles per CTA that ping-pong on the tensor pipe, taken when the
-  problem has more 128-row query tiles than the GPU has SMs (148 on B200);
-  the half-S schedule, one tile per CTA, where S is computed in two 64-key
-  halves and P overwrites the second half, taken for fewer tiles than SMs
-  (short problems, decoding).
-The host picks by the tile count, so every case is sized on one side of that
-line: TWO = B 2 x H 40 at L_q 300 is 240 tiles (ping-pong), ONE = B 1 x H 3 is
-9 tiles (half-S).  Large-variance inputs (std 3: scaled scores of spread ~9,
+The host gives each CTA two query tiles when the problem has more 128-row
+tiles than the GPU has SMs (148 on B200), else one, and the kernel's
+schedule follows:
+  D > 64, two tiles: the tiles ping-pong on the tensor pipe;
+  D > 64, one tile: the half-S schedule (S in two 64-key halves, P over the
+  second half);
+  D <= 64, two tiles: decoupled P, both tiles' softmax warpgroups at once;
+  D <= 64, one tile: the dual softmax (the two warpgroups take the two key
+  halves of every block, each with its own running max, sum and O, merged
+  at the end).
+Every case is sized on one side of the tile-count line: TWO = B 2 x H 40 at
+L_q 300 is 240 tiles, ONE = B 1 x H 3 is 9 tiles.  Large-variance inputs (std 3: scaled scores of spread ~9,
 ~13 in log2 units) make the running maximum move past the rescale threshold
 inside blocks, including between a block's two halves, which is the rare
 path of the half-S softmax (P of the first half recomputed)."""
@@ -34,7 +37,7 @@ def _w(shape, **kw):
 
 
 @pytest.mark.parametrize("shape", ["two", "one"])
-@pytest.mark.parametrize("D", [80, 96, 112, 128])
+@pytest.mark.parametrize("D", [16, 32, 48, 64, 80, 96, 112, 128])
 @pytest.mark.parametrize("dtype", [F16, BF16])
 @pytest.mark.parametrize("causal", [False, True])
 def test_both_schedules(shape, D, dtype, causal):
@@ -43,7 +46,7 @@ def test_both_schedules(shape, D, dtype, causal):
 
 
 @pytest.mark.parametrize("shape", ["two", "one"])
-@pytest.mark.parametrize("D", [96, 128])
+@pytest.mark.parametrize("D", [32, 64, 96, 128])
 def test_rescale_heavy(shape, D):
     check_full(_w(shape, D=D, L_q=400, L_k=900, std=3.0, seed=9100 + D), derived=True)
 
@@ -56,12 +59,19 @@ def test_gqa_window(shape):
 
 
 @pytest.mark.parametrize("shape", ["two", "one"])
-@pytest.mark.parametrize("D,kind", [(128, "bool"), (96, "f32")])
+@pytest.mark.parametrize("D,kind", [(128, "bool"), (96, "f32"), (64, "f16"), (32, "bool")])
 def test_masked(shape, D, kind):
     w = _w(shape, D=D, L_k=333, seed=9300 + D)
     check_masked(w, _mask((w.B, w.H, w.L_q, w.L_k), kind, 9400 + D))
 
 
 @pytest.mark.parametrize("shape", ["two", "one"])
-def test_split_kv(shape):
-    check_full(_w(shape, L_q=300, L_k=1000, seed=9500), n_splits=3, derived=True)
+@pytest.mark.parametrize("D", [64, 128])
+def test_split_kv(shape, D):
+    check_full(_w(shape, L_q=300, L_k=1000, D=D, seed=9500 + D), n_splits=3, derived=True)
+
+
+@pytest.mark.parametrize("D", [16, 64])
+def test_gqa_window_small_head_dims(D):
+    check_full(_w("one", D=D, H=6, H_kv=3, L_q=500, L_k=700, causal=True, window_left=150,
+                  window_right=0, seed=9250 + D), derived=True)
