@@ -154,12 +154,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def code_hash(texts) -> str:
+    """sha256 (16 hex digits) of source texts with // comments, trailing
+    blanks and empty lines removed: a comment edit keeps the hash, any code
+    edit changes it."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for text in texts:
+        for line in text.splitlines():
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode("utf-8") + b"\n")
     return h.hexdigest()[:16]
+
+
+def kernel_source_hash() -> str:
+    """code_hash of the forward kernel's device code (the committed ncu
+    summary records the value its counters were taken on)."""
+    texts = []
+    for p in KERNEL_SOURCES:
+        with open(p, encoding="utf-8") as f:
+            texts.append(f.read())
+    return code_hash(texts)
 
 
 def profiled_traffic():

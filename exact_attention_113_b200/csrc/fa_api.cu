@@ -138,15 +138,15 @@ int launch_kernel(const FwdParams &prm, int B, int H, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// One query tile per CTA: D > 64 takes the half-S schedule, 16-bit D <= 64
-// the dual softmax (the tile's keys split between both softmax
-// warpgroups); everything else the kernel's default for its head dim.
+// One query tile per CTA: 16-bit inputs take the dual softmax (the tile's
+// keys split between both softmax warpgroups), fp8 at D > 64 the half-S
+// schedule; everything else the kernel's default for its head dim.
 template <int D, int DT, bool kMask>
 int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
-  if constexpr (D > 64) {
-    if (prm.tiles == 1) return launch_kernel<D, DT, kMask, true>(prm, B, H, stream);
-  } else if constexpr (DT != 2) {
+  if constexpr (DT != 2) {
     if (prm.tiles == 1) return launch_kernel<D, DT, kMask, false, true>(prm, B, H, stream);
+  } else if constexpr (D > 64) {
+    if (prm.tiles == 1) return launch_kernel<D, DT, kMask, true>(prm, B, H, stream);
   }
   return launch_kernel<D, DT, kMask, false>(prm, B, H, stream);
 }

@@ -34,9 +34,10 @@
 // PV_t(j), which reads P_t from the same TMEM columns; tcgen05 MMAs issued by
 // one thread execute in issue order.
 //
-// D > 64, one query tile (kHalfS; problems with fewer query tiles than SMs,
-// decoding): with no second tile to ping-pong with, S_t is computed in two
-// 64-key halves and P_t is written over the second half, columns [64, 128).
+// D > 64, one query tile, fp8 inputs (kHalfS; problems with fewer query
+// tiles than SMs, decoding): with no second tile to ping-pong with, S_t is
+// computed in two 64-key halves and P_t is written over the second half,
+// columns [64, 128).
 // Per block j the MMA issuer runs
 //   S_t(j) keys [0, 64)     once the softmax holds S_t(j-1) (s_free),
 //   PV_t(j-1)               once P_t(j-1) is in TMEM (p_full),
@@ -47,13 +48,13 @@
 // softmax warpgroups competing for the exp unit cost more than the shorter
 // chain saves.)
 //
-// D <= 64, one query tile (kDual): the second softmax warpgroup would be
-// idle, so the two warpgroups split every block's keys: warpgroup h takes
-// keys [64h, 64h + 64) of S0 with its own running max and sum, its own P_h
-// (columns [384 + 64h, 416 + 64h)) and its own O_h (the O0 / O1 slots); the
-// MMA issuer runs S(j) once both hold S(j-1), then PV_0(j-1) and PV_1(j-1)
-// over the two key halves.  The epilogue merges the two (m, l, O) like two
-// key slices.
+// One query tile, 16-bit inputs, any D (kDual): the second softmax
+// warpgroup would be idle, so the two warpgroups split every block's keys:
+// warpgroup h takes keys [64h, 64h + 64) of S0 with its own running max and
+// sum, its own P_h (columns [128 + 64h, 160 + 64h), S1's unused slot) and
+// its own O_h (the O0 / O1 slots); the MMA issuer runs S(j) once both hold
+// S(j-1), then PV_0(j-1) and PV_1(j-1) over the two key halves.  The
+// epilogue merges the two (m, l, O) like two key slices.
 //
 // D <= 64 (room to spare): P_t has its own columns [384 + 64t, 448 + 64t).
 // The softmax frees S_t as soon as it holds the row in registers and its
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   // half-S schedule (D > 64, one query tile per CTA).  kDual: one query
   // tile, its keys split between the two softmax warpgroups (D <= 64).
   static_assert(!kHalfS || D > 64, "half-S schedule is for D > 64");
-  static_assert(!kDual || (D <= 64 && !kHalfS && DT != 2), "dual softmax is for 16-bit D <= 64");
+  static_assert(!kDual || (!kHalfS && DT != 2), "dual softmax is for 16-bit inputs");
   constexpr bool kF8 = DT == 2;
   constexpr int kES = kF8 ? 1 : 2;
   constexpr int kKStep = 32 / kES;             // K of one MMA instruction (32 bytes)
@@ -587,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         int ns = 0;
         auto issue_pv_h = [&](int h, int slot) {
           const uint32_t vlo = desc_lo(sRing + slot * G::kTileBytes, G::kBoxBytes);
-          const uint32_t a_tmem = tmem + 384u + (h ? 64u : 0u);
+          const uint32_t a_tmem = tmem + 128u + (h ? 64u : 0u);   // P_h: S1's free slot
           const uint32_t d_tmem = tmem + 256u + (h ? D : 0u);
           const bool first = (h ? npv1 : npv0) == 0;
           constexpr int kHalfSteps = kBN / kKStep / 2;
@@ -802,11 +803,17 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     // second tile's slots hold the second key half's)
     const uint32_t tS = tmem + lane_base + (kDual ? 64u * t : t * 128u);
     const uint32_t tO = tmem + lane_base + 256u + t * D;
-    const uint32_t tPs = tmem + lane_base + 384u + t * 64u;   // split-P: P_t columns
+    // split-P: P_t columns; kDual: P_t of its key half in S1's free slot
+    const uint32_t tPs = tmem + lane_base + (kDual ? 128u : 384u) + t * 64u;
     // packed tiles: row r is query position r % tile_q of head bh + r / tile_q
     const int r_loc = p.packed ? (r & (p.tile_q - 1)) : r;
     const int row_head = p.packed ? bh + (r >> p.tile_q_shift) : bh;
     const int i = tq0 + r_loc;           // query index of this row
+    // One-tile schedules: a warp none of whose rows is a real query (short
+    // query ranges: decoding) skips its loads, exponentials and P stores but
+    // keeps every wait and arrival, so the barrier phases stay in step.
+    // Its P rows are never written; PV then fills O rows that no one stores.
+    const bool idle_warp = (kDual || kHalfS) && !__any_sync(0xffffffffu, r_loc < trows);
     const int row_lo = p.wl < 0 ? 0 : i - p.wl;
     const int row_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, i + p.wr);
     const int first = tq0, last = tq0 + trows - 1;
@@ -1004,7 +1011,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           }
         };
 
-        if constexpr (kDual) {
+        if (kDual && idle_warp) {
+          tc_fence_before_sync();
+          mbar_arrive(smem_u32(&bars->s_free[0]));
+          if (n > 0) {
+            const bool got = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n - 1) & 1, abort_flag);
+            ok = ok && got;
+          }
+        } else if (kHalfS && idle_warp) {
+          ok = mbar_wait_warp(smem_u32(&bars->s_full[t]), n & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after_sync();
+          tc_fence_before_sync();
+          mbar_arrive(smem_u32(&bars->s_free[t]));
+        } else if constexpr (kDual) {
           // keys [64t, 64t + 64) of this block: max first, then free S (both
           // warpgroups arrive) for the next block's S MMA, then P_t
           float sv[kBN / 2];
@@ -1201,7 +1221,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       // O row chunk (columns [c, c + W)) into registers; kDual: merged
       auto load_o = [&](int c, auto wd, auto &o) {
         constexpr int W = decltype(wd)::value;
-        if (n_blocks > 0) {
+        if (n_blocks > 0 && !idle_warp) {
           tmem_ld_cols<W>(tO + c, o);
           if constexpr (kDual) {
             uint32_t ob[W];

@@ -118,3 +118,12 @@ def test_exp_roof_closed_form():
     assert r["exps_per_launch"] == exps
     assert abs(r["achieved_per_clk_per_sm"] - round(exps / (1e-3 * 1e9 * 148), 3)) < 1e-9
     assert abs(r["frac"] - round(exps / (1e-3 * 1e9 * 148) / 16.0, 4)) < 1e-9
+
+
+def test_code_hash_ignores_comments_only():
+    a = "int f(int x) {  // doubles\n  return 2 * x;\n}\n"
+    b = "// a new header line\nint f(int x) {\n\n  return 2 * x;   // same code\n}\n"
+    c = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench.code_hash([a]) == bench.code_hash([b])
+    assert bench.code_hash([a]) != bench.code_hash([c])
+    assert len(bench.kernel_source_hash()) == 16

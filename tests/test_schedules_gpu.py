@@ -4,12 +4,12 @@ The host gives each CTA two query tiles when the problem has more 128-row
 tiles than the GPU has SMs (148 on B200), else one, and the kernel's
 schedule follows:
   D > 64, two tiles: the tiles ping-pong on the tensor pipe;
-  D > 64, one tile: the half-S schedule (S in two 64-key halves, P over the
-  second half);
   D <= 64, two tiles: decoupled P, both tiles' softmax warpgroups at once;
-  D <= 64, one tile: the dual softmax (the two warpgroups take the two key
+  one tile, any D: the dual softmax (the two warpgroups take the two key
   halves of every block, each with its own running max, sum and O, merged
-  at the end).
+  at the end); with one real query row in a warp's 32, the other warps
+  skip their exponentials.
+(fp8 one-tile D = 128 takes the half-S schedule; tests/test_fp8_gpu.py.)
 Every case is sized on one side of the tile-count line: TWO = B 2 x H 40 at
 L_q 300 is 240 tiles, ONE = B 1 x H 3 is 9 tiles.  Large-variance inputs (std 3: scaled scores of spread ~9,
 ~13 in log2 units) make the running maximum move past the rescale threshold
