@@ -95,6 +95,18 @@ def test_flash_fwd_rejects_bad_tensors(lib):
         fa.flash_fwd(q, q[:, :, :, :32], q)         # D mismatch
 
 
+def test_other_wrappers_reject_bad_tensors(lib):
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.float16)
+    c = torch.zeros(1, 2, 8, 64, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        fa.flash_fwd_fp8(q, q, q)                   # not E4M3 codes
+    with pytest.raises(ValueError):
+        fa.flash_fwd_fp8(c, c, c)                   # CPU tensors
+    with pytest.raises(TypeError):
+        fa.flash_fwd_host(q.float(), q.float(), q.float())
+
+
 # ------------------------------------------------------------ split-KV entry
 def _call_split(n_splits=2, ws=256, ws_bytes=None, **kw):
     a = dict(GOOD)
