@@ -10,7 +10,14 @@ The metric is forward TFLOPS with the pages' convention 4*B*H*L_q*L_k*D
 (halved when causal).  Timing: W untimed warm-up steps, then K steps timed
 with CUDA events on the launching stream, bracketed by a barrier and a
 device synchronise; the slowest rank's time counts.  The inputs (1.2 GB) are
-larger than the 126 MB L2, so no flush is needed between steps.
+larger than the 126 MB L2, so no flush is needed between steps; a workload
+whose inputs and outputs are smaller than twice the L2 gets 256 MiB written
+between its steps (outside the steps' events, whose times are summed).
+Clocks and throttle reasons are sampled through NVML every 10 ms during the
+timed steps.  `roofline.traffic` is read from the machine-written summary
+profiles/fa_fwd_kernel_roofline_b4h48l8192d128_dram.txt (an ncu capture of
+the DRAM byte counters on this workload, ingested with --ingest-ncu) while
+the kernel's code is unchanged since the capture.
 
 N > 1 (torchrun, one process per GPU, NCCL for the barrier and the max):
 every rank runs the same-sized problem on its own inputs (weak scaling; the
@@ -72,11 +79,17 @@ BWD_FLOP_FACTOR = 2.5      # backward: S, dP, dV, dK, dQ = 5 GEMMs vs the forwar
 MUFU_EX2_PER_CLK_SM = 16.0
 SM_COUNT = 148
 DEFAULT_WORKLOAD = W.ROOFLINE.name
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fa_fwd_roofline_b4h48l8192d128_ncu.md")
+# DRAM traffic of the forward kernel on the default workload: written by
+# `bench.py --ingest-ncu` from an ncu capture of that workload
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "fa_fwd_kernel_roofline_b4h48l8192d128_dram.txt")
+TRAFFIC_METRICS = ("dram__bytes_read.sum", "dram__bytes_write.sum")
 # the forward kernel's device code (the ncu summary is valid while it is
 # unchanged; the host-side launch code lives in fa_api.cu)
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_113_b200", "csrc", f)
                   for f in ("fa_fwd_kernel.cuh", "sm100.cuh")]
+L2_BYTES = 126 * 1024 * 1024
+L2_FLUSH_BELOW = 2 * L2_BYTES         # workloads smaller than this get an L2 flush
+L2_FLUSH_BYTES = 256 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -177,17 +190,71 @@ def kernel_source_hash() -> str:
     return code_hash(texts)
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the kernel sources as they are now (else None)."""
-    if not os.path.exists(PROFILE_SUMMARY):
+def profiled_traffic(path: str = TRAFFIC_SUMMARY):
+    """DRAM bytes per launch from the machine-written traffic summary, if it
+    was taken on the kernel sources as they are now (else None)."""
+    if not os.path.exists(path):
         return None
-    text = open(PROFILE_SUMMARY).read()
-    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    text = open(path).read()
+    m_hash = re.search(r"^kernel_source_hash:\s*([0-9a-f]+)", text, re.M)
+    m_bytes = re.search(r"^dram_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
     if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
         return None
     return float(m_bytes.group(1))
+
+
+_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+          "kibyte": 1024.0, "mibyte": 1024.0 ** 2, "gibyte": 1024.0 ** 3}
+
+
+def parse_ncu_metrics_csv(text: str, kernel_regex: str = "fa_fwd_kernel") -> dict:
+    """{launch id: {"kernel": name, metric: bytes}} from `ncu --csv
+    --metrics ...` output (one row per launch and metric)."""
+    import csv
+    import io
+    lines = [ln for ln in text.splitlines() if ln.startswith('"')]
+    rows = list(csv.reader(io.StringIO("\n".join(lines))))
+    if not rows:
+        return {}
+    head = rows[0]
+    col = {name: head.index(name) for name in ("ID", "Kernel Name", "Metric Name",
+                                               "Metric Unit", "Metric Value")}
+    out = {}
+    for r in rows[1:]:
+        if len(r) < len(head) or not re.search(kernel_regex, r[col["Kernel Name"]]):
+            continue
+        unit = r[col["Metric Unit"]].strip().lower()
+        val = float(r[col["Metric Value"]].replace(",", "")) * _UNITS.get(unit, 1.0)
+        d = out.setdefault(r[col["ID"]], {"kernel": r[col["Kernel Name"]]})
+        d[r[col["Metric Name"]]] = val
+    return out
+
+
+def ingest_ncu(csv_path: str, command: str, w: W.Workload, out_path: str = TRAFFIC_SUMMARY):
+    """Write the traffic summary that `roofline.traffic` reads from an ncu
+    capture of `TRAFFIC_METRICS` on workload ``w``."""
+    launches = parse_ncu_metrics_csv(open(csv_path, errors="replace").read())
+    launches = {k: v for k, v in launches.items() if all(m in v for m in TRAFFIC_METRICS)}
+    if not launches:
+        raise SystemExit(f"no fa_fwd_kernel launch with {TRAFFIC_METRICS} in {csv_path}")
+    rd = statistics.mean(v[TRAFFIC_METRICS[0]] for v in launches.values())
+    wr = statistics.mean(v[TRAFFIC_METRICS[1]] for v in launches.values())
+    kernels = sorted({v["kernel"] for v in launches.values()})
+    alg = min_hbm_bytes(w)
+    text = (f"# DRAM traffic of the forward kernel on the workload {w.name}\n"
+            f"# (machine-written by: python bench.py --ingest-ncu <csv> --workload {w.name})\n"
+            f"command: {command}\n"
+            f"kernel: {'; '.join(kernels)}\n"
+            f"kernel_source_hash: {kernel_source_hash()}\n"
+            f"launches_captured: {len(launches)}\n"
+            f"dram_bytes_read_per_launch: {rd:.6g}\n"
+            f"dram_bytes_write_per_launch: {wr:.6g}\n"
+            f"dram_bytes_per_launch: {rd + wr:.6g}\n"
+            f"algorithmic_bytes_per_launch: {alg:.6g}\n"
+            f"traffic_over_algorithmic: {(rd + wr) / alg:.4f}\n")
+    with open(out_path, "w") as f:
+        f.write(text)
+    print(text, end="")
 
 
 # ------------------------------------------------------------------ clocks
@@ -202,32 +269,88 @@ def physical_gpu_index(cuda_index: int) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock, power and throttle reasons sampled during the timed region.
+
+    Reads NVML (read-only queries, every 10 ms from a thread), so that even a
+    timed region of ~0.1 s gets several samples; falls back to `nvidia-smi
+    -lms 200` without NVML.  ``summary()`` counts only samples taken between
+    mark_start() and mark_end()."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, pci_bus_id: str | None = None, period_s: float = 0.01):
         self.gpu = gpu_index
+        self.pci = pci_bus_id
+        self.period = period_s
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.stop = threading.Event()
+        self.samples = []          # (time, sm_mhz, max_mhz, reasons set)
+        self.source = None
+        self.t0, self.t1 = -1e30, 1e30
+
+    # -- NVML
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.pci:
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(self.pci)
+            except pynvml.NVMLError:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll_nvml(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop.is_set():
+            ts = time.perf_counter()
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except nv.NVMLError:
+                break
+            self.samples.append((ts, sm, mx, {n for n, b in bits.items() if rs & b}))
+            self.stop.wait(self.period)
+
+    # -- nvidia-smi fallback
+    def _read_smi(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            rs = {n for n, v in zip(self.REASONS, parts[4:8]) if v.lower() == "active"}
+            self.samples.append((time.perf_counter(), sm, mx, rs))
 
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.source = "nvml, every %g ms" % (self.period * 1e3)
+            self.thread.start()
+            return self
+        except Exception:  # no NVML: sample with nvidia-smi instead
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
+            self.source = "nvidia-smi -lms 200"
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
         return self
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.perf_counter(), line.strip()))
 
     def mark_start(self):
         self.t0 = time.perf_counter()
@@ -236,37 +359,28 @@ class ClockSampler:
         self.t1 = time.perf_counter()
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self.thread is not None:
-                self.thread.join(timeout=5)
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        """Median SM clock and active throttle reasons over the samples that
-        arrived inside the marked (timed) window."""
-        sm, mx, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        t0, t1 = getattr(self, "t0", -1e30), getattr(self, "t1", 1e30)
-        for ts, line in self.lines:
-            if not t0 <= ts <= t1 + 0.25:
-                continue
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[4:8]):
-                if val.lower() == "active":
-                    reasons.add(name)
+        """Median SM clock and active throttle reasons over the samples taken
+        inside the marked (timed) window."""
+        inside = [s for s in self.samples if self.t0 <= s[0] <= self.t1]
+        sm = [s[1] for s in inside]
+        reasons = set()
+        for s in inside:
+            reasons |= s[3]
+        mx = inside[-1][2] if inside else (self.samples[-1][2] if self.samples else None)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_mhz_min": min(sm) if sm else None, "reasons": sorted(reasons),
+                "samples": len(sm), "source": self.source}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -361,13 +475,23 @@ def run_ours(args, w: W.Workload):
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with ClockSampler(physical_gpu_index(dev.index)) as clk:
-        time.sleep(0.5)                    # let the sampler start
+    # inputs and outputs that fit in L2 twice over: write a buffer larger than
+    # L2 between timed steps (outside their events); the step time is then the
+    # sum of the steps' own times
+    flush = None
+    if min_hbm_bytes(w, 1 if fp8 else 2) < L2_FLUSH_BELOW:
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    props = torch.cuda.get_device_properties(dev)
+    pci = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    with ClockSampler(physical_gpu_index(dev.index), pci) as clk:
+        time.sleep(0.3)                    # let the sampler start
         barrier(world, dev)
         torch.cuda.synchronize(dev)
         clk.mark_start()
         with torch.cuda.stream(stream):
             for s in range(args.steps):
+                if flush is not None:
+                    flush.fill_(float(s))
                 starts[s].record(stream)
                 step()
                 ends[s].record(stream)
@@ -375,7 +499,10 @@ def run_ours(args, w: W.Workload):
         clk.mark_end()
         barrier(world, dev)
     launch_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    total_s = starts[0].elapsed_time(ends[-1]) / 1e3
+    if flush is None:
+        total_s = starts[0].elapsed_time(ends[-1]) / 1e3
+    else:
+        total_s = sum(launch_ms) / 1e3
     if fa.fa_get_device_status(stream.cuda_stream) != 0:
         raise RuntimeError("device watchdog fired during the timed steps")
     max_total = max_over_ranks(total_s, world, dev)
@@ -401,6 +528,8 @@ def run_ours(args, w: W.Workload):
                     "peak_sustained": sustained,
                     "frac_of_sustained": round(achieved / sustained, 4),
                     "traffic": profiled_traffic() if w.name == W.ROOFLINE.name else None,
+                    "traffic_source": (os.path.relpath(TRAFFIC_SUMMARY, ROOT)
+                                       if w.name == W.ROOFLINE.name else None),
                     "peak_source": (f"{peak_kind} cuBLAS bf16 burst x 2 (nominal fp8 ratio)" if fp8
                                     else f"{peak_kind} cuBLAS bf16 burst (fp16 dense rate is the same)")}
     else:
@@ -417,8 +546,12 @@ def run_ours(args, w: W.Workload):
         roofline["timed"] = (f"whole step: split-KV launch ({n_splits} key slices) "
                              "plus merge launch")
     clocks = clk.summary()
+    if clocks.get("sm_mhz"):
+        clocks["ms_x_mhz"] = round(avg_launch_s * 1e3 * clocks["sm_mhz"], 1)
     exp_bound = exp_roof(w, avg_launch_s, clocks.get("sm_mhz") or clocks.get("sm_max_mhz"),
                          bwd)
+    exp_bound["clock"] = ("median SM clock sampled in the timed region" if clocks.get("sm_mhz")
+                          else "no sample in the timed region: the maximum SM clock")
 
     # ---- end to end through host buffers (pinned), rank-local
     e2e = None
@@ -491,7 +624,7 @@ def run_ours(args, w: W.Workload):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if fp8 else ("f16" if w.dtype == W.F16 else "bf16"),
         "data": "synthetic (seeded N(0,%g) inputs, per-rank seeds)" % w.std,
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, flush is not None),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "clocks": clocks, "gpu_launches": args.steps * launches_per_step,
         "exp_bound": exp_bound,
@@ -546,12 +679,14 @@ def min_hbm_bytes(w: W.Workload, in_bytes: int = 2) -> int:
     return (q + kv) * in_bytes + q * 2 + 4 * w.B * w.H * w.L_q
 
 
-def workload_config(w: W.Workload, world: int) -> dict:
+def workload_config(w: W.Workload, world: int, flushed: bool = False) -> dict:
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "L_q": w.L_q,
             "L_k": w.L_k, "D": w.D, "causal": w.causal, "window_left": w.window_left,
             "window_right": w.window_right, "scale": w.softmax_scale,
             "input_dtype": W.DTYPE_NAME[w.dtype], "accumulate": "fp32",
-            "l2": "inputs larger than L2 (no flush between steps)",
+            "l2": (f"L2 flushed between steps ({L2_FLUSH_BYTES >> 20} MiB written outside "
+                   "the steps' events)" if flushed
+                   else "inputs larger than L2 (no flush between steps)"),
             "parallelism": f"{world} independent replica(s), one per GPU"}
 
 
@@ -626,7 +761,15 @@ def main(argv=None):
                     help="CPU work in the cpu_baseline sample")
     ap.add_argument("--ref-step-seconds", type=float, default=4.0,
                     help="CPU work per step of --impl reference")
+    ap.add_argument("--ingest-ncu", metavar="CSV",
+                    help="write the DRAM traffic summary of the workload from an ncu "
+                         "--csv capture of dram__bytes_read.sum and dram__bytes_write.sum")
+    ap.add_argument("--ncu-command", default="",
+                    help="with --ingest-ncu: the command line that made the capture")
     args = ap.parse_args(argv)
+    if args.ingest_ncu:
+        ingest_ncu(args.ingest_ncu, args.ncu_command, W.ALL[args.workload])
+        return
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
     if args.sweep and args.impl == "ours":

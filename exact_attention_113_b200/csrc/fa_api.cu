@@ -927,21 +927,65 @@ namespace fa {
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+// The cached address belongs to the context the module was loaded in: a
+// device whose primary context is destroyed and made again (cudaDeviceReset)
+// reloads the module, possibly elsewhere, so the cache is keyed on the
+// context's unique id as well as the device.
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  void *addr;
+};
+ScratchSlot g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch on the current device, looked up on the
-// first call there and cached.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context, 0 if there is none or
+// the driver does not say.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch in the current device's context: looked
+// up with cudaGetSymbolAddress on the first call there (and again after the
+// context has been made anew), then cached.
 int static_scratch(void **addr) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_fa_static_scratch) != cudaSuccess || p == nullptr)
-      return FA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
   }
-  *addr = g_scratch_addr[dev];
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  const unsigned long long id = current_ctx_id();
+  if (id == 0 || g_scratch[dev].addr == nullptr || g_scratch[dev].ctx_id != id) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();   // leave no error behind for the caller's next check
+      return FA_ERR_CUDA;
+    }
+    // the lookup made the primary context current if none was: key on it
+    g_scratch[dev].ctx_id = current_ctx_id();
+    g_scratch[dev].addr = p;
+  }
+  *addr = g_scratch[dev].addr;
   return FA_OK;
 }
 }  // namespace

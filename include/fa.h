@@ -316,8 +316,10 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *out, cons
  * D = 128; lower n_splits to fit); other errors as fa_fwd_splitkv.
  *
  * Set-up: the first call on each device (with that device current) looks
- * up the scratch's device address once and caches it; make that first call
- * before any stream capture.  Nothing in the scratch has to start at zero:
+ * up the scratch's device address once and caches it, keyed on the device's
+ * context (a context made anew, e.g. after cudaDeviceReset, is looked up
+ * again on its first call); make that first call before any stream
+ * capture.  Nothing in the scratch has to start at zero:
  * every partial the merge reads is written earlier in the same call.
  * There is ONE scratch per device: calls whose work overlaps on the GPU
  * (different streams, or different host threads) race on it and corrupt

@@ -115,7 +115,7 @@ class Oracle:
         lib.oracle_attention_rows_ex.argtypes = [
             u16p, u16p, u16p, ctypes.c_int, i64, i64, i64, i64, i64, i64,
             ctypes.c_double, ctypes.c_int, i64, i64, ctypes.c_void_p, ctypes.c_int, i64, i64,
-            i64, i64p, i64, dp, dp, dp, dp, dp, ctypes.c_int]
+            i64, i64p, i64, dp, dp, dp, dp, dp, dp, ctypes.c_int]
         lib.oracle_attention_rows_ex.restype = ctypes.c_int
         lib.oracle_attention_f64.argtypes = [dp, dp, dp, i64, i64, i64, i64, i64, i64,
                                              ctypes.c_double, ctypes.c_int, i64, i64, dp, dp]
@@ -185,10 +185,17 @@ class Oracle:
     # ------------------------------------------------------------- attention
     def attention_rows(self, q, k, v, dtype, scale, causal=False,
                        window_left=-1, window_right=-1, rows=None,
-                       n_threads=0, with_wabs=False):
+                       n_threads=0, with_wabs=False, with_wrss=False):
         """Exact attention for flattened row ids r = (b*H + h)*L_q + i
         (None = every row).  Returns (out [n, D], lse [n], threads_used), or
-        (out, lse, threads_used, wabs [n, D]) with ``with_wabs``."""
+        (out, lse, threads_used, wabs [n, D]) with ``with_wabs``; with
+        ``with_wrss`` the error scales wabs and wrss [n, D] are appended
+        (out, lse, threads_used, wabs, wrss)."""
+        if with_wrss:
+            out, lse, _, _, wabs, wrss = self.attention_rows_ex(
+                q, k, v, dtype, scale, causal, window_left, window_right, rows=rows,
+                n_threads=n_threads, with_wabs=True, with_wrss=True)
+            return out, lse, 0, wabs, wrss
         q, k, v, B, H, H_kv, L_q, L_k, D = _shape_args(q, k, v)
         if rows is None:
             n, rows_p = B * H * L_q, None
@@ -271,10 +278,11 @@ class Oracle:
 
     def attention_rows_ex(self, q, k, v, dtype, scale, causal=False, window_left=-1,
                           window_right=-1, mask=None, rows=None, n_threads=0,
-                          with_wabs=False):
+                          with_wabs=False, with_wrss=False):
         """Exact attention with an optional mask (see attention_ref.c for
         its reading); returns (out [n, D], lse, softmax_max, softmax_sum),
-        plus wabs [n, D] with ``with_wabs``."""
+        plus wabs [n, D] with ``with_wabs`` and then wrss [n, D] with
+        ``with_wrss`` (the two error scales stated in attention_ref.c)."""
         q, k, v, B, H, H_kv, L_q, L_k, D = _shape_args(q, k, v)
         m, mtype, sb, sh, sq = self.mask_args(mask, B, H, L_q, L_k)
         if rows is None:
@@ -284,6 +292,7 @@ class Oracle:
             n, rows_p = rows.size, _ptr(rows, ctypes.c_int64)
         out = np.zeros((n, D), dtype=np.float64)
         wabs = np.zeros((n, D), dtype=np.float64) if with_wabs else None
+        wrss = np.zeros((n, D), dtype=np.float64) if with_wrss else None
         lse, smax, ssum = (np.zeros((n,), dtype=np.float64) for _ in range(3))
         rc = self.lib.oracle_attention_rows_ex(
             _ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
@@ -292,12 +301,16 @@ class Oracle:
             m.ctypes.data_as(ctypes.c_void_p) if m is not None else None, mtype, sb, sh, sq,
             rows_p, n, _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
             _ptr(wabs, ctypes.c_double) if with_wabs else None,
+            _ptr(wrss, ctypes.c_double) if with_wrss else None,
             _ptr(smax, ctypes.c_double), _ptr(ssum, ctypes.c_double), int(n_threads))
         if rc < 0:
             raise ValueError("oracle rejected the arguments")
+        res = (out, lse, smax, ssum)
         if with_wabs:
-            return out, lse, smax, ssum, wabs
-        return out, lse, smax, ssum
+            res = res + (wabs,)
+        if with_wrss:
+            res = res + (wrss,)
+        return res
 
     # ------------------------------------------------------------- fp64 inputs
     @staticmethod

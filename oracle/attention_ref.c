@@ -248,6 +248,12 @@ static double mask_value(const void *mask, int mask_type, int64_t idx, int *hidd
  *          it is the scale of the error that rounding the weights p_j to a
  *          t-bit format causes in O (at most 2^-t * wabs per element, first
  *          order), which the parity tests use in their tolerance.
+ *   wrss : [n_rows, D] fp64 (may be NULL): sqrt(sum_j p_j^2 v_j[d]^2), the
+ *          root of the sum of squares of the same terms.  Also not part of
+ *          the result: when the rounding errors of the weights are
+ *          independent, their effect on O[d] has a standard deviation of
+ *          at most 2^-t / sqrt(3) * wrss, which the parity tests use for a
+ *          tolerance that does not grow with the number of keys.
  *   mask, mask_type, stride_b/h/q : the optional mask (type 0 = none),
  *          read as stated above mask_value();
  *   smax, ssum : [n_rows] fp64 (may be NULL): softmax_max, softmax_sum.
@@ -262,7 +268,7 @@ static int rows_core(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const void *mask, int mask_type, int64_t stride_b,
                      int64_t stride_h, int64_t stride_q, const int64_t *rows,
                      int64_t n_rows, double *out, double *lse, double *wabs,
-                     double *smax, double *ssum, int n_threads)
+                     double *wrss, double *smax, double *ssum, int n_threads)
 {
     if (B < 1 || H < 1 || H_kv < 1 || L_q < 0 || L_k < 0 || D < 1)
         return -1;
@@ -342,6 +348,20 @@ static int rows_core(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         w[d] += p[j] * fabs(tab[vp[j * D + d]]);
                 }
             }
+            if (wrss) {
+                double *w = wrss + t * D;
+                for (int64_t d = 0; d < D; d++)
+                    w[d] = 0.0;
+                for (int64_t j = 0; j < L_k; j++) {
+                    if (p[j] == 0.0) continue;
+                    for (int64_t d = 0; d < D; d++) {
+                        const double term = p[j] * tab[vp[j * D + d]];
+                        w[d] += term * term;
+                    }
+                }
+                for (int64_t d = 0; d < D; d++)
+                    w[d] = sqrt(w[d]);
+            }
         }
         free(qrow);
         free(s);
@@ -361,11 +381,11 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k,
 {
     return rows_core(q, k, v, dtype, B, H, H_kv, L_q, L_k, D, scale, causal,
                      window_left, window_right, NULL, 0, 0, 0, 0, rows, n_rows,
-                     out, lse, wabs, NULL, NULL, n_threads);
+                     out, lse, wabs, NULL, NULL, NULL, n_threads);
 }
 
-/* The same with a mask and the two softmax statistics (wabs, smax, ssum
- * nullable), as stated above the mask helpers. */
+/* The same with a mask and the two softmax statistics (wabs, wrss, smax,
+ * ssum nullable), as stated above the mask helpers. */
 int oracle_attention_rows_ex(const uint16_t *q, const uint16_t *k,
                              const uint16_t *v, int dtype, int64_t B, int64_t H,
                              int64_t H_kv, int64_t L_q, int64_t L_k, int64_t D,
@@ -374,13 +394,13 @@ int oracle_attention_rows_ex(const uint16_t *q, const uint16_t *k,
                              int mask_type, int64_t stride_b, int64_t stride_h,
                              int64_t stride_q, const int64_t *rows,
                              int64_t n_rows, double *out, double *lse,
-                             double *wabs, double *smax, double *ssum,
-                             int n_threads)
+                             double *wabs, double *wrss, double *smax,
+                             double *ssum, int n_threads)
 {
     return rows_core(q, k, v, dtype, B, H, H_kv, L_q, L_k, D, scale, causal,
                      window_left, window_right, mask, mask_type, stride_b,
-                     stride_h, stride_q, rows, n_rows, out, lse, wabs, smax,
-                     ssum, n_threads);
+                     stride_h, stride_q, rows, n_rows, out, lse, wabs, wrss,
+                     smax, ssum, n_threads);
 }
 
 /*

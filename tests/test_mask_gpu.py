@@ -6,8 +6,9 @@ scores), full [B, H, L_q, L_k] or broadcast ([L_q, L_k], key padding
 [B, 1, 1, L_k], per-head [1, H, 1, L_k]), with and without the causal /
 window rule, aligned (16-byte vector loads) and unaligned strides.
 
-Gate: O as the plain forward's derived gate (3e-3 + ulp/2 + 2u * wabs: a
-random mask leaves some rows a handful of keys); lse, softmax_max within
+Gate: O as the plain forward's derived gate (3e-3 + ulp/2 + P's rounding
+term, min(u wabs, 8 sigma_P): a random mask leaves some rows a handful of
+keys) and the aggregate check of tests/parity.py; lse, softmax_max within
 1e-3 (both log-domain quantities); softmax_sum within a relative 1e-3 (its
 log is lse - softmax_max)."""
 from __future__ import annotations
@@ -18,7 +19,7 @@ import torch
 
 import oracle
 from exact_attention_113_b200.inputs import BF16, F16, Workload, make_qkv, to_bits
-from tests.parity import compare
+from tests.parity import compare, reference
 
 pytestmark = pytest.mark.gpu
 
@@ -51,11 +52,9 @@ def check_masked(w, mask, stats=True):
     torch.cuda.synchronize()
     assert fa.fa_get_device_status() == 0
     mnp = None if mask is None else mask.numpy()
-    ref, ref_lse, ref_max, ref_sum, wabs = oracle.attention_rows_ex(
-        to_bits(q), to_bits(k), to_bits(v), w.dtype, w.softmax_scale, w.causal, w.window_left,
-        w.window_right, mask=mnp, with_wabs=True)
+    ref, ref_lse, pr, heads, ref_max, ref_sum = reference(w, q, k, v, mask=mnp, stats=True)
     compare(out.float().cpu().numpy().reshape(-1, w.D), lse.cpu().numpy().reshape(-1), ref,
-            ref_lse, w.dtype, w.name, wabs)
+            ref_lse, w.dtype, w.name, pr, True, heads)
     if stats:
         gm = smax.cpu().numpy().reshape(-1).astype(np.float64)
         gs = ssum.cpu().numpy().reshape(-1).astype(np.float64)

@@ -41,6 +41,9 @@ MUTATIONS = {
                         "double r = round(ldexp(a, -q_exp));"),
     "wabs_signed": ("w[d] += p[j] * fabs(tab[vp[j * D + d]]);",
                     "w[d] += p[j] * tab[vp[j * D + d]];"),
+    "wrss_no_root": ("                    w[d] = sqrt(w[d]);", "                    w[d] = w[d];"),
+    "wrss_weight_not_squared": ("const double term = p[j] * tab[vp[j * D + d]];\n                        w[d] += term * term;",
+                                "const double term = tab[vp[j * D + d]];\n                        w[d] += p[j] * term * term;"),
     "online_stale_max": ("d = d * exp(m - m_new) + exp(x[i] - m_new);",
                          "d = d + exp(x[i] - m_new);"),
     # backward
@@ -97,6 +100,7 @@ def _battery(orc):
     yield lambda: pins.test_shifting_every_key(orc)
     yield lambda: pins.test_fully_masked_rows(orc)
     yield lambda: pins.test_weighted_abs_value_closed_forms(orc)
+    yield lambda: pins.test_weighted_rss_closed_forms(orc)
     for c in bwd_pins.CASES:
         yield lambda c=c: bwd_pins.test_finite_differences_of_the_forward(orc, c)
         yield lambda c=c: bwd_pins.test_matches_torch_fp64_autograd(orc, c)

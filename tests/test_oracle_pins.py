@@ -172,6 +172,7 @@ def _brute(qf, kf, vf, scale, causal, wl, wr):
     out = np.zeros((B, H, L_q, D))
     lse = np.zeros((B, H, L_q))
     wabs = np.zeros((B, H, L_q, D))
+    wrss = np.zeros((B, H, L_q, D))
     for b in range(B):
         for h in range(H):
             g = h // grp
@@ -194,8 +195,11 @@ def _brute(qf, kf, vf, scale, causal, wl, wr):
                     wabs[b, h, i, d] = math.fsum(
                         math.exp(t - m) / den * abs(float(vf[b, g, j, d]))
                         for j, t in s)
+                    wrss[b, h, i, d] = math.sqrt(math.fsum(
+                        (math.exp(t - m) / den * float(vf[b, g, j, d])) ** 2
+                        for j, t in s))
                 lse[b, h, i] = m + math.log(den)
-    return out, lse, wabs
+    return out, lse, wabs, wrss
 
 
 BRUTE_CASES = [
@@ -219,12 +223,16 @@ def test_matches_brute_force(orc, case):
     v = _rand_bits((B, H_kv, L_k, D), dtype, 13)
     scale = 1.0 / math.sqrt(D)
     out, lse = orc.attention(q, k, v, dtype, scale, causal, wl, wr)
-    ro, rl, rw = _brute(_lib_decode(q, dtype), _lib_decode(k, dtype),
-                        _lib_decode(v, dtype), scale, causal, wl, wr)
+    ro, rl, rw, rr = _brute(_lib_decode(q, dtype), _lib_decode(k, dtype),
+                            _lib_decode(v, dtype), scale, causal, wl, wr)
     assert np.allclose(out, ro, rtol=0, atol=1e-12)
     _, _, _, wabs = orc.attention_rows(q, k, v, dtype, scale, causal, wl, wr,
                                        with_wabs=True)
     assert np.allclose(wabs, rw.reshape(wabs.shape), rtol=0, atol=1e-12)
+    _, _, _, wabs2, wrss = orc.attention_rows(q, k, v, dtype, scale, causal, wl, wr,
+                                              with_wrss=True)
+    assert np.array_equal(wabs2, wabs)
+    assert np.allclose(wrss, rr.reshape(wrss.shape), rtol=0, atol=1e-12)
     inf = np.isinf(rl)
     assert np.array_equal(np.isinf(lse), inf)
     assert np.allclose(lse[~inf], rl[~inf], rtol=0, atol=1e-12)
@@ -310,6 +318,30 @@ def test_weighted_abs_value_closed_forms(orc):
     _, _, _, w1 = orc.attention_rows(q, k1, v1, F16, 0.3, False, with_wabs=True)
     assert np.array_equal(w1.reshape(B, H, L, D),
                           np.broadcast_to(np.abs(_lib_decode(v1, F16)), (B, H, L, D)))
+
+
+def test_weighted_rss_closed_forms(orc):
+    # K = 0: every visible key weighs 1/n, so wrss = sqrt(sum_vis v^2) / n;
+    # one key: wrss = |v_0|; wrss <= wabs <= sqrt(n) * wrss (Cauchy-Schwarz)
+    B, H, L, D = 1, 2, 11, 4
+    q = _rand_bits((B, H, L, D), BF16, 151)
+    k = _const_bits((B, H, L, D), 0.0, BF16)
+    v = _rand_bits((B, H, L, D), BF16, 152)
+    vf = _lib_decode(v, BF16)
+    _, _, _, wabs, wrss = orc.attention_rows(q, k, v, BF16, 0.7, True, 3, -1, with_wrss=True)
+    wrss = wrss.reshape(B, H, L, D)
+    wabs = wabs.reshape(B, H, L, D)
+    for i in range(L):
+        lo = max(0, i - 3)
+        n = i - lo + 1
+        want = np.sqrt((vf[:, :, lo:i + 1] ** 2).sum(axis=2)) / n
+        assert np.allclose(wrss[:, :, i], want, rtol=1e-14, atol=0)
+        assert np.all(wrss[:, :, i] <= wabs[:, :, i] * (1 + 1e-14))
+        assert np.all(wabs[:, :, i] <= np.sqrt(n) * wrss[:, :, i] * (1 + 1e-14))
+    k1, v1 = _rand_bits((B, H, 1, D), BF16, 153), _rand_bits((B, H, 1, D), BF16, 154)
+    _, _, _, _, w1 = orc.attention_rows(q, k1, v1, BF16, 0.3, False, with_wrss=True)
+    assert np.array_equal(w1.reshape(B, H, L, D),
+                          np.broadcast_to(np.abs(_lib_decode(v1, BF16)), (B, H, L, D)))
 
 
 def test_single_key_is_v0(orc):
