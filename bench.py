@@ -432,7 +432,7 @@ def run_ours(args, w: W.Workload):
     lse = torch.empty((w.B, w.H, w.L_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     bwd = args.pass_ == "bwd"
-    n_splits = 0 if bwd else resolve_splits(args.splits, w)
+    n_splits = 0 if bwd else resolve_splits(args.splits, w, fp8)
     ws = None
     if n_splits:
         ws = torch.empty(fa.fa_splitkv_workspace_bytes(w.B, w.H, w.L_q, w.D, n_splits),
@@ -655,11 +655,12 @@ def exp_roof(w: W.Workload, launch_s: float, sm_mhz, bwd: bool = False) -> dict:
             "note": "backward: P recomputed once" if bwd else "forward"}
 
 
-def resolve_splits(arg: str, w: W.Workload, sm_count: int = 148) -> int:
+def resolve_splits(arg: str, w: W.Workload, fp8: bool = False) -> int:
     """--splits: 0 (fa_fwd), an explicit slice count, or auto."""
     if arg == "auto":
         from exact_attention_113_b200.binding import choose_splits
-        return choose_splits(w.B, w.H, w.L_q, w.L_k, sm_count, H_kv=w.H_kv)
+        return choose_splits(w.B, w.H, w.L_q, w.L_k, H_kv=w.H_kv, D=w.D,
+                             dtype=2 if fp8 else w.dtype)
     return int(arg)
 
 

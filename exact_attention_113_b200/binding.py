@@ -28,7 +28,8 @@ EXPORTS = ("fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_bytes", "fa_fwd", "fa_fwd_ex
            "fa_fwd_fp8_ex", "fa_fwd_fp8_splitkv",
            "fa_fwd_host", "fa_fwd_host_workspace_bytes", "fa_fwd_splitkv",
            "fa_fwd_splitkv_static", "fa_get_device_status", "fa_selftest_wait_timeout",
-           "fa_splitkv_workspace_bytes", "fa_status_string", "fa_version")
+           "fa_splitkv_auto_splits", "fa_splitkv_workspace_bytes", "fa_status_string",
+           "fa_version")
 # size of the library's static split-KV scratch (FA_STATIC_SCRATCH_BYTES)
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -95,6 +96,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.fa_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
+        lib.fa_splitkv_auto_splits.argtypes = [i, i, i, i, i, i, i]
+        lib.fa_splitkv_auto_splits.restype = i
         lib.fa_get_device_status.argtypes = [vp]
         lib.fa_get_device_status.restype = i
         lib.fa_selftest_wait_timeout.argtypes = [vp, vp]
@@ -245,22 +248,12 @@ def query_tiles(B, H, H_kv, L_q) -> int:
     return B * H * max(1, -(-L_q // 128))
 
 
-def choose_splits(B, H, L_q, L_k, sm_count=148, H_kv=None) -> int:
-    """Key slices for fa_fwd_splitkv (1..64, at least two 128-key blocks per
-    slice) minimising a cost model fitted to B200 decode timings: a CTA costs
-    about 4.5 key blocks of fixed work (set-up, pipeline fill, epilogue) plus
-    its blocks, and CTAs run in waves of ``sm_count`` (one per SM)."""
-    tiles = query_tiles(B, H, H if H_kv is None else H_kv, L_q)
-    blocks = max(1, -(-L_k // 128))
-    best, best_cost = 1, None
-    for sp in range(1, 65):
-        per = -(-blocks // sp)
-        if sp > 1 and per < 2:
-            break
-        cost = -(-tiles * sp // sm_count) * (4.5 + per)
-        if best_cost is None or cost < best_cost:
-            best, best_cost = sp, cost
-    return best
+def choose_splits(B, H, L_q, L_k, sm_count=None, H_kv=None, D=128, dtype=FA_F16) -> int:
+    """Key slices for fa_fwd_splitkv: the library's own choice
+    (fa_splitkv_auto_splits, on the current device; ``sm_count`` is not
+    used, the device's count is).  dtype 2 = E4M3 inputs."""
+    return int(load().fa_splitkv_auto_splits(B, H, H if H_kv is None else H_kv, L_q, L_k, D,
+                                             dtype))
 
 
 def fa_get_device_status(stream=None) -> int:
@@ -372,9 +365,8 @@ def flash_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1
             raise FaError(st, "fa_fwd_ex")
         return out, lse, smax, ssum
     if n_splits == "auto":
-        n_splits = choose_splits(B, H, L_q, L_k,
-                                 torch.cuda.get_device_properties(q.device).multi_processor_count,
-                                 H_kv=H_kv)
+        with torch.cuda.device(q.device):
+            n_splits = choose_splits(B, H, L_q, L_k, H_kv=H_kv, D=D, dtype=dtype)
     with torch.cuda.device(q.device):
         if not n_splits:
             st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
@@ -515,9 +507,8 @@ def flash_fwd_fp8(q, k, v, scale=None, descale_q=1.0, descale_k=1.0, descale_v=1
             raise FaError(st, "fa_fwd_fp8_ex")
         return out, lse, smax, ssum
     if n_splits == "auto":
-        n_splits = choose_splits(B, H, L_q, L_k,
-                                 torch.cuda.get_device_properties(q.device).multi_processor_count,
-                                 H_kv=H_kv)
+        with torch.cuda.device(q.device):
+            n_splits = choose_splits(B, H, L_q, L_k, H_kv=H_kv, D=D, dtype=2)
     with torch.cuda.device(q.device):
         if not n_splits:
             st = fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),

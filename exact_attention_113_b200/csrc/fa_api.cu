@@ -18,6 +18,7 @@
 #include "fa.h"
 #include "fa_fwd_kernel.cuh"
 #include "fa_bwd_kernel.cuh"
+#include "fa_decode_kernel.cuh"
 
 namespace fa {
 namespace {
@@ -221,6 +222,85 @@ int launch_combine(const float *ws_o, const float2 *ws_ml, void *out, float *lse
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- decoding
+// Problems with at most kDecMaxRows query rows per K/V head (decoding: one
+// new token per head, or a GQA group's few heads, against a long cache) run
+// on the CUDA-core decode kernel (fa_decode_kernel.cuh) instead of the
+// tensor-core kernel, whose 128-row tiles would hold one real row.
+constexpr int kDecMaxRows = 2;
+
+bool decode_eligible(int D, int dtype, int64_t rows_per_kv_head) {
+  if (rows_per_kv_head < 1 || rows_per_kv_head > kDecMaxRows) return false;
+  if (dtype == 2) return D == 32 || D == 64 || D == 128;
+  return D == 16 || D == 32 || D == 64 || D == 128;
+}
+
+int sm_count() {
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    return sms;
+  cudaGetLastError();
+  return 148;
+}
+
+template <int D, int DT, int R>
+int launch_decode_kernel(const DecParams &prm, unsigned grid, cudaStream_t stream) {
+  using G = DecGeo<D, DT == 2 ? 1 : 2>;
+  auto kern = fa_decode_kernel<D, DT, R>;
+  const int smem = G::kStages * G::kStageBytes + kDecWarps * R * D * 4 + kDecWarps * R * 8 +
+                   2 * G::kStages * 8 + 16;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  static bool configured[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    if (!configured[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return FA_ERR_CUDA;
+      configured[dev] = true;
+    }
+  }
+  kern<<<grid, kDecThreads, smem, stream>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, int DT>
+int launch_decode(const DecParams &prm, unsigned grid, cudaStream_t stream) {
+  if (prm.rows <= 1) return launch_decode_kernel<D, DT, 1>(prm, grid, stream);
+  return launch_decode_kernel<D, DT, 2>(prm, grid, stream);
+}
+
+// Keys a CTA of the decode kernel should get at least (two chunks), so that
+// its fixed work (set-up, the first copies' latency, the merge) stays small.
+constexpr int64_t kDecMinKeysPerCta = 2 * kDecChunk;
+
+// Grid of the decode kernel.  One slot per row: one CTA per K/V head (at
+// most one per SM; heads taken with a stride).  n_splits >= 2 slots: the
+// flattened (head, key) space of U = heads * key_span keys in G equal
+// ranges, each at least ceil(key_span / (n_splits - 1)) keys long (and at
+// least kDecMinKeysPerCta), so that one head's key_span keys meet at most
+// (n_splits - 1) + 1 ranges: no head needs more slots than it has.
+unsigned decode_grid(int64_t heads, int64_t key_span, int n_splits, int sms) {
+  if (n_splits <= 1) return static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(heads, sms)));
+  const int64_t per_min = std::max<int64_t>((key_span + n_splits - 2) / (n_splits - 1),
+                                            kDecMinKeysPerCta);
+  const int64_t g = std::min<int64_t>(sms, heads * key_span / per_min);
+  return static_cast<unsigned>(std::max<int64_t>(g, 1));
+}
+
+// Slots for the decode kernel: enough that every SM gets an equal share of
+// the keys (decode_grid then uses one CTA per SM when there are enough).
+int decode_auto_splits(int64_t kv_heads, int64_t key_span, int sms) {
+  const int64_t g = std::min<int64_t>(sms, kv_heads * key_span / kDecMinKeysPerCta);
+  if (g <= 1) return 1;
+  const int64_t need = (g + kv_heads - 1) / kv_heads + 2;
+  return static_cast<int>(std::min<int64_t>(kMaxSplits, need));
+}
+
 // Optional inputs / outputs beyond fa_fwd's: the mask and softmax
 // statistics of fa_fwd_ex, the value descale of fa_fwd_fp8.
 struct FwdExtras {
@@ -232,6 +312,11 @@ struct FwdExtras {
 };
 
 constexpr int kE4M3 = 2;           // internal dtype code of fp8 e4m3 inputs
+
+// The split-KV merge for any head dim / dtype (oscale: descale_v of fp8).
+int launch_combine_any(int D, int dtype, const float *ws_o, const float2 *ws_ml, void *out,
+                       float *lse, int n_splits, long long rows_total, cudaStream_t stream,
+                       float oscale);
 
 // Shared body of fa_fwd, fa_fwd_ex and fa_fwd_splitkv (n_splits == 0: plain
 // forward; mx == nullptr: no mask, no statistics).
@@ -312,6 +397,65 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
   if (causal) wr = 0;                      // causal => wr := min(wr, 0)
   if (wl >= L_q) wl = -1;                  // no constraint left of row 0
   if (wr >= L_k) wr = -1;                  // no constraint right of L_k - 1
+
+  // decoding shapes: the CUDA-core kernel (no mask, no softmax statistics)
+  if (!masked && (mx == nullptr || mx->smax == nullptr) &&
+      decode_eligible(D, dtype, static_cast<int64_t>(L_q) * (H / H_kv))) {
+    DecParams dp;
+    std::memset(&dp, 0, sizeof(dp));
+    dp.q = static_cast<const uint8_t *>(q);
+    dp.k = static_cast<const uint8_t *>(k);
+    dp.v = static_cast<const uint8_t *>(v);
+    dp.out = out;
+    dp.lse = lse;
+    dp.H = H;
+    dp.H_kv = H_kv;
+    dp.L_q = L_q;
+    dp.L_k = L_k;
+    dp.group = H / H_kv;
+    dp.rows = L_q * (H / H_kv);
+    dp.wl = wl;
+    dp.wr = wr;
+    dp.n_splits = n_splits > 0 ? n_splits : 1;
+    // visible keys of the rows 0 .. L_q-1 of a head: [0, key_hi]
+    dp.key_span = (wr < 0 ? L_k - 1 : std::min(L_k - 1, L_q - 1 + wr)) + 1;
+    dp.heads = static_cast<long long>(B) * H_kv;
+    dp.rows_total = rows_total;
+    const unsigned grid = decode_grid(dp.heads, dp.key_span, dp.n_splits, sm_count());
+    {
+      const float sl2 = scale * 1.4426950408889634f;
+      dp.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;
+    }
+    dp.oscale = mx != nullptr ? mx->descale_v : 1.0f;
+    if (n_splits > 0) {
+      dp.ws_o = static_cast<float *>(workspace);
+      dp.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) +
+                                            ws_ml_offset(rows_total, D, n_splits));
+    }
+    int st = FA_ERR_HEADDIM;
+    switch (D * 2 + dtype) {
+#ifndef FA_TEST_HOOKS
+      case 32: st = launch_decode<16, 0>(dp, grid, stream); break;
+      case 33: st = launch_decode<16, 1>(dp, grid, stream); break;
+      case 64: st = launch_decode<32, 0>(dp, grid, stream); break;
+      case 65: st = launch_decode<32, 1>(dp, grid, stream); break;
+      case 128: st = launch_decode<64, 0>(dp, grid, stream); break;
+      case 129: st = launch_decode<64, 1>(dp, grid, stream); break;
+      case 256: st = launch_decode<128, 0>(dp, grid, stream); break;
+      case 257: st = launch_decode<128, 1>(dp, grid, stream); break;
+      case 66: st = launch_decode<32, kE4M3>(dp, grid, stream); break;
+      case 130: st = launch_decode<64, kE4M3>(dp, grid, stream); break;
+      case 258: st = launch_decode<128, kE4M3>(dp, grid, stream); break;
+#else
+    // the watchdog test library (FA_TEST_HOOKS): fp16 head dims 64 and 128 only
+      case 128: st = launch_decode<64, 0>(dp, grid, stream); break;
+      case 256: st = launch_decode<128, 0>(dp, grid, stream); break;
+#endif
+    }
+    if (st != FA_OK || n_splits == 0) return st;
+    return launch_combine_any(D, dtype, dp.ws_o, dp.ws_ml, out, lse, n_splits, rows_total,
+                              stream, dp.oscale);
+  }
   prm.lse = lse;
   prm.H = H;
   prm.H_kv = H_kv;
@@ -386,6 +530,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
 
   int st = FA_ERR_HEADDIM;
   switch (D * 2 + dtype + (masked ? 1000 : 0)) {
+#ifndef FA_TEST_HOOKS
     case 32: st = launch<16, 0, false>(prm, B, H, stream); break;
     case 33: st = launch<16, 1, false>(prm, B, H, stream); break;
     case 64: st = launch<32, 0, false>(prm, B, H, stream); break;
@@ -424,28 +569,46 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
     case 1066: st = launch<32, kE4M3, true>(prm, B, H, stream); break;
     case 1130: st = launch<64, kE4M3, true>(prm, B, H, stream); break;
     case 1258: st = launch<128, kE4M3, true>(prm, B, H, stream); break;
+#else
+    // the watchdog test library (FA_TEST_HOOKS): fp16 head dims 64 and 128 only
+    case 128: st = launch<64, 0, false>(prm, B, H, stream); break;
+    case 256: st = launch<128, 0, false>(prm, B, H, stream); break;
+#endif
   }
   if (st != FA_OK || n_splits == 0) return st;
+  return launch_combine_any(D, dtype, prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total,
+                            stream, prm.descale_v);
+}
+
+int launch_combine_any(int D, int dtype, const float *ws_o, const float2 *ws_ml, void *out,
+                       float *lse, int n_splits, long long rows_total, cudaStream_t stream,
+                       float oscale) {
   switch (D * 2 + dtype) {
-    case 32: return launch_combine<16, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 33: return launch_combine<16, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 64: return launch_combine<32, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 65: return launch_combine<32, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 128: return launch_combine<64, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 129: return launch_combine<64, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 256: return launch_combine<128, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 257: return launch_combine<128, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 96: return launch_combine<48, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 97: return launch_combine<48, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 160: return launch_combine<80, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 161: return launch_combine<80, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 192: return launch_combine<96, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 193: return launch_combine<96, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 224: return launch_combine<112, 0>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 225: return launch_combine<112, 1>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream);
-    case 66: return launch_combine<32, kE4M3>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream, prm.descale_v);
-    case 130: return launch_combine<64, kE4M3>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream, prm.descale_v);
-    case 258: return launch_combine<128, kE4M3>(prm.ws_o, prm.ws_ml, out, lse, n_splits, rows_total, stream, prm.descale_v);
+#ifndef FA_TEST_HOOKS
+    case 32: return launch_combine<16, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 33: return launch_combine<16, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 64: return launch_combine<32, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 65: return launch_combine<32, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 128: return launch_combine<64, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 129: return launch_combine<64, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 256: return launch_combine<128, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 257: return launch_combine<128, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 96: return launch_combine<48, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 97: return launch_combine<48, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 160: return launch_combine<80, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 161: return launch_combine<80, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 192: return launch_combine<96, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 193: return launch_combine<96, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 224: return launch_combine<112, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 225: return launch_combine<112, 1>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 66: return launch_combine<32, kE4M3>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream, oscale);
+    case 130: return launch_combine<64, kE4M3>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream, oscale);
+    case 258: return launch_combine<128, kE4M3>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream, oscale);
+#else
+    // the watchdog test library (FA_TEST_HOOKS): fp16 head dims 64 and 128 only
+    case 128: return launch_combine<64, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+    case 256: return launch_combine<128, 0>(ws_o, ws_ml, out, lse, n_splits, rows_total, stream);
+#endif
   }
   return FA_ERR_HEADDIM;
 }
@@ -538,6 +701,36 @@ extern "C" int fa_fwd_fp8_splitkv(const void *q, const void *k, const void *v, v
   return fa::fp8_impl(q, k, v, out, lse, B, H, H_kv, L_q, L_k, D, scale, descale_q, descale_k,
                       descale_v, causal, window_left, window_right, n_splits, workspace,
                       workspace_bytes, fa::FwdExtras{}, stream);
+}
+
+extern "C" int fa_splitkv_auto_splits(int B, int H, int H_kv, int L_q, int L_k, int D,
+                                      int dtype) {
+  if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || L_q < 1 || L_k < 1) return 1;
+  const int sms = fa::sm_count();
+  const int64_t rows_kv = static_cast<int64_t>(L_q) * (H / H_kv);
+  if (fa::decode_eligible(D, dtype == FA_F16 || dtype == FA_BF16 ? dtype : 2, rows_kv))
+    return fa::decode_auto_splits(static_cast<int64_t>(B) * H_kv, L_k, sms);   // upper bound
+  // tensor-core kernel: query tiles (GQA-packed when the group is a power of
+  // two and L_q < 128) x slices in waves of one CTA per SM; a CTA costs about
+  // 4.5 key blocks of fixed work (set-up, pipeline fill, epilogue) plus its
+  // blocks (a fit to decode timings on B200)
+  const int g = H / H_kv;
+  const bool packed = g >= 2 && g <= 128 && (g & (g - 1)) == 0 && L_q < 128;
+  const int64_t tile_q = packed ? 128 / g : 128;
+  const int64_t tiles = static_cast<int64_t>(B) * (packed ? H_kv : H) * ((L_q + tile_q - 1) / tile_q);
+  const int64_t blocks = std::max<int64_t>(1, (static_cast<int64_t>(L_k) + 127) / 128);
+  int best = 1;
+  double best_cost = 0.0;
+  for (int sp = 1; sp <= fa::kMaxSplits; ++sp) {
+    const int64_t per = (blocks + sp - 1) / sp;
+    if (sp > 1 && per < 2) break;
+    const double cost = static_cast<double>((tiles * sp + sms - 1) / sms) * (4.5 + per);
+    if (sp == 1 || cost < best_cost) {
+      best = sp;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 extern "C" size_t fa_splitkv_workspace_bytes(int B, int H, int L_q, int D, int n_splits) {
@@ -849,6 +1042,7 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *out, const
       !encode_map_f32(&prm.tm_dq, prm.dq_acc, B * H, L_q, D, D % 32 == 0 ? 32 : 16))
     return FA_ERR_CUDA;
   switch (D * 2 + dtype + (masked ? 1000 : 0)) {
+#ifndef FA_TEST_HOOKS
     case 32: return launch_bwd<16, 0, false>(prm, out, dout, lse, dq, B, H, stream);
     case 33: return launch_bwd<16, 1, false>(prm, out, dout, lse, dq, B, H, stream);
     case 64: return launch_bwd<32, 0, false>(prm, out, dout, lse, dq, B, H, stream);
@@ -881,6 +1075,11 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *out, const
     case 1193: return launch_bwd<96, 1, true>(prm, out, dout, lse, dq, B, H, stream);
     case 1224: return launch_bwd<112, 0, true>(prm, out, dout, lse, dq, B, H, stream);
     case 1225: return launch_bwd<112, 1, true>(prm, out, dout, lse, dq, B, H, stream);
+#else
+    // the watchdog test library (FA_TEST_HOOKS): fp16 head dims 64 and 128 only
+    case 128: return launch_bwd<64, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+    case 256: return launch_bwd<128, 0, false>(prm, out, dout, lse, dq, B, H, stream);
+#endif
   }
   return FA_ERR_HEADDIM;
 }
@@ -1061,6 +1260,18 @@ extern "C" int fa_selftest_wait_timeout(int *result, cudaStream_t stream) {
   fa::wait_selftest_kernel<<<1, 64, 0, stream>>>(result);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
+
+#ifdef FA_TEST_HOOKS
+// Watchdog test library only (include/fa_test_hooks.h): the key block whose
+// copy the K producer of CTA 0 withholds in the forward kernel (-1: none).
+extern "C" int fa_test_set_withhold(int block) {
+  if (cudaMemcpyToSymbol(fa::g_fa_test_withhold_block, &block, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+#endif
 
 extern "C" int fa_get_device_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;

@@ -98,6 +98,13 @@ constexpr int kLoadWarpV = 10;   // V
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 
+#ifdef FA_TEST_HOOKS
+// Watchdog test library only (never in libfa.so): the K producer of CTA 0
+// skips the copy of this key block (-1: none), so that the MMA warp's
+// bounded wait for it runs out and the abort path of every role runs.
+__device__ int g_fa_test_withhold_block = -1;
+#endif
+
 struct FwdParams {
   CUtensorMap tm_q;   // [B*H,    L_q, D]
   CUtensorMap tm_k;   // [B*H_kv, L_k, D]
@@ -494,6 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       const CUtensorMap *map = is_k ? &p.tm_k : &p.tm_v;
       int q = 0;
       bool ok = true;
+#ifdef FA_TEST_HOOKS
+      const int withheld = (is_k && blockIdx.x == 0) ? g_fa_test_withhold_block : -1;
+#else
+      constexpr int withheld = -1;
+#endif
       for (int j = lo; j < hi; ++j, ++q) {
         const int slot = base + q % nslot;
         if (q >= nslot) {
@@ -501,6 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           if (!ok) break;
         }
         const uint32_t bar = smem_u32(&bars->full[slot]);
+        if (j == withheld) continue;   // test library only: this fill never arrives
         if (elect_one()) {
           mbar_arrive_expect_tx(bar, G::kTileBytes);
 #pragma unroll
@@ -512,9 +525,16 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       }
       if (!ok) {
         // drain: let the copies already issued land before the CTA exits
+        // (Q tiles first: nothing else may have waited for them)
+        if (is_k) {
+          for (int t = 0; t < 2; ++t)
+            if (rng[t].hi > rng[t].lo)
+              mbar_wait_slow(smem_u32(&bars->q_full[t]), 0, abort_flag, false);
+        }
         for (int k = max(0, q - nslot); k < q; ++k)
-          mbar_wait_slow(smem_u32(&bars->full[base + k % nslot]), (k / nslot) & 1, abort_flag,
-                         false);
+          if (lo + k != withheld)
+            mbar_wait_slow(smem_u32(&bars->full[base + k % nslot]), (k / nslot) & 1,
+                           abort_flag, false);
       }
     }
   } else if (warp == kMmaWarp) {

@@ -18,7 +18,12 @@ namespace fa {
 // compiled into exactly one translation unit (fa_api.cu), which owns it.
 __device__ unsigned int g_fa_status = 0u;
 
-constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+// Wait limit: 1 s in the library; the watchdog test library is built with a
+// shorter one (FA_WAIT_LIMIT_NS) so that its withheld-copy test ends quickly.
+#ifndef FA_WAIT_LIMIT_NS
+#define FA_WAIT_LIMIT_NS (1000ull * 1000ull * 1000ull)
+#endif
+constexpr unsigned long long kWaitLimitNs = FA_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -96,6 +96,13 @@ typedef enum {
  * The call only enqueues work: argument errors are returned before anything
  * is enqueued; device-side watchdog errors are reported by
  * fa_get_device_status().
+ *
+ * Decoding shapes -- at most two query rows per K/V head (L_q * H / H_kv
+ * <= 2) and D in {16, 32, 64, 128} -- run on a CUDA-core kernel that
+ * streams the key/value cache through shared memory (the product with one
+ * or two query rows is a matrix-vector product, far from the tensor cores'
+ * work); it keeps the softmax weights in fp32.  Everything else runs on the
+ * tcgen05 tensor-core kernel.  The result is the same function either way.
  */
 int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
            int B, int H, int H_kv, int L_q, int L_k, int D, float scale,
@@ -296,6 +303,19 @@ int fa_bwd_ex(const void *q, const void *k, const void *v, const void *out, cons
               int H, int H_kv, int L_q, int L_k, int D, float scale, int causal,
               int window_left, int window_right, int dtype, void *workspace,
               size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fa_splitkv_auto_splits -- the number of key slices the library would pick
+ * for fa_fwd_splitkv / fa_fwd_fp8_splitkv on the current device (dtype:
+ * FA_F16, FA_BF16, or 2 for E4M3 inputs).  For decoding shapes (at most two
+ * query rows per K/V head: L_q * H / H_kv <= 2, head dims 16, 32, 64, 128)
+ * the forward runs on the CUDA cores over a persistent grid of one CTA per
+ * SM, and the slices make (B * H_kv * slices) work items whose last round is
+ * nearly full; otherwise the tensor-core kernel's query tiles and slices
+ * fill waves of one CTA per SM.  Returns 1 for empty or invalid sizes.
+ * This is a planning helper: a split count, not a result of the method.
+ */
+int fa_splitkv_auto_splits(int B, int H, int H_kv, int L_q, int L_k, int D, int dtype);
 
 /*
  * fa_fwd_splitkv_static -- fa_fwd_splitkv with no workspace argument: the

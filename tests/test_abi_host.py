@@ -140,10 +140,15 @@ def test_splitkv_argument_errors(lib, kw, code):
 
 
 def test_choose_splits():
-    assert fa.choose_splits(1, 32, 1, 32768) == 9       # 32 tiles -> 288 CTAs, two waves
-    assert fa.choose_splits(4, 48, 8192, 8192) == 1     # already many waves
-    assert fa.choose_splits(1, 1, 1, 128) == 1          # one key block
+    # decoding shapes (one or two rows per K/V head) go to the CUDA-core kernel,
+    # whose slots let every one of the 148 SMs take an equal share of the keys:
+    # ceil(148 / heads) + 2 slots
+    assert fa.choose_splits(1, 32, 1, 32768) == 7       # 32 heads -> 5 + 2
+    assert fa.choose_splits(4, 32, 1, 16384) == 4       # 128 heads -> 2 + 2
+    assert fa.choose_splits(1, 1, 1, 128) == 1          # too few keys to split
     assert fa.choose_splits(1, 1, 1, 1 << 20) == 64     # capped
+    # the tensor-core kernel: query tiles x slices in waves of one CTA per SM
+    assert fa.choose_splits(4, 48, 8192, 8192) == 1     # already many waves
     # GQA packing: 32 query heads over 8 K/V heads, one query row -> 8 tiles
     assert fa.binding.query_tiles(1, 32, 8, 1) == 8
     assert fa.binding.query_tiles(1, 32, 8, 40) == 16      # 32 rows per head per tile
@@ -351,3 +356,18 @@ def test_bwd_ex_argument_errors(lib, kw, code):
 def test_watchdog_selftest_rejects_null(lib):
     # returns before any CUDA call
     assert fa.fa_selftest_wait_timeout(None, None) == -1
+
+
+# ------------------------------------------------------------ watchdog test library
+def test_product_library_has_no_test_hook(lib):
+    # the withheld-copy hook exists only in lib/libfa_testhooks.so
+    assert not hasattr(lib, "fa_test_set_withhold")
+
+
+def test_test_library_exports_the_hook():
+    import ctypes
+    from exact_attention_113_b200 import build as fa_build
+    if not os.path.exists(fa_build.TESTHOOKS_PATH):
+        pytest.skip("watchdog test library not built (build(testhooks=True))")
+    t = ctypes.CDLL(fa_build.TESTHOOKS_PATH)
+    assert hasattr(t, "fa_test_set_withhold") and hasattr(t, "fa_fwd")
