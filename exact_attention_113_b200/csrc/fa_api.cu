@@ -246,10 +246,8 @@ int sm_count() {
 
 template <int D, int DT, int R>
 int launch_decode_kernel(const DecParams &prm, unsigned grid, cudaStream_t stream) {
-  using G = DecGeo<D, DT == 2 ? 1 : 2>;
   auto kern = fa_decode_kernel<D, DT, R>;
-  const int smem = G::kStages * G::kStageBytes + kDecWarps * R * D * 4 + kDecWarps * R * 8 +
-                   2 * G::kStages * 8 + 16;
+  const int smem = DecSmem<D, DT, R>::kBytes;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   static bool configured[64] = {};
@@ -274,9 +272,9 @@ int launch_decode(const DecParams &prm, unsigned grid, cudaStream_t stream) {
   return launch_decode_kernel<D, DT, 2>(prm, grid, stream);
 }
 
-// Keys a CTA of the decode kernel should get at least (two chunks), so that
-// its fixed work (set-up, the first copies' latency, the merge) stays small.
-constexpr int64_t kDecMinKeysPerCta = 2 * kDecChunk;
+// Keys a CTA of the decode kernel should get at least, so that its fixed
+// work (set-up, the first copies' latency, the merge) stays small.
+constexpr int64_t kDecMinKeysPerCta = 256;
 
 // Grid of the decode kernel.  One slot per row: one CTA per K/V head (at
 // most one per SM; heads taken with a stride).  n_splits >= 2 slots: the
@@ -296,7 +294,9 @@ unsigned decode_grid(int64_t heads, int64_t key_span, int n_splits, int sms) {
 // the keys (decode_grid then uses one CTA per SM when there are enough).
 int decode_auto_splits(int64_t kv_heads, int64_t key_span, int sms) {
   const int64_t g = std::min<int64_t>(sms, kv_heads * key_span / kDecMinKeysPerCta);
-  if (g <= 1) return 1;
+  // with at least three K/V heads per four SMs, whole heads (one slot, no
+  // merge launch) measured faster than equal ranges over every SM
+  if (g <= 1 || 4 * kv_heads >= 3 * static_cast<int64_t>(sms)) return 1;
   const int64_t need = (g + kv_heads - 1) / kv_heads + 2;
   return static_cast<int>(std::min<int64_t>(kMaxSplits, need));
 }
@@ -427,7 +427,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
       dp.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;
     }
     dp.oscale = mx != nullptr ? mx->descale_v : 1.0f;
-    if (n_splits > 0) {
+    if (n_splits > 1) {   // one slot: whole heads write their rows directly
       dp.ws_o = static_cast<float *>(workspace);
       dp.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) +
                                             ws_ml_offset(rows_total, D, n_splits));
@@ -452,7 +452,7 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
       case 256: st = launch_decode<128, 0>(dp, grid, stream); break;
 #endif
     }
-    if (st != FA_OK || n_splits == 0) return st;
+    if (st != FA_OK || n_splits <= 1) return st;
     return launch_combine_any(D, dtype, dp.ws_o, dp.ws_ml, out, lse, n_splits, rows_total,
                               stream, dp.oscale);
   }

@@ -5,7 +5,7 @@
 // There S = Q K^T is a matrix-vector product per head: one multiply-add per
 // byte of K read, far below what the tensor cores are for, so the work is
 // bounded by how fast the cache streams out of HBM.  The kernel therefore
-// keeps every SM pulling bytes:
+// keeps every SM pulling bytes with as few instructions per key as it can:
 //   - a persistent grid of at most one CTA per SM walks "segments" (a K/V
 //     head and a range of its visible keys).  With a single partial slot per
 //     row (fa_fwd: no workspace) a segment is a whole head and CTAs take
@@ -13,19 +13,24 @@
 //     into equal contiguous ranges, one per CTA (the ranges cross head
 //     boundaries), so every SM gets the same number of keys and a head is
 //     covered by at most n_splits CTAs, each writing its slice's partial;
-//   - one producer warp streams chunks of 128 keys of K and of V (each a
+//   - one producer warp streams chunks of keys of K and of V (each a
 //     contiguous run of rows) into a ring of shared-memory stages with
 //     untiled bulk copies, completion counted on mbarriers;
-//   - eight compute warps take 16 keys of every chunk each: a group of LPR
-//     lanes holds one key (16 bytes per lane), its dot products with the R
-//     query rows are reduced across the group with shuffles; the online
-//     softmax ("Flash Attention是怎么做到又快又省显存的？": running maximum,
-//     normaliser rescaled when the maximum grows, here conditionally: the
-//     reference maximum moves only when a chunk exceeds it by 2^8) runs per
-//     row with a warp-wide reference, and the V rows are accumulated into
-//     per-lane partial outputs;
-//   - at the end of a segment the eight warps' partials are merged through
-//     shared memory (key slices of one row, the merge of
+//   - eight compute warps: a lane holds one key (two or four lanes for long
+//     rows) and HD of its dimensions, so the dot products and the V
+//     accumulation are plain per-lane multiply-adds with no shuffles; lane
+//     k reads the 16-byte units of its row starting at unit k (mod the row's
+//     units), so a warp's shared-memory reads never share a bank more than
+//     the 512 bytes they move require; the query slice and the output slice
+//     of a lane are kept in that same rotated order;
+//   - the online softmax ("Flash Attention是怎么做到又快又省显存的？":
+//     running maximum, normaliser rescaled when the maximum grows; here
+//     conditionally, the reference maximum moves only when a chunk exceeds
+//     it by 2^8) runs per row with a warp-wide reference; the weights stay
+//     fp32;
+//   - at the end of a segment the lanes' partial outputs are summed (first
+//     across lanes that share a rotation, then through shared memory) and
+//     the warps' partials are merged as key slices of one row (the merge of
 //     "FlashAttention算法原理与性能优化实战" section 1.2.2), then written
 //     either as the final row (O / l, lse) or as the slice's unnormalised
 //     partial (O, m, l) for the split-KV merge kernel.
@@ -38,10 +43,8 @@
 
 namespace fa {
 
-constexpr int kDecChunk = 128;          // keys per stage
 constexpr int kDecWarps = 8;            // compute warps
 constexpr int kDecThreads = 32 * (kDecWarps + 1);
-constexpr int kDecKeysPerWarp = kDecChunk / kDecWarps;
 constexpr int kDecRingBytes = 192 * 1024;
 
 struct DecParams {
@@ -78,19 +81,24 @@ __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads,
   return r != 0;
 }
 
-template <int D, int ES>
+// Geometry for head dim D, ES-byte elements and R query rows.
+template <int D, int ES, int R>
 struct DecGeo {
-  static constexpr int kEPL = 16 / ES;                 // elements per lane per key
-  static constexpr int kLPR = D / kEPL;                // lanes per key
-  static constexpr int kKPI = 32 / kLPR;               // keys per warp instruction
-  static constexpr int kIters = kDecKeysPerWarp / kKPI;
+  static constexpr int kHD = D < 64 / R ? D : 64 / R;     // dimensions a lane holds
+  static constexpr int kLPK = D / kHD;                    // lanes per key
+  static constexpr int kKPW = 32 / kLPK;                  // keys per warp per chunk
+  static constexpr int kChunk = kDecWarps * kKPW;         // keys per stage
+  static constexpr int kEPU = 16 / ES;                    // elements per 16-byte unit
+  static constexpr int kU = kHD * ES / 16;                // units a lane reads per row
   static constexpr int kRowBytes = D * ES;
-  static constexpr int kTileBytes = kDecChunk * kRowBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;   // K and V
+  static constexpr int kTileBytes = kChunk * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;      // K and V
   static constexpr int kStages = kDecRingBytes / kStageBytes < 8 ? kDecRingBytes / kStageBytes : 8;
-  static_assert(kEPL * kLPR == D && kLPR >= 2 && kLPR <= 32 && (kLPR & (kLPR - 1)) == 0,
-                "a key row is a power-of-two number of 16-byte lane slices");
-  static_assert(kIters >= 1 && kIters * kKPI == kDecKeysPerWarp, "keys per warp");
+  // lanes that hold the same rotation of their units: one group per
+  // rotation after the sum across lanes kU keys apart
+  static constexpr int kRot = kU < kKPW ? kU : kKPW;
+  static_assert(kHD * kLPK == D && kU >= 1 && kU * 16 == kHD * ES, "lane slices of 16-byte units");
+  static_assert((kU & (kU - 1)) == 0 && (kLPK & (kLPK - 1)) == 0, "powers of two");
   static_assert(kStages >= 2, "ring depth");
 };
 
@@ -145,7 +153,18 @@ struct DecWalk {
   }
 };
 
-// 16 bytes of one key row -> kEPL floats.
+// Untiled bulk copy global -> shared (as bulk_load_1d) with an L2 policy:
+// the cache is streamed once, so its lines are marked evict-first.
+__device__ __forceinline__ void bulk_load_1d_hint(uint32_t dst, const void *src, uint32_t bytes,
+                                                  uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// One 16-byte unit -> its elements as floats.
 template <int DT>
 __device__ __forceinline__ void dec_unpack(const uint4 &w, float (&x)[16 / (DT == 2 ? 1 : 2)]) {
   const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -179,18 +198,34 @@ __device__ __forceinline__ void dec_unpack(const uint4 &w, float (&x)[16 / (DT =
   }
 }
 
+// Shared memory of one instance: the ring, then the warps' partial outputs
+// (one per rotation group), then (m, l) per warp and row, then barriers.
+template <int D, int DT, int R>
+struct DecSmem {
+  using G = DecGeo<D, DT == 2 ? 1 : 2, R>;
+  static constexpr int kOffXo = G::kStages * G::kStageBytes;
+  static constexpr int kXoFloats = kDecWarps * G::kRot * R * D;
+  static constexpr int kOffXml = kOffXo + kXoFloats * 4;
+  static constexpr int kOffBar = kOffXml + kDecWarps * R * 2 * 4;
+  static constexpr int kBytes = kOffBar + 2 * G::kStages * 8 + 16;
+  static_assert(kOffBar % 8 == 0, "barrier alignment");
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
 // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 (bf16 output).  R: most query rows per
 // K/V head.
 template <int D, int DT, int R>
 __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_constant__ DecParams p) {
   constexpr int ES = DT == 2 ? 1 : 2;
-  using G = DecGeo<D, ES>;
-  constexpr int EPL = G::kEPL, LPR = G::kLPR, KPI = G::kKPI, NS = G::kStages;
+  using G = DecGeo<D, ES, R>;
+  using SM = DecSmem<D, DT, R>;
+  constexpr int HD = G::kHD, LPK = G::kLPK, KPW = G::kKPW, CH = G::kChunk;
+  constexpr int EPU = G::kEPU, U = G::kU, NS = G::kStages, ROT = G::kRot;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint8_t *ring = smem_raw;                                        // NS x (K, V)
-  float *xo = reinterpret_cast<float *>(smem_raw + NS * G::kStageBytes);   // [warps][R][D]
-  float *xml = xo + kDecWarps * R * D;                              // [warps][R][2]
-  uint64_t *full = reinterpret_cast<uint64_t *>(xml + kDecWarps * R * 2);
+  uint8_t *ring = smem_raw;                                          // NS x (K, V)
+  float *xo = reinterpret_cast<float *>(smem_raw + SM::kOffXo);      // [warps][ROT][R][D]
+  float *xml = reinterpret_cast<float *>(smem_raw + SM::kOffXml);    // [warps][R][2]
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem_raw + SM::kOffBar);
   uint64_t *empty = full + NS;
   int *abort_i = reinterpret_cast<int *>(empty + NS);
   volatile int *abort_flag = abort_i;
@@ -211,23 +246,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
     // ============================================= producer
     int q = 0;           // chunks issued by this CTA so far (ring position)
     bool ok = true;
+    const uint64_t pol = policy_evict_first();
     DecWalk walk(p);
     DecSegment sg;
     while (ok && walk.advance(p, sg)) {
-      for (int j0 = sg.a; j0 < sg.b; j0 += kDecChunk, ++q) {
+      for (int j0 = sg.a; j0 < sg.b; j0 += CH, ++q) {
         const int s = q % NS;
         if (q >= NS) {
           ok = mbar_wait_warp(smem_u32(&empty[s]), ((q / NS) - 1) & 1, abort_flag);
           if (!ok) break;
         }
-        const int n = min(kDecChunk, sg.b - j0);
+        const int n = min(CH, sg.b - j0);
         const uint32_t bytes = static_cast<uint32_t>(n) * G::kRowBytes;
         const size_t off = (static_cast<size_t>(sg.head) * p.L_k + j0) * G::kRowBytes;
         if (elect_one()) {
           const uint32_t bar = smem_u32(&full[s]);
           mbar_arrive_expect_tx(bar, 2 * bytes);
-          bulk_load_1d(smem_u32(ring + s * G::kStageBytes), p.k + off, bytes, bar);
-          bulk_load_1d(smem_u32(ring + s * G::kStageBytes + G::kTileBytes), p.v + off, bytes, bar);
+          bulk_load_1d_hint(smem_u32(ring + s * G::kStageBytes), p.k + off, bytes, bar, pol);
+          bulk_load_1d_hint(smem_u32(ring + s * G::kStageBytes + G::kTileBytes), p.v + off, bytes,
+                            bar, pol);
         }
         __syncwarp();
       }
@@ -239,8 +276,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
     }
   } else {
     // ============================================= compute warps
-    const int grp = lane / LPR;          // key within the warp instruction
-    const int sub = lane % LPR;          // 16-byte column of the key row
+    const int kl = lane / LPK;             // key of this lane within the warp's keys
+    const int part = lane % LPK;           // which HD-slice of the row
+    const int rot = kl % U;                // this lane reads unit (u + rot) % U at step u
+    const int kk = warp * KPW + kl;        // key within the chunk
+    const uint32_t row_off = kk * G::kRowBytes + part * HD * ES;
     int q = 0;
     bool ok = true;
     DecWalk walk(p);
@@ -249,8 +289,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       const int b = static_cast<int>(sg.head / p.H_kv);
       const int hk = static_cast<int>(sg.head - static_cast<long long>(b) * p.H_kv);
 
-      // this lane's 16-byte slice of every query row, as floats
-      float qv[R][EPL];
+      // this lane's slice of every query row, units in rotated order
+      float qv[R][U][EPU];
       int qpos[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -258,114 +298,120 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         const int g = rr / p.L_q, i = rr - g * p.L_q;
         qpos[r] = r < p.rows ? i : -1;
         const long long row = (static_cast<long long>(b) * p.H + hk * p.group + g) * p.L_q + i;
-        const uint4 w = *reinterpret_cast<const uint4 *>(p.q + row * G::kRowBytes + sub * 16);
-        dec_unpack<DT>(w, qv[r]);
+        const uint8_t *qrow = p.q + row * G::kRowBytes + part * HD * ES;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(qrow + ((u + rot) % U) * 16);
+          dec_unpack<DT>(w, qv[r][u]);
+        }
       }
-      float m_ref[R], l[R], o[R][EPL];
+      float m_ref[R], l[R], o[R][U][EPU];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         m_ref[r] = -INFINITY;
         l[r] = 0.0f;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) o[r][e] = 0.0f;
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int e = 0; e < EPU; ++e) o[r][u][e] = 0.0f;
       }
 
-      for (int j0 = sg.a; j0 < sg.b && ok; j0 += kDecChunk, ++q) {
+      for (int j0 = sg.a; j0 < sg.b && ok; j0 += CH, ++q) {
         const int s = q % NS;
         ok = mbar_wait_warp(smem_u32(&full[s]), (q / NS) & 1, abort_flag);
         if (!ok) break;
-        const uint8_t *kt = ring + s * G::kStageBytes;
+        const uint8_t *kt = ring + s * G::kStageBytes + row_off;
         const uint8_t *vt = kt + G::kTileBytes;
-        // every key of the chunk visible to every row?
-        const bool full_vis = (j0 + kDecChunk <= sg.b) &&
-                              (p.wl < 0 || j0 >= p.L_q - 1 - p.wl) &&
-                              (p.wr < 0 || j0 + kDecChunk - 1 <= p.wr);
-        // scores of this warp's 16 keys, in log2 units of the scaled score
-        float sc[G::kIters][R];
-        float cmax[R];
+        const int j = j0 + kk;                 // this lane's key
+        // S for this lane's key: per-lane multiply-adds over its slice
+        float acc[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) cmax[r] = -INFINITY;
+        for (int r = 0; r < R; ++r) acc[r] = 0.0f;
 #pragma unroll
-        for (int t = 0; t < G::kIters; ++t) {
-          const int kk = warp * kDecKeysPerWarp + t * KPI + grp;    // key in the chunk
-          const uint4 w = *reinterpret_cast<const uint4 *>(kt + kk * G::kRowBytes + sub * 16);
-          float kx[EPL];
+        for (int u = 0; u < U; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(kt + ((u + rot) % U) * 16);
+          float kx[EPU];
           dec_unpack<DT>(w, kx);
 #pragma unroll
-          for (int r = 0; r < R; ++r) {
-            float acc = 0.0f;
+          for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) acc = fmaf(qv[r][e], kx[e], acc);
-#pragma unroll
-            for (int off = LPR / 2; off > 0; off >>= 1)
-              acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            float x = acc * p.scale_log2;
-            if (!full_vis) {
-              const int j = j0 + kk;
-              const bool vis = j < sg.b && qpos[r] >= 0 && (p.wl < 0 || j >= qpos[r] - p.wl) &&
-                               (p.wr < 0 || j <= qpos[r] + p.wr);
-              x = vis ? x : -INFINITY;
-            }
-            sc[t][r] = x;
-            cmax[r] = fmaxf(cmax[r], x);
-          }
+            for (int e = 0; e < EPU; ++e) acc[r] = fmaf(qv[r][u][e], kx[e], acc[r]);
         }
-        // warp-wide maximum of the chunk per row; conditional rescale
+        float sc[R], cmax[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
 #pragma unroll
-          for (int off = 16; off >= LPR; off >>= 1)
+          for (int off = LPK / 2; off > 0; off >>= 1)
+            acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
+          const bool vis = j < sg.b && qpos[r] >= 0 && (p.wl < 0 || j >= qpos[r] - p.wl) &&
+                           (p.wr < 0 || j <= qpos[r] + p.wr);
+          sc[r] = vis ? acc[r] * p.scale_log2 : -INFINITY;
+          // warp-wide maximum of the chunk; conditional rescale
+          cmax[r] = sc[r];
+#pragma unroll
+          for (int off = 16; off >= LPK; off >>= 1)
             cmax[r] = fmaxf(cmax[r], __shfl_xor_sync(0xffffffffu, cmax[r], off));
           if (cmax[r] > m_ref[r] + kRescaleThreshold) {
             const float a = (m_ref[r] == -INFINITY) ? 1.0f : ex2(m_ref[r] - cmax[r]);
             m_ref[r] = cmax[r];
             l[r] *= a;
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[r][e] *= a;
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+              for (int e = 0; e < EPU; ++e) o[r][u][e] *= a;
           }
         }
         // P and O += P V
+        float pr[R];
+        bool any = false;
 #pragma unroll
-        for (int t = 0; t < G::kIters; ++t) {
-          const int kk = warp * kDecKeysPerWarp + t * KPI + grp;
-          float pr[R];
-          bool any = false;
+        for (int r = 0; r < R; ++r) {
+          pr[r] = (sc[r] == -INFINITY) ? 0.0f : ex2(sc[r] - m_ref[r]);
+          l[r] += pr[r];
+          any = any || pr[r] != 0.0f;
+        }
+        if (any) {   // masked keys (and rows past the segment's end) add nothing
 #pragma unroll
-          for (int r = 0; r < R; ++r) {
-            pr[r] = (sc[t][r] == -INFINITY) ? 0.0f : ex2(sc[t][r] - m_ref[r]);
-            l[r] += pr[r];
-            any = any || pr[r] != 0.0f;
-          }
-          if (any) {   // masked keys (and rows past the segment's end) add nothing
-            const uint4 w = *reinterpret_cast<const uint4 *>(vt + kk * G::kRowBytes + sub * 16);
-            float vx[EPL];
+          for (int u = 0; u < U; ++u) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(vt + ((u + rot) % U) * 16);
+            float vx[EPU];
             dec_unpack<DT>(w, vx);
 #pragma unroll
             for (int r = 0; r < R; ++r)
 #pragma unroll
-              for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(pr[r], vx[e], o[r][e]);
+              for (int e = 0; e < EPU; ++e) o[r][u][e] = fmaf(pr[r], vx[e], o[r][u][e]);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
       }
 
-      // ---- the segment's row results: sum the key groups of the warp ...
+      // ---- the segment's row results.  l: the sum over the warp's keys (each
+      // key counted by one lane of its group).  O: first summed across the
+      // lanes that share a rotation (keys U apart), then each rotation group
+      // writes its slice, un-rotated, for the merge below.
 #pragma unroll
       for (int r = 0; r < R; ++r) {
+        if (part != 0) l[r] = 0.0f;
 #pragma unroll
-        for (int off = 16; off >= LPR; off >>= 1) {
-          l[r] += __shfl_xor_sync(0xffffffffu, l[r], off);
+        for (int off = 16; off >= 1; off >>= 1) l[r] += __shfl_xor_sync(0xffffffffu, l[r], off);
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) o[r][e] += __shfl_xor_sync(0xffffffffu, o[r][e], off);
-        }
+        for (int off = 16; off >= LPK * ROT; off >>= 1)
+#pragma unroll
+          for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int e = 0; e < EPU; ++e)
+              o[r][u][e] += __shfl_xor_sync(0xffffffffu, o[r][u][e], off);
       }
-      // ... then merge the warps (key slices of every row)
-      if (grp == 0) {
+      if (kl < ROT) {
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) xo[(warp * R + r) * D + sub * EPL + e] = o[r][e];
+          for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int e = 0; e < EPU; ++e)
+              xo[((warp * ROT + kl) * R + r) * D + part * HD + ((u + rot) % U) * EPU + e] =
+                  o[r][u][e];
       }
       if (lane == 0) {
 #pragma unroll
@@ -388,7 +434,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
             if (mw == -INFINITY) continue;
             const float a = ex2(mw - m);
             lt += a * xml[(w * R + r) * 2 + 1];
-            ot += a * xo[(w * R + r) * D + d];
+            float os = 0.0f;
+#pragma unroll
+            for (int g = 0; g < ROT; ++g) os += xo[((w * ROT + g) * R + r) * D + d];
+            ot += a * os;
           }
         }
         const int g = r / p.L_q, i = r - g * p.L_q;

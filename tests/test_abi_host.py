@@ -142,9 +142,9 @@ def test_splitkv_argument_errors(lib, kw, code):
 def test_choose_splits():
     # decoding shapes (one or two rows per K/V head) go to the CUDA-core kernel,
     # whose slots let every one of the 148 SMs take an equal share of the keys:
-    # ceil(148 / heads) + 2 slots
+    # ceil(148 / heads) + 2 slots, or whole heads from 3 heads per 4 SMs on
     assert fa.choose_splits(1, 32, 1, 32768) == 7       # 32 heads -> 5 + 2
-    assert fa.choose_splits(4, 32, 1, 16384) == 4       # 128 heads -> 2 + 2
+    assert fa.choose_splits(4, 32, 1, 16384) == 1       # 128 heads: whole heads, no merge
     assert fa.choose_splits(1, 1, 1, 128) == 1          # too few keys to split
     assert fa.choose_splits(1, 1, 1, 1 << 20) == 64     # capped
     # the tensor-core kernel: query tiles x slices in waves of one CTA per SM
