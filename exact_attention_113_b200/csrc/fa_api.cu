@@ -114,10 +114,10 @@ __global__ void fill_kernel(float *p, size_t n, float value) {
   for (; i < n; i += stride) p[i] = value;
 }
 
-template <int D, int DT, bool kMask, bool kHalfS, bool kDual = false>
+template <int D, int DT, bool kMask, bool kDual = false>
 int launch_kernel(const FwdParams &prm, int B, int H, cudaStream_t stream) {
   using G = Geo<D, DT == 2 ? 1 : 2>;
-  auto kern = fa_fwd_kernel<D, DT, kMask, kHalfS, kDual>;
+  auto kern = fa_fwd_kernel<D, DT, kMask, kDual>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   static bool configured[64] = {};
@@ -139,16 +139,11 @@ int launch_kernel(const FwdParams &prm, int B, int H, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// One query tile per CTA: 16-bit inputs take the dual softmax (the tile's
-// keys split between both softmax warpgroups), fp8 at D > 64 the half-S
-// schedule; everything else the kernel's default for its head dim.
+// One query tile per CTA: the dual softmax (the tile's keys split between
+// both softmax warpgroups); two tiles: the kernel's default for its head dim.
 template <int D, int DT, bool kMask>
 int launch(const FwdParams &prm, int B, int H, cudaStream_t stream) {
-  if constexpr (DT != 2) {
-    if (prm.tiles == 1) return launch_kernel<D, DT, kMask, false, true>(prm, B, H, stream);
-  } else if constexpr (D > 64) {
-    if (prm.tiles == 1) return launch_kernel<D, DT, kMask, true>(prm, B, H, stream);
-  }
+  if (prm.tiles == 1) return launch_kernel<D, DT, kMask, true>(prm, B, H, stream);
   return launch_kernel<D, DT, kMask, false>(prm, B, H, stream);
 }
 

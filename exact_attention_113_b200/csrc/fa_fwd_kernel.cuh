@@ -34,21 +34,7 @@
 // PV_t(j), which reads P_t from the same TMEM columns; tcgen05 MMAs issued by
 // one thread execute in issue order.
 //
-// D > 64, one query tile, fp8 inputs (kHalfS; problems with fewer query
-// tiles than SMs, decoding): with no second tile to ping-pong with, S_t is
-// computed in two 64-key halves and P_t is written over the second half,
-// columns [64, 128).
-// Per block j the MMA issuer runs
-//   S_t(j) keys [0, 64)     once the softmax holds S_t(j-1) (s_free),
-//   PV_t(j-1)               once P_t(j-1) is in TMEM (p_full),
-//   S_t(j) keys [64, 128)   into the columns PV_t(j-1) has just read,
-// so the softmax of block j starts on the first half while the tensor pipe
-// still runs PV_t(j-1) and the second half.  (With two tiles this schedule
-// measured 11-15 % slower than the ping-pong: the N = 64 halves and the two
-// softmax warpgroups competing for the exp unit cost more than the shorter
-// chain saves.)
-//
-// One query tile, 16-bit inputs, any D (kDual): the second softmax
+// One query tile, any D (kDual): the second softmax
 // warpgroup would be idle, so the two warpgroups split every block's keys:
 // warpgroup h takes keys [64h, 64h + 64) of S0 with its own running max and
 // sum, its own P_h (columns [128 + 64h, 160 + 64h), S1's unused slot) and
@@ -81,12 +67,9 @@ constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kBN = 128;        // keys per K/V block
 constexpr int kThreads = 384;
 constexpr uint32_t kLaunchRegs = 168;   // 65536 / 384, rounded down to 8
-// Softmax / other-warpgroup register split per instance: the half-S issuer
-// keeps more state than 56 registers hold (fewest spills measured with
-// ptxas -v for each choice).
-template <int D, int DT, bool kHalfS>
+// Softmax / other-warpgroup register split.
 struct RegSplit {
-  static constexpr uint32_t kBig = !kHalfS ? 224 : (D < 128 ? 216 : (DT == 2 ? 224 : 208));
+  static constexpr uint32_t kBig = 224;
   static constexpr uint32_t kSmall = (kThreads * kLaunchRegs - 2 * 128 * kBig) / 128;
   static_assert(kSmall % 8 == 0 && kSmall >= 24, "setmaxnreg takes multiples of 8");
   static_assert(2 * 128 * kBig + 128 * kSmall <= kThreads * kLaunchRegs,
@@ -200,14 +183,13 @@ struct Bars {
   uint64_t q_full[2];
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
-  uint64_t s_full[2];     // S_t complete (half-S: keys [64, 128) of S_t)
+  uint64_t s_full[2];     // S_t complete
   uint64_t s_free[2];     // softmax holds S_t in registers
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
-  uint64_t s_lo_full[2];  // half-S: keys [0, 64) of S_t complete
 };
 
 // Key range [lo, hi) in blocks for query rows [first, last] of one tile.
@@ -350,13 +332,10 @@ __device__ __forceinline__ void store_p_half(uint32_t base, int half, const uint
     tmem_st_x32(base + 32u * half, pk);
 }
 
-template <int D, int DT, bool kMask, bool kHalfS, bool kDual = false>
+template <int D, int DT, bool kMask, bool kDual = false>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
-  // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 inputs (bf16 output).  kHalfS: the
-  // half-S schedule (D > 64, one query tile per CTA).  kDual: one query
+  // DT: 0 fp16, 1 bf16, 2 fp8 e4m3 inputs (bf16 output).  kDual: one query
   // tile, its keys split between the two softmax warpgroups (D <= 64).
-  static_assert(!kHalfS || D > 64, "half-S schedule is for D > 64");
-  static_assert(!kDual || (!kHalfS && DT != 2), "dual softmax is for 16-bit inputs");
   constexpr bool kF8 = DT == 2;
   constexpr int kES = kF8 ? 1 : 2;
   constexpr int kKStep = 32 / kES;             // K of one MMA instruction (32 bytes)
@@ -438,7 +417,6 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&bars->q_full[t]), 1);
       mbar_init(smem_u32(&bars->s_full[t]), 1);
-      if (kHalfS) mbar_init(smem_u32(&bars->s_lo_full[t]), 1);
       mbar_init(smem_u32(&bars->s_free[t]), (kDual && t == 0) ? 2 * kBM : kBM);
       mbar_init(smem_u32(&bars->p_full[t]), kBM);
       mbar_init(smem_u32(&bars->pv_done[t]), 1);
@@ -471,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 
   if (warp >= 8) {
   // ===================================================== warpgroup 2
-  regs_dec<RegSplit<D, DT, kHalfS>::kSmall>();
+  regs_dec<RegSplit::kSmall>();
   if (warp == kLoadWarp || warp == kLoadWarpV) {
     // =================================================== TMA producers
     // Warp 9 loads Q and the K ring, warp 10 the V ring.  The whole warp
@@ -571,11 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       };
       auto issue_pv = [&](int t, int slot) {
         const uint32_t vlo = desc_lo(sRing + slot * G::kTileBytes, G::kBoxBytes);
-        // P_t: own columns (D <= 64), S_t columns [64, 128) (half-S) or
-        // [0, 64) (ping-pong)
-        const uint32_t a_tmem =
-            tmem + (G::kSplitP ? 384u + (t ? 64u : 0u)
-                               : (t ? 128u : 0u) + (kHalfS ? 64u : 0u));
+        // P_t: own columns (D <= 64) or S_t columns [0, 64) (ping-pong)
+        const uint32_t a_tmem = tmem + (G::kSplitP ? 384u + (t ? 64u : 0u) : (t ? 128u : 0u));
         const uint32_t d_tmem = tmem + 256u + (t ? D : 0u);
         const bool first = (t ? npv1 : npv0) == 0;
         if (elect_one()) {
@@ -696,69 +671,6 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             commit(smem_u32(&bars->empty[vslot(q - 1)]));
           }
         }
-      } else if constexpr (kHalfS) {
-        // Per tile and block j: S_t(j) keys [0, 64) as soon as the softmax
-        // holds S_t(j-1) in registers (s_free), then PV_t(j-1) once P_t(j-1)
-        // is in TMEM (p_full), then S_t(j) keys [64, 128) into the columns
-        // that PV_t(j-1) has just read P from (MMAs of one thread run in
-        // issue order).
-        int ns0 = 0, ns1 = 0;
-        constexpr uint32_t kIdescHalf =
-            kF8 ? make_idesc_e4m3(kBM, kBN / 2, 0, 0) : make_idesc_f16(kBM, kBN / 2, DT, 0, 0);
-        auto issue_s_half = [&](int t, int slot, int h) {
-          const uint32_t qlo = t ? q_lo1 : q_lo0;
-          const uint32_t klo =
-              desc_lo(sRing + slot * G::kTileBytes + h * (kBN / 2) * G::kSwBytes, 16);
-          const uint32_t d_tmem = tmem + (t ? 128u : 0u) + (h ? 64u : 0u);
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < D / kKStep; ++kk) {
-              const int byte = kk * 32;
-              const uint32_t off =
-                  ((byte / G::kSwBytes) * G::kBoxBytes + (byte % G::kSwBytes)) >> 4;
-              mma_ss_t<kF8>(d_tmem, desc_join(qlo + off, kHi), desc_join(klo + off, kHi),
-                            kIdescHalf, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(smem_u32(h ? &bars->s_full[t] : &bars->s_lo_full[t]));
-          }
-          __syncwarp();
-        };
-        auto tile_step = [&](int t, int j, int q) -> bool {
-          const bool cur = j < hi && in(t, j);
-          if (cur) {
-            const int ns = t ? ns1 : ns0;
-            if (ns > 0) {
-              if (!mbar_wait_warp(smem_u32(&bars->s_free[t]), (ns - 1) & 1, abort_flag))
-                return false;
-              tc_fence_after_sync();
-            }
-            issue_s_half(t, kslot(q), 0);
-          }
-          if (j > lo && in(t, j - 1)) {
-            if (!mbar_wait_warp(smem_u32(&bars->full[vslot(q - 1)]), vpar(q - 1), abort_flag) ||
-                !mbar_wait_warp(smem_u32(&bars->p_full[t]), (t ? npv1 : npv0) & 1, abort_flag))
-              return false;
-            tc_fence_after_sync();
-            issue_pv(t, vslot(q - 1));
-          }
-          if (cur) {
-            issue_s_half(t, kslot(q), 1);
-            if (t) ++ns1; else ++ns0;
-          }
-          return true;
-        };
-        for (int j = lo; j <= hi && ok; ++j) {
-          const int q = j - lo;
-          if (j < hi) {
-            ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
-            if (!ok) break;
-            tc_fence_after_sync();
-          }
-          ok = tile_step(0, j, q) && tile_step(1, j, q);
-          if (!ok) break;
-          if (j < hi) commit(smem_u32(&bars->empty[kslot(q)]));
-          if (j > lo) commit(smem_u32(&bars->empty[vslot(q - 1)]));
-        }
       } else {
       // D > 64, two tiles: ping-pong
       for (int j = lo; j < hi && ok; ++j) {
@@ -807,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   }
   } else {
     // =================================================== softmax / epilogue
-    regs_inc<RegSplit<D, DT, kHalfS>::kBig>();
+    regs_inc<RegSplit::kBig>();
     // warpgroup t: the softmax of query tile t, or (kDual) of keys
     // [64t, 64t + 64) of every block of tile 0
     const int t = warp >> 2;
@@ -833,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     // query ranges: decoding) skips its loads, exponentials and P stores but
     // keeps every wait and arrival, so the barrier phases stay in step.
     // Its P rows are never written; PV then fills O rows that no one stores.
-    const bool idle_warp = (kDual || kHalfS) && !__any_sync(0xffffffffu, r_loc < trows);
+    const bool idle_warp = kDual && !__any_sync(0xffffffffu, r_loc < trows);
     const int row_lo = p.wl < 0 ? 0 : i - p.wl;
     const int row_hi = p.wr < 0 ? p.L_k - 1 : min(p.L_k - 1, i + p.wr);
     const int first = tq0, last = tq0 + trows - 1;
@@ -857,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       for (int n = 0; n < n_blocks; ++n) {
         const int j = tlo + n;
         ok = mbar_wait_warp(
-            smem_u32(kHalfS ? &bars->s_lo_full[t] : &bars->s_full[tt]), n & 1, abort_flag);
+            smem_u32(&bars->s_full[tt]), n & 1, abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
 
@@ -889,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         };
         const float2 sl2v = make_float2(sl2, sl2);
 
-        // 64-key helpers of the half-S and dual schedules
+        // 64-key helpers of the dual schedule
         float alpha = 1.0f;
         bool rescaled = false;
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -1038,12 +950,6 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             const bool got = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n - 1) & 1, abort_flag);
             ok = ok && got;
           }
-        } else if (kHalfS && idle_warp) {
-          ok = mbar_wait_warp(smem_u32(&bars->s_full[t]), n & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after_sync();
-          tc_fence_before_sync();
-          mbar_arrive(smem_u32(&bars->s_free[t]));
         } else if constexpr (kDual) {
           // keys [64t, 64t + 64) of this block: max first, then free S (both
           // warpgroups arrive) for the next block's S MMA, then P_t
@@ -1119,44 +1025,6 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             store_p_half<DT>(tPs, 1, pk[1]);
             if (warp_rescale && n > 0) scale_o_row<D>(tO, alpha);
           }
-        } else if constexpr (kHalfS) {
-          // D > 64, one tile: the block in two 64-key halves.  Keys [0, 64) arrive
-          // first (s_lo_full) and their exponentials run while the tensor
-          // pipe does PV_t(j-1) and keys [64, 128) (s_full).  Each half takes
-          // its maximum first, then the conditional rescale, then P.  P_t is
-          // stored over columns [64, 128) of S_t once both halves are in
-          // registers; S_t is freed for the next block's first half then.
-          uint32_t pk[2][32];
-          {
-            float sv[kBN / 2];
-            load64(tS, j * kBN, sv);
-            raise(half_max(sv));
-            exp_any(sv, pk[0]);
-          }
-          // keys [64, 128): issued after PV_t(j-1), so O_t holds blocks < j
-          // and P_t(j-1) has been read once this wait returns
-          ok = mbar_wait_warp(smem_u32(&bars->s_full[t]), n & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after_sync();
-          {
-            float sv[kBN / 2];
-            load64(tS + 64, j * kBN + 64, sv);
-            if (raise(half_max(sv))) {
-              // the first half's P used the old reference: redo it from
-              // S_t keys [0, 64), still in TMEM until s_free
-              float s0[kBN / 2];
-              load64(tS, j * kBN, s0);
-              ls[0] = ls[1] = make_float2(0.f, 0.f);
-              exp_any(s0, pk[0]);
-            }
-            tc_fence_before_sync();
-            mbar_arrive(smem_u32(&bars->s_free[t]));
-            store_p_half<DT>(tS + 64, 0, pk[0]);
-            exp_any(sv, pk[1]);
-          }
-          l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
-          if (rescaled && n > 0) scale_o_row<D>(tO, alpha);
-          store_p_half<DT>(tS + 64, 1, pk[1]);
         } else {
         // D > 64, two tiles.  Speculative pass (unmasked blocks, once every row has a reference
         // max): P = 2^(s*scale*log2e - m_use) against the current reference
@@ -1314,14 +1182,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 #pragma unroll
           for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
-            if (n_blocks > 0) {
-              tmem_ld_x32(tO + c, o);
-              tmem_wait_ld();
-              reg_dep(o);
-            } else {
-#pragma unroll
-              for (int u = 0; u < 32; ++u) o[u] = 0u;
-            }
+            load_o(c, std::integral_constant<int, 32>{}, o);   // kDual: both halves merged
             if (r_loc < trows) {
 #pragma unroll
               for (int u = 0; u < 4; ++u)
