@@ -931,7 +931,7 @@ int launch_bwd(const BwdParams &prm, const void *out, const void *dout, const fl
   kern<<<grid, kBwdThreads, BG::kSmemBytes, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const size_t n = static_cast<size_t>(B) * H * prm.L_q * D;
-  const unsigned cblocks = static_cast<unsigned>(std::min<size_t>((n / 2 + 255) / 256, 148 * 16));
+  const unsigned cblocks = static_cast<unsigned>(std::min<size_t>((n / 4 + 255) / 256, 148 * 16));
   fa_bwd_dq_kernel<DT><<<cblocks, 256, 0, stream>>>(prm.dq_acc, dq, n);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

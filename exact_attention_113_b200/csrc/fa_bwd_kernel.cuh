@@ -656,19 +656,28 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const void *out, const
   const int i = static_cast<int>(row - bh * L_q_pad);
   float dsum = 0.0f;
   if (i < L_q) {
+    // 16-byte loads of O and dO (8 elements a lane), 16-byte zero stores of
+    // the fp32 dQ accumulator (4 a lane)
     const size_t base = (static_cast<size_t>(bh) * L_q + i) * D;
-    for (int d = lane; d < D; d += 32) {
-      float o, g;
-      if constexpr (DT == 0) {
-        o = __half2float(reinterpret_cast<const __half *>(out)[base + d]);
-        g = __half2float(reinterpret_cast<const __half *>(dout)[base + d]);
-      } else {
-        o = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(out)[base + d]);
-        g = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(dout)[base + d]);
+    for (int u = lane; u < D / 8; u += 32) {
+      const uint4 ow = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(out) + base)[u];
+      const uint4 gw = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(dout) + base)[u];
+      const uint32_t os[4] = {ow.x, ow.y, ow.z, ow.w}, gs[4] = {gw.x, gw.y, gw.z, gw.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float2 o, g;
+        if constexpr (DT == 0) {
+          o = __half22float2(*reinterpret_cast<const __half2 *>(&os[k]));
+          g = __half22float2(*reinterpret_cast<const __half2 *>(&gs[k]));
+        } else {
+          o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&os[k]));
+          g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gs[k]));
+        }
+        dsum = fmaf(o.x, g.x, fmaf(o.y, g.y, dsum));
       }
-      dsum = fmaf(o, g, dsum);
-      dq_acc[base + d] = 0.0f;
     }
+    for (int u = lane; u < D / 4; u += 32)
+      reinterpret_cast<float4 *>(dq_acc + base)[u] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
@@ -687,11 +696,13 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const void *out, const
 template <int DT>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const float *dq_acc, void *dq,
                                                         size_t n) {
-  size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
-  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x * 2;
+  // n is a multiple of 16 (rows of D elements, D a multiple of 16): 16-byte
+  // loads, 8-byte stores
+  size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x * 4;
   for (; i < n; i += stride) {
-    const float2 v = *reinterpret_cast<const float2 *>(dq_acc + i);
-    reinterpret_cast<uint32_t *>(dq)[i / 2] = pack2<DT>(v.x, v.y);
+    const float4 v = *reinterpret_cast<const float4 *>(dq_acc + i);
+    reinterpret_cast<uint2 *>(dq)[i / 4] = make_uint2(pack2<DT>(v.x, v.y), pack2<DT>(v.z, v.w));
   }
 }
 
