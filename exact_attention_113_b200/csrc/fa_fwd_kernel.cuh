@@ -603,30 +603,31 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         for (int j = lo; j <= hi && ok; ++j) {
           const int q = j - lo;
           if (j < hi) {
-            ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
+            if (ns > 0) {
+              const uint32_t b2[2] = {smem_u32(&bars->full[kslot(q)]), smem_u32(&bars->s_free[0])};
+              const uint32_t p2[2] = {kpar(q), static_cast<uint32_t>((ns - 1) & 1)};
+              ok = mbar_wait_all(b2, p2, abort_flag);
+            } else {
+              ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
+            }
             if (!ok) break;
             tc_fence_after_sync();
-            if (ns > 0) {
-              ok = mbar_wait_warp(smem_u32(&bars->s_free[0]), (ns - 1) & 1, abort_flag);
-              if (!ok) break;
-              tc_fence_after_sync();
-            }
             issue_s(0, kslot(q));
             ++ns;
             commit(smem_u32(&bars->empty[kslot(q)]));
           }
           if (j > lo) {
-            ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q - 1)]), vpar(q - 1), abort_flag);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              ok = ok && mbar_wait_warp(smem_u32(&bars->p_full[h]), (h ? npv1 : npv0) & 1,
-                                        abort_flag);
-              if (ok) {
-                tc_fence_after_sync();
-                issue_pv_h(h, vslot(q - 1));
-              }
-            }
+            // V(j-1) and both halves' P(j-1): the two halves finish within a
+            // few tens of cycles of each other, so one wait covers both
+            const uint32_t b3[3] = {smem_u32(&bars->full[vslot(q - 1)]),
+                                    smem_u32(&bars->p_full[0]), smem_u32(&bars->p_full[1])};
+            const uint32_t p3[3] = {vpar(q - 1), static_cast<uint32_t>(npv0 & 1),
+                                    static_cast<uint32_t>(npv1 & 1)};
+            ok = mbar_wait_all(b3, p3, abort_flag);
             if (!ok) break;
+            tc_fence_after_sync();
+            issue_pv_h(0, vslot(q - 1));
+            issue_pv_h(1, vslot(q - 1));
             commit(smem_u32(&bars->empty[vslot(q - 1)]));
           }
         }
@@ -673,17 +674,17 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
       } else {
       // D > 64, two tiles: ping-pong
+      // The fills of K(j+1) and V(j) are waited for at the end of block j,
+      // before the wait for P0(j) (the one that really waits), so that
+      // PV0(j) and S0(j+1) issue back to back and PV1(j) waits only for P1.
+      ok = mbar_wait_warp(smem_u32(&bars->full[kslot(0)]), kpar(0), abort_flag);
+      if (ok) tc_fence_after_sync();
       for (int j = lo; j < hi && ok; ++j) {
         const int q = j - lo;
-        ok = mbar_wait_warp(smem_u32(&bars->full[kslot(q)]), kpar(q), abort_flag);
-        if (!ok) break;
-        tc_fence_after_sync();
         if (in(0, j)) issue_s(0, kslot(q));
         if (j > lo) {
           if (in(1, j - 1)) {
-            ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q - 1)]), vpar(q - 1),
-                                abort_flag) &&
-                 mbar_wait_warp(smem_u32(&bars->p_full[1]), npv1 & 1, abort_flag);
+            ok = mbar_wait_warp(smem_u32(&bars->p_full[1]), npv1 & 1, abort_flag);
             if (!ok) break;
             tc_fence_after_sync();
             issue_pv(1, vslot(q - 1));
@@ -692,19 +693,23 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
         if (in(1, j)) issue_s(1, kslot(q));
         commit(smem_u32(&bars->empty[kslot(q)]));
+        ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q)]), vpar(q), abort_flag) &&
+             (j + 1 >= hi ||
+              mbar_wait_warp(smem_u32(&bars->full[kslot(q + 1)]), kpar(q + 1), abort_flag));
+        if (!ok) break;
         if (in(0, j)) {
-          ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q)]), vpar(q), abort_flag) &&
-               mbar_wait_warp(smem_u32(&bars->p_full[0]), npv0 & 1, abort_flag);
+          ok = mbar_wait_warp(smem_u32(&bars->p_full[0]), npv0 & 1, abort_flag);
           if (!ok) break;
           tc_fence_after_sync();
           issue_pv(0, vslot(q));
+        } else {
+          tc_fence_after_sync();
         }
       }
       if (ok) {
         const int q = hi - 1 - lo;
         if (in(1, hi - 1)) {
-          ok = mbar_wait_warp(smem_u32(&bars->full[vslot(q)]), vpar(q), abort_flag) &&
-               mbar_wait_warp(smem_u32(&bars->p_full[1]), npv1 & 1, abort_flag);
+          ok = mbar_wait_warp(smem_u32(&bars->p_full[1]), npv1 & 1, abort_flag);
           if (ok) {
             tc_fence_after_sync();
             issue_pv(1, vslot(q));

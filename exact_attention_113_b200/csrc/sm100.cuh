@@ -98,6 +98,29 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// Waits until every listed phase has completed.  The barriers are first
+// probed together (non-blocking test_wait, so their latencies overlap);
+// only the ones not yet complete are then waited for one by one.
+template <int N>
+__device__ __forceinline__ bool mbar_wait_all(const uint32_t (&bar)[N], const uint32_t (&par)[N],
+                                              volatile int *abort_flag) {
+  uint32_t done[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done[i])
+        : "r"(bar[i]), "r"(par[i])
+        : "memory");
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (!done[i]) ok = ok && mbar_wait(bar[i], par[i], abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // One lane of a converged warp: the same lane (the lowest active) every time.
 __device__ __forceinline__ bool elect_one() {
   uint32_t e;
