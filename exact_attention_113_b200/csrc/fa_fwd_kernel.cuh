@@ -13,7 +13,8 @@
 //   warps 0-3   softmax warpgroup for query tile 0 (rows q0 .. q0+127)
 //   warps 4-7   softmax warpgroup for query tile 1 (rows q0+128 .. q0+255)
 //   warp  8     MMA issuer (one elected thread) and TMEM owner
-//   warp  9     TMA producer of Q and K (one elected thread)
+//   warp  9     TMA producer of K (one elected thread; thread 0 requests the Q
+//               tiles and the first K block during setup)
 //   warp  10    TMA producer of V (one elected thread)
 //   warp  11    idle
 // Each softmax thread owns one query row, which is one TMEM lane.
@@ -428,14 +429,42 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     mbar_init(smem_u32(&bars->mma_done), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
+    // The Q tiles and the first K block are requested right here, so that
+    // their latency overlaps the TMEM allocation and the block-wide barrier
+    // (the K producer starts at the second block).
+    if (any_work) {
+      const uint32_t sQ0 = smem_u32(smem + G::kOffQ);
+      const uint64_t pol_stream = policy_evict_first();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (rng[t].hi <= rng[t].lo) continue;
+        const uint32_t bar = smem_u32(&bars->q_full[t]);
+        mbar_arrive_expect_tx(bar, G::kTileBytes);
+#pragma unroll
+        for (int bx = 0; bx < G::kNumBox; ++bx)
+          tma_load_3d(sQ0 + t * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, bar,
+                      bx * G::kBoxCols, q0[t], bh, pol_stream);
+      }
+#ifdef FA_TEST_HOOKS
+      const bool withhold_first = blockIdx.x == 0 && g_fa_test_withhold_block == lo;
+#else
+      constexpr bool withhold_first = false;
+#endif
+      if (!withhold_first) {
+        const uint32_t bar = smem_u32(&bars->full[0]);
+        mbar_arrive_expect_tx(bar, G::kTileBytes);
+#pragma unroll
+        for (int bx = 0; bx < G::kNumBox; ++bx)
+          tma_load_3d(smem_u32(smem + G::kOffRing) + bx * G::kBoxBytes, &p.tm_k, bar,
+                      bx * G::kBoxCols, lo * kBN, bh_kv, policy_evict_last());
+      }
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
     tmem_relinquish();
   }
   if (warp == kLoadWarp && lane == 0) {
-    prefetch_tensormap(&p.tm_q);
-    prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
     prefetch_tensormap(&p.tm_o);
   }
@@ -452,28 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   regs_dec<RegSplit::kSmall>();
   if (warp == kLoadWarp || warp == kLoadWarpV) {
     // =================================================== TMA producers
-    // Warp 9 loads Q and the K ring, warp 10 the V ring.  The whole warp
-    // walks the schedule (its operands stay warp-uniform); one elected lane
-    // issues each copy.
+    // Warp 9 loads the K ring (from its second block), warp 10 the V ring.
+    // The whole warp walks the schedule (its operands stay warp-uniform);
+    // one elected lane issues each copy.
     if (any_work) {
       const bool is_k = warp == kLoadWarp;
-      const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
-      if (is_k) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (rng[t].hi <= rng[t].lo) continue;
-          const uint32_t bar = smem_u32(&bars->q_full[t]);
-          if (elect_one()) {
-            mbar_arrive_expect_tx(bar, G::kTileBytes);
-#pragma unroll
-            for (int bx = 0; bx < G::kNumBox; ++bx)
-              tma_load_3d(sQ + t * G::kTileBytes + bx * G::kBoxBytes, &p.tm_q, bar,
-                          bx * G::kBoxCols, q0[t], bh, pol_stream);
-          }
-          __syncwarp();
-        }
-      }
       const int nslot = is_k ? G::kSlotsK : G::kSlotsV;
       const int base = is_k ? 0 : G::kSlotsK;           // first slot of this ring
       const CUtensorMap *map = is_k ? &p.tm_k : &p.tm_v;
@@ -485,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       constexpr int withheld = -1;
 #endif
       for (int j = lo; j < hi; ++j, ++q) {
+        if (is_k && q == 0) continue;   // the first K block: requested at setup
         const int slot = base + q % nslot;
         if (q >= nslot) {
           ok = mbar_wait_warp(smem_u32(&bars->empty[slot]), ((q / nslot) - 1) & 1, abort_flag);
@@ -1220,7 +1234,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           tma_store_3d(&p.tm_o, smem_u32(stage + bx * G::kBoxBytes), bx * G::kBoxCols, tq0,
                        bh);
         bulk_commit_group();
-        bulk_wait_group_all();
+        bulk_wait_group_read_all();   // the staging tile has been read
       }
       }   // 16-bit output through TMA
       if (ok && p.smax != nullptr && r_loc < trows) {
