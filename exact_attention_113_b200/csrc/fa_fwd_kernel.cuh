@@ -970,16 +970,35 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             ok = ok && got;
           }
         } else if constexpr (kDual) {
-          // keys [64t, 64t + 64) of this block: max first, then free S (both
-          // warpgroups arrive) for the next block's S MMA, then P_t
+          // keys [64t, 64t + 64) of this block: free S (both warpgroups
+          // arrive) for the next block's S MMA as soon as it is in
+          // registers, then P_t.  Unmasked blocks, once every row of the
+          // warp has a reference max, take the exponentials against that
+          // reference while the half max is reduced alongside (as the
+          // ping-pong's speculative pass); if some row's max grew by more
+          // than 2^8 they are redone after the rescale.
           float sv[kBN / 2];
           load64(tS, j * kBN + 64 * t, sv);
-          const float m_half = half_max(sv);
           tc_fence_before_sync();
           mbar_arrive(smem_u32(&bars->s_free[0]));
-          raise(m_half);
           uint32_t pk[32];
-          exp_any(sv, pk);
+          bool spec_ok = false;
+          if (full && __all_sync(0xffffffffu, m_use != -INFINITY)) {
+            const float m_half = half_max(sv);
+            exp_half(sv, pk, std::true_type{});
+            m_true = fmaxf(m_true, m_half);
+            spec_ok = !__any_sync(0xffffffffu, m_half > m_use + kRescaleThreshold);
+            if (!spec_ok) {
+              ls[0] = make_float2(0.f, 0.f);
+              ls[1] = make_float2(0.f, 0.f);
+              raise(m_half);
+              exp_half(sv, pk, std::true_type{});
+            }
+          } else {
+            const float m_half = half_max(sv);
+            raise(m_half);
+            exp_any(sv, pk);
+          }
           l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
           // P_t and O_t are read / written by PV_t(j-1): wait for it
           if (n > 0) {
