@@ -485,6 +485,12 @@ def run_ours(args, w: W.Workload):
     pci = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
     with ClockSampler(physical_gpu_index(dev.index), pci) as clk:
         time.sleep(0.3)                    # let the sampler start
+        # the GPU idled during that pause: warm it up again right before the
+        # timed steps, or the first of them pays for the wake-up
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                step()
+        torch.cuda.synchronize(dev)
         barrier(world, dev)
         torch.cuda.synchronize(dev)
         clk.mark_start()
