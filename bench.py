@@ -486,9 +486,12 @@ def run_ours(args, w: W.Workload):
     with ClockSampler(physical_gpu_index(dev.index), pci) as clk:
         time.sleep(0.3)                    # let the sampler start
         # the GPU idled during that pause: warm it up again right before the
-        # timed steps, or the first of them pays for the wake-up
+        # timed steps (the same sequence as a timed step, flush included), or
+        # the first of them pays for the wake-up
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
+                if flush is not None:
+                    flush.fill_(0.0)
                 step()
         torch.cuda.synchronize(dev)
         barrier(world, dev)

@@ -1012,8 +1012,13 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           }
         } else if constexpr (G::kSplitP) {
           // row max first, then free S_t for the next block's S MMA, then P
+          // (D = 16: S_t is freed right after its load, before the max)
           float s[kBN];
           load_s(s);
+          if constexpr (D <= 16) {
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&bars->s_free[t]));
+          }
           float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
           for (int c = 4; c < kBN - 4; c += 8)
@@ -1022,8 +1027,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           const float m_blk = fmax3(fmax3(mx[0], mx[1], s[kBN - 4]),
                                     fmax3(mx[2], mx[3], s[kBN - 3]),
                                     fmaxf(s[kBN - 2], s[kBN - 1]));
-          tc_fence_before_sync();
-          mbar_arrive(smem_u32(&bars->s_free[t]));
+          if constexpr (D > 16) {
+            tc_fence_before_sync();
+            mbar_arrive(smem_u32(&bars->s_free[t]));
+          }
           const float m_new = (m_blk == -INFINITY) ? -INFINITY : m_blk * sl2;
           m_true = fmaxf(m_true, m_new);
           const bool need = m_new > m_use + kRescaleThreshold;
