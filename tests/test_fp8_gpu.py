@@ -137,9 +137,9 @@ def test_fp8_splitkv_matches_single_pass():
 
 
 # ------------------------------------------------------------ both D = 128 schedules
-# One query tile per CTA (fewer 128-row tiles than SMs) takes the half-S
-# schedule, more tiles the two-tile ping-pong: B 2 x H 40 at L_q 300 is 240
-# tiles (ping-pong), B 1 x H 3 is 9 (half-S).  std 3 moves the running max
+# One query tile per CTA (fewer 128-row tiles than SMs) takes the dual
+# softmax, more tiles the two-tile ping-pong: B 2 x H 40 at L_q 300 is 240
+# tiles (ping-pong), B 1 x H 3 is 9 (dual).  std 3 moves the running max
 # past the rescale threshold inside blocks.
 @pytest.mark.parametrize("shape", ["two", "one"])
 @pytest.mark.parametrize("causal,std", [(False, 1.0), (True, 1.0), (False, 3.0)])

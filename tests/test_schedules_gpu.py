@@ -9,12 +9,14 @@ schedule follows:
   halves of every block, each with its own running max, sum and O, merged
   at the end); with one real query row in a warp's 32, the other warps
   skip their exponentials.
-(fp8 one-tile D = 128 takes the half-S schedule; tests/test_fp8_gpu.py.)
+(fp8 one-tile CTAs take the dual softmax too; tests/test_fp8_gpu.py.)
 Every case is sized on one side of the tile-count line: TWO = B 2 x H 40 at
-L_q 300 is 240 tiles, ONE = B 1 x H 3 is 9 tiles.  Large-variance inputs (std 3: scaled scores of spread ~9,
-~13 in log2 units) make the running maximum move past the rescale threshold
-inside blocks, including between a block's two halves, which is the rare
-path of the half-S softmax (P of the first half recomputed)."""
+L_q 300 is 240 tiles, ONE = B 1 x H 3 is 9 tiles.  Large-variance inputs
+(std 3: scaled scores of spread ~9, ~13 in log2 units) make the running
+maximum move past the rescale threshold inside blocks: the rare path of the
+speculative passes (exponentials taken against the running reference are
+dropped and redone after the rescale), in the ping-pong and the dual
+softmax alike."""
 import numpy as np
 import pytest
 import torch
@@ -46,7 +48,7 @@ def test_both_schedules(shape, D, dtype, causal):
 
 
 @pytest.mark.parametrize("shape", ["two", "one"])
-@pytest.mark.parametrize("D", [32, 64, 96, 128])
+@pytest.mark.parametrize("D", [16, 32, 64, 96, 128])
 def test_rescale_heavy(shape, D):
     check_full(_w(shape, D=D, L_q=400, L_k=900, std=3.0, seed=9100 + D), derived=True)
 
