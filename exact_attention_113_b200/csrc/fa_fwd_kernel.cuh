@@ -1044,10 +1044,13 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           }
           const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
           const float2 negm = make_float2(-m_sub, -m_sub);
-          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          // P = 2^(s*scale*log2e - m); at D <= 32 the two halves of the row
+          // are interleaved (more independent exponentials in flight: the
+          // softmax warps are the whole cost there), else in column order
+          float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
           uint32_t pk[2][32];
-#pragma unroll
-          for (int c = 0; c < kBN; c += 2) {
+          auto exp_pair = [&](int c, float2 &acc) {
             const int pair = c >> 1;
             const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2v, negm);
             float2 pp;
@@ -1055,10 +1058,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
               pp = exp2_poly2(x);
             else
               pp = make_float2(ex2(x.x), ex2(x.y));
-            ls[pair & 1] = __fadd2_rn(ls[pair & 1], pp);
+            acc = __fadd2_rn(acc, pp);
             put_p<DT>(pk[c >> 6], pair & 31, pp.x, pp.y);
+          };
+          if constexpr (D <= 32) {
+#pragma unroll
+            for (int c0 = 0; c0 < kBN / 2; c0 += 2) {
+              exp_pair(c0, ls[(c0 >> 1) & 1]);
+              exp_pair(c0 + kBN / 2, ls[2 + ((c0 >> 1) & 1)]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kBN; c += 2) exp_pair(c, ls[(c >> 1) & 1]);
           }
-          l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+          l += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
           // P_t and O_t are read / written by PV_t(j-1): wait for it
           if (n > 0) {
             const bool got = mbar_wait_warp(smem_u32(&bars->pv_done[t]), (n - 1) & 1, abort_flag);
