@@ -67,14 +67,17 @@ CASES = [
 ]
 
 
+# block 2 is requested by the K producer warp; block 0 (the CTA's first) by
+# thread 0 during set-up, before the block-wide barrier
+@pytest.mark.parametrize("withheld", [2, 0])
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
-def test_withheld_copy_ends_the_launch_with_a_timeout(hooks, w):
+def test_withheld_copy_ends_the_launch_with_a_timeout(hooks, w, withheld):
     q, k, v = (t.cuda() for t in make_qkv(w))
     out = torch.full_like(q, float("nan"))
     lse = torch.full((w.B, w.H, w.L_q), float("nan"), device="cuda")
     assert hooks.fa_get_device_status(None) == FA_OK       # nothing pending
     # CTA 0 covers the first query tile(s) of head 0: key blocks 0 .. 7
-    assert hooks.fa_test_set_withhold(2) == FA_OK
+    assert hooks.fa_test_set_withhold(withheld) == FA_OK
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     stream = _launch(hooks, w, q, k, v, out, lse)
