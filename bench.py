@@ -485,14 +485,13 @@ def run_ours(args, w: W.Workload):
     pci = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
     with ClockSampler(physical_gpu_index(dev.index), pci) as clk:
         time.sleep(0.3)                    # let the sampler start
-        # the GPU idled during that pause: warm it up again right before the
-        # timed steps (the same sequence as a timed step, flush included), or
-        # the first of them pays for the wake-up
+        # the GPU idled during that pause: one more untimed step right before
+        # the timed ones (the same sequence as a timed step, flush included),
+        # or the first of them pays for the wake-up
         with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                if flush is not None:
-                    flush.fill_(0.0)
-                step()
+            if flush is not None:
+                flush.fill_(0.0)
+            step()
         torch.cuda.synchronize(dev)
         barrier(world, dev)
         torch.cuda.synchronize(dev)
