@@ -133,6 +133,44 @@ int launch_kernel(const FwdParams &prm, int B, int H, cudaStream_t stream) {
     }
   }
   const unsigned items = static_cast<unsigned>(B) * (prm.packed ? prm.H_kv : H);
+  if (prm.bal) {
+    // balanced one-wave schedule: clusters of two CTAs, all resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * items * static_cast<unsigned>(prm.bal_cpi), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = G::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static int max_clusters[64] = {};   // per device: pairs resident at once (0: not known)
+    int mc = 0;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (max_clusters[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+          cudaGetLastError();
+          n = -1;
+        }
+        max_clusters[dev] = n;
+      }
+      mc = max_clusters[dev];
+    }
+    if (mc >= static_cast<int>(items) * prm.bal_cpi) {
+      if (cudaLaunchKernelEx(&cfg, kern, prm) != cudaSuccess) return FA_ERR_CUDA;
+      return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
+    FwdParams plain = prm;                // the pairs would not all fit: plain grid
+    plain.bal = 0;
+    dim3 grid(static_cast<unsigned>(plain.n_qpairs) * items, 1, 1);
+    kern<<<grid, kThreads, G::kSmemBytes, stream>>>(plain);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
   dim3 grid(static_cast<unsigned>(prm.n_qpairs) * items * static_cast<unsigned>(prm.n_splits),
             1, 1);
   kern<<<grid, kThreads, G::kSmemBytes, stream>>>(prm);
@@ -486,6 +524,49 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
   prm.wl = wl;
   prm.wr = wr;
   prm.reverse = (wr >= 0) ? 1 : 0;         // later query tiles see more keys
+  // Balanced one-wave schedule: with one tile per CTA (a single wave) and
+  // uneven key ranges (causal, windows), the kernel time is the longest
+  // tile's.  Tiles with more than half the longest range's key blocks are
+  // then split between the two CTAs of a cluster pair, which merge their
+  // (m, l, O) in shared memory; the other tiles run alone, two clusters'
+  // worth at a time.  Only when every CTA still fits in one wave.
+  if (prm.tiles == 1 && n_splits <= 0 && !prm.packed && dtype != kE4M3) {
+    const int n_t = static_cast<int>(q_tiles);
+    int nb[kBalMaxEntries * 2];
+    int nb_max = 0;
+    if (n_t <= kBalMaxEntries * 2) {
+      for (int tq = 0; tq < n_t; ++tq) {
+        const int first = tq * kBM, last = std::min(L_q, first + kBM) - 1;
+        const int klo = wl < 0 ? 0 : std::max(0, first - wl);
+        const int khi = wr < 0 ? L_k - 1 : std::min(L_k - 1, last + wr);
+        nb[tq] = khi < klo ? 0 : khi / kBN - klo / kBN + 1;
+        nb_max = std::max(nb_max, nb[tq]);
+      }
+    }
+    // (at most 1024 blocks: the pair's hand-off waits are bounded by the
+    // device wait limit, far above the time such a slice takes)
+    if (nb_max >= 4 && nb_max <= 1024) {
+      int heavy[kBalMaxEntries * 2], light[kBalMaxEntries * 2];
+      int n_heavy = 0, n_light = 0;
+      for (int tq = 0; tq < n_t; ++tq) {
+        if (2 * nb[tq] > nb_max + 1)
+          heavy[n_heavy++] = tq;
+        else
+          light[n_light++] = tq;
+      }
+      const int cpi = n_heavy + (n_light + 1) / 2;
+      if (n_heavy > 0 && cpi <= kBalMaxEntries && 2 * items * cpi <= sm_count()) {
+        int e = 0;
+        for (int h = n_heavy - 1; h >= 0; --h)     // heaviest first
+          prm.bal_desc[e++] = static_cast<uint32_t>(heavy[h]) | (0xffu << 8) | (1u << 16);
+        for (int i2 = 0; i2 < n_light; i2 += 2)
+          prm.bal_desc[e++] = static_cast<uint32_t>(light[i2]) |
+                              (static_cast<uint32_t>(i2 + 1 < n_light ? light[i2 + 1] : 0xff) << 8);
+        prm.bal = 1;
+        prm.bal_cpi = cpi;
+      }
+    }
+  }
   {
     float sl2 = scale * 1.4426950408889634f;
     prm.scale_log2 = sl2 < 1e-30f ? 1e-30f : sl2;

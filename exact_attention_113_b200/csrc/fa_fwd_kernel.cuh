@@ -81,6 +81,7 @@ constexpr int kLoadWarp = 9;     // Q and K
 constexpr int kLoadWarpV = 10;   // V
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
+constexpr int kBalMaxEntries = 74;         // cluster pairs per item: at most 148 CTAs
 
 #ifdef FA_TEST_HOOKS
 // Watchdog test library only (never in libfa.so): the K producer of CTA 0
@@ -132,6 +133,15 @@ struct FwdParams {
   // of the scaled, masked scores and sum_j e^{s_j - max}; nullptr = skip
   float *smax;
   float *ssum;
+  // balanced one-wave schedule (bal != 0, one tile per CTA, launched as
+  // clusters of two CTAs): cluster c serves item c / bal_cpi with entry
+  // bal_desc[c % bal_cpi] = tile A (bits 0-7) | tile B (bits 8-15, 0xff:
+  // none) | bit 16 when the pair splits tile A's key blocks (rank 0 the
+  // first half, rank 1 the second, which rank 1 hands to rank 0 through
+  // shared memory); otherwise rank 0 takes tile A and rank 1 tile B alone
+  int bal;
+  int bal_cpi;
+  uint32_t bal_desc[kBalMaxEntries];
 };
 
 // Tile geometry for head dim D and element size ES bytes (2: fp16 / bf16,
@@ -170,7 +180,14 @@ struct Geo {
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
   static constexpr int kBarBytes = 512;
-  static constexpr int kUsed = kOffBar + kBarBytes;
+  // balanced split pairs: the sender's slice (128 fp32 O rows and a
+  // (m, l, max, ok) quadruple per row) lands in a buffer of its own where
+  // the budget leaves room (D <= 64), else in the receiver's K/V ring once
+  // that is idle
+  static constexpr int kPartnerBytes = kBM * (D * 4 + 16);
+  static constexpr int kOffPartner = kOffBar + kBarBytes;
+  static constexpr bool kPartnerOwn = kOffPartner + kPartnerBytes + 1024 <= 232448;
+  static constexpr int kUsed = kOffPartner + (kPartnerOwn ? kPartnerBytes : 0);
   // at least ~116 KB so that only one CTA (and one 512-column TMEM
   // allocation) fits on an SM
   static constexpr int kSmemBytes = (kUsed + 1024 > 118 * 1024) ? kUsed + 1024 : 118 * 1024;
@@ -189,6 +206,9 @@ struct Bars {
   uint64_t p_full[2];
   uint64_t pv_done[2];
   uint64_t mma_done;
+  uint64_t recv_ready;    // balanced pairs, sender: the receiver's ring is free (remote arrival)
+  uint64_t partner_full;  // balanced pairs, receiver: the sender's rows have landed (bytes)
+  uint64_t partner_ack;   // balanced pairs, sender: its copy has landed (remote arrival)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -361,12 +381,27 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   // ---- work item: (batch*head, pair of query tiles, key slice);
   // consecutive CTAs take consecutive query pairs of one head, so a head's
   // K/V stays hot in L2.
-  const int per_item = p.n_qpairs * p.n_splits;
-  const int item = static_cast<int>(blockIdx.x) / per_item;
-  const int rem = static_cast<int>(blockIdx.x) - item * per_item;
-  const int qp_idx = rem / p.n_splits;
-  const int split = rem - qp_idx * p.n_splits;
-  const int qpair = p.reverse ? (p.n_qpairs - 1 - qp_idx) : qp_idx;
+  int item, split, qpair;
+  int bal_role = 0;   // balanced split pair: 1 receives the partner's slice, 2 sends its own
+  if (p.bal) {
+    const int c = static_cast<int>(blockIdx.x) >> 1;
+    item = c / p.bal_cpi;
+    const uint32_t e = p.bal_desc[c - item * p.bal_cpi];
+    const uint32_t rank = cluster_rank();
+    const bool pair_split = (e >> 16) & 1u;
+    int tile = static_cast<int>(pair_split || rank == 0 ? (e & 0xffu) : ((e >> 8) & 0xffu));
+    if (tile == 0xff) tile = p.n_qpairs;   // no tile: rows past L_q, nothing to do
+    qpair = tile;
+    split = 0;
+    if (pair_split) bal_role = rank == 0 ? 1 : 2;
+  } else {
+    const int per_item = p.n_qpairs * p.n_splits;
+    item = static_cast<int>(blockIdx.x) / per_item;
+    const int rem = static_cast<int>(blockIdx.x) - item * per_item;
+    const int qp_idx = rem / p.n_splits;
+    split = rem - qp_idx * p.n_splits;
+    qpair = p.reverse ? (p.n_qpairs - 1 - qp_idx) : qp_idx;
+  }
   // bh: (first) query head of the tile in [B*H]; bh_kv: its K/V head
   int bh, bh_kv;
   if (p.packed) {
@@ -408,6 +443,18 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       if (rng[t].hi <= rng[t].lo) rng[t].lo = rng[t].hi = 0;
     }
   }
+  if (bal_role != 0) {
+    // the pair's shares of the tile's key blocks (the host splits only tiles
+    // with at least three): halves, or, when the sender's rows have a buffer
+    // of their own and their hand-off overlaps the receiver's last blocks,
+    // one more block for the receiver
+    const int nb = rng[0].hi - rng[0].lo;
+    const int mid = rng[0].lo + (G::kPartnerOwn ? (nb + 2) / 2 : (nb + 1) / 2);
+    if (bal_role == 1)
+      rng[0].hi = mid;
+    else
+      rng[0].lo = mid;
+  }
   const bool act0 = rng[0].hi > rng[0].lo, act1 = rng[1].hi > rng[1].lo;
   const int lo = act0 ? (act1 ? min(rng[0].lo, rng[1].lo) : rng[0].lo) : rng[1].lo;
   const int hi = act0 ? (act1 ? max(rng[0].hi, rng[1].hi) : rng[0].hi) : rng[1].hi;
@@ -427,8 +474,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       mbar_init(smem_u32(&bars->empty[s]), 1);
     }
     mbar_init(smem_u32(&bars->mma_done), 1);
+    mbar_init(smem_u32(&bars->recv_ready), 1);
+    mbar_init(smem_u32(&bars->partner_full), 1);
+    mbar_init(smem_u32(&bars->partner_ack), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
+    // a receiver with its own buffer expects the sender's bytes from the start
+    if (kDual && G::kPartnerOwn && bal_role == 1)
+      mbar_arrive_expect_tx(smem_u32(&bars->partner_full), G::kPartnerBytes);
     // The Q tiles and the first K block are requested right here, so that
     // their latency overlaps the TMEM allocation and the block-wide barrier
     // (the K producer starts at the second block).
@@ -469,7 +522,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     prefetch_tensormap(&p.tm_o);
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if (p.bal)
+    cluster_sync_all();   // both CTAs' barriers are initialised before any remote use
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
@@ -734,6 +790,21 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       }   // ping-pong schedule
     }
     if (elect_one()) tc_commit(smem_u32(&bars->mma_done));
+    __syncwarp();
+  } else if (kDual && G::kPartnerOwn && bal_role == 1) {
+    // =================================================== balanced receiver, warp 11
+    // The sender's rows land in this CTA's own buffer whenever the sender
+    // finishes its slice, whatever this CTA is doing; this otherwise idle
+    // warp acknowledges them at once (so that the sender, which waits for
+    // that before leaving, never waits on a CTA that has gone) and holds
+    // this CTA until they have landed.  Bounded by three wait limits: the
+    // sender copies even after its own waits gave up.
+    if (lane == 0) {
+      bool landed = false;
+      for (int k = 0; k < 3 && !landed; ++k)
+        landed = mbar_wait_cluster(smem_u32(&bars->partner_full), 0, abort_flag, false);
+      if (landed) mbar_arrive_cluster(cluster_map(smem_u32(&bars->partner_ack), 1));
+    }
     __syncwarp();
   }
   } else {
@@ -1164,6 +1235,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           m_true = fmaxf(m_true, tb);
         }
       }
+      // balanced split pair: the partner slice's weight and O row (receiver)
+      constexpr int kUnitsO = D / 4;                  // 16-byte units of an fp32 O row
+      float wc = 0.0f;
+      const float4 *prow = nullptr;
       // O row chunk (columns [c, c + W)) into registers; kDual: merged
       auto load_o = [&](int c, auto wd, auto &o) {
         constexpr int W = decltype(wd)::value;
@@ -1178,6 +1253,16 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 #pragma unroll
             for (int u = 0; u < W; ++u)
               o[u] = __float_as_uint(wa * __uint_as_float(o[u]) + wb * __uint_as_float(ob[u]));
+            if (prow != nullptr) {
+#pragma unroll
+              for (int u = 0; u < W / 4; ++u) {
+                const float4 v = prow[(c / 4 + u + r) % kUnitsO];
+                o[4 * u] = __float_as_uint(__uint_as_float(o[4 * u]) + wc * v.x);
+                o[4 * u + 1] = __float_as_uint(__uint_as_float(o[4 * u + 1]) + wc * v.y);
+                o[4 * u + 2] = __float_as_uint(__uint_as_float(o[4 * u + 2]) + wc * v.z);
+                o[4 * u + 3] = __float_as_uint(__uint_as_float(o[4 * u + 3]) + wc * v.w);
+              }
+            }
           } else {
             tmem_wait_ld();
             reg_dep(o);
@@ -1187,8 +1272,106 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           for (int u = 0; u < W; ++u) o[u] = 0u;
         }
       };
+      // Balanced split pair (one tile on the two CTAs of a cluster): the
+      // sender stages its slice's unnormalised O rows and (m, l, exact max)
+      // and copies them into the receiver, one bulk copy per warp of 32
+      // rows; the receiver joins them to its own as two key slices and
+      // acknowledges, after which the sender may leave.  With a buffer of
+      // their own (D <= 64) the rows are staged there and copied at once;
+      // otherwise they are staged in the sender's K/V ring and copied into
+      // the receiver's once the receiver reports it idle (both halves' last
+      // PV complete, which warpgroup 0 knows after the barrier above).  Per
+      // warp the buffer holds its 32 O rows, then their (m, l, exact max,
+      // ok); the units of a row are stored rotated by the row index, so
+      // that a warp's 16-byte accesses spread over the banks.
+      if constexpr (kDual) {
+        constexpr uint32_t kWarpPartBytes = 32 * (D * 4 + 16);
+        constexpr uint32_t kPartnerBytes = 4 * kWarpPartBytes;
+        static_assert(kPartnerBytes == G::kPartnerBytes, "partner buffer size");
+        static_assert(kPartnerBytes <= G::kSlots * G::kTileBytes,
+                      "the partner's rows fit in the K/V ring");
+        if (bal_role != 0 && t == 0) {
+          uint8_t *part = smem + (G::kPartnerOwn ? G::kOffPartner : G::kOffRing) +
+                          (warp & 3) * kWarpPartBytes;   // this warp's rows
+          float4 *prow_w = reinterpret_cast<float4 *>(part) + (r & 31) * kUnitsO;
+          float4 *pml = reinterpret_cast<float4 *>(part + 32 * D * 4) + (r & 31);
+          if (bal_role == 1) {
+            // the receiver: with an own buffer it always waits for the
+            // sender's rows (bounded), so that no copy reaches it after it
+            // has gone; with the ring it first reports the ring idle
+            if constexpr (!G::kPartnerOwn) {
+              if (r == 0 && ok) {
+                mbar_arrive_expect_tx(smem_u32(&bars->partner_full), kPartnerBytes);
+                mbar_arrive_cluster(cluster_map(smem_u32(&bars->recv_ready), 1));
+              }
+            }
+            // (once the go-ahead has gone out, or with an own buffer, the
+            // sender's copy will come: wait for it, bounded, even after an
+            // abort, so that it never lands in a CTA that has gone)
+            bool got = false;
+            if (ok || G::kPartnerOwn)
+              got = mbar_wait_cluster(smem_u32(&bars->partner_full), 0, abort_flag, false);
+            got = __all_sync(0xffffffffu, got);
+            ok = ok && got;
+            if (ok) {
+              const float4 ml = *pml;
+              ok = __all_sync(0xffffffffu, ml.w != 0.0f);   // the sender's warp is uniform
+              const float m = fmaxf(m_use, ml.x);
+              const float sa = (m_use == -INFINITY) ? 0.0f : ex2(m_use - m);
+              wc = (ml.x == -INFINITY) ? 0.0f : ex2(ml.x - m);
+              wa *= sa;
+              wb *= sa;
+              l = sa * l + wc * ml.y;
+              m_use = m;
+              m_true = fmaxf(m_true, ml.z);
+              prow = prow_w;
+            }
+          } else {
+            if (ok) {
+              for_o_chunks<D>([&](int c, auto w) {
+                constexpr int W = decltype(w)::value;
+                uint32_t o[W];
+                load_o(c, w, o);
+#pragma unroll
+                for (int u = 0; u < W / 4; ++u)
+                  prow_w[(c / 4 + u + r) % kUnitsO] =
+                      make_float4(__uint_as_float(o[4 * u]), __uint_as_float(o[4 * u + 1]),
+                                  __uint_as_float(o[4 * u + 2]), __uint_as_float(o[4 * u + 3]));
+              });
+            }
+            *pml = make_float4(m_use, l, m_true, ok ? 1.0f : 0.0f);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              // always copy (the receiver waits for it) and wait (bounded) for
+              // the acknowledgement before leaving: no remote operation may
+              // reach this CTA after it has gone
+              const bool go =
+                  G::kPartnerOwn ||
+                  mbar_wait_cluster(smem_u32(&bars->recv_ready), 0, abort_flag, false);
+              if (go) {
+                bulk_copy_to_cluster(cluster_map(smem_u32(part), 0), smem_u32(part),
+                                     kWarpPartBytes,
+                                     cluster_map(smem_u32(&bars->partner_full), 0));
+                if (r == 0) mbar_wait_cluster(smem_u32(&bars->partner_ack), 0, abort_flag, false);
+              }
+            }
+            __syncwarp();
+          }
+        }
+      }
       if (kDual && t == 1) {
-        // warpgroup 1 is done: warpgroup 0 writes the row
+        // warpgroup 1 is done: warpgroup 0 writes the row.  In a balanced
+        // receiver whose rows land in its K/V ring, its first thread
+        // acknowledges the sender's copy (requested by warpgroup 0 above, so
+        // it lands while this CTA is in its epilogue), off warpgroup 0's path.
+        if constexpr (!G::kPartnerOwn) {
+          if (bal_role == 1 && r == 0 &&
+              mbar_wait_cluster(smem_u32(&bars->partner_full), 0, abort_flag, false))
+            mbar_arrive_cluster(cluster_map(smem_u32(&bars->partner_ack), 1));
+        }
+      } else if (bal_role == 2) {
+        // the receiver writes the row
       } else if (p.ws_o != nullptr) {
         // split-KV partial: unnormalised O (fp32) and (m, l) of this slice.
         // tcgen05.ld is warp-collective: every lane loads (ok and n_blocks
