@@ -528,8 +528,8 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
   // uneven key ranges (causal, windows), the kernel time is the longest
   // tile's.  Tiles with more than half the longest range's key blocks are
   // then split between the two CTAs of a cluster pair, which merge their
-  // (m, l, O) in shared memory; the other tiles run alone, two clusters'
-  // worth at a time.  Only when every CTA still fits in one wave.
+  // (m, l, O) in shared memory; the other tiles run alone, two to a
+  // cluster.  Only when every CTA still fits in one wave.
   if (prm.tiles == 1 && n_splits <= 0 && !prm.packed && dtype != kE4M3) {
     const int n_t = static_cast<int>(q_tiles);
     int nb[kBalMaxEntries * 2];
@@ -555,7 +555,10 @@ int fwd_impl(const void *q, const void *k, const void *v, void *out, float *lse,
           light[n_light++] = tq;
       }
       const int cpi = n_heavy + (n_light + 1) / 2;
-      if (n_heavy > 0 && cpi <= kBalMaxEntries && 2 * items * cpi <= sm_count()) {
+      // only uneven ranges: with every tile as long as the longest, the
+      // pair's hand-off costs about what the halved range saves
+      if (n_heavy > 0 && n_light > 0 && cpi <= kBalMaxEntries &&
+          2 * items * cpi <= sm_count()) {
         int e = 0;
         for (int h = n_heavy - 1; h >= 0; --h)     // heaviest first
           prm.bal_desc[e++] = static_cast<uint32_t>(heavy[h]) | (0xffu << 8) | (1u << 16);

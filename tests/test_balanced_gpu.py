@@ -8,8 +8,8 @@ first CTA takes the first half of the blocks, the second the rest and hands
 its (m, l, O) to the first through distributed shared memory; the first
 merges the two as two key slices and writes the row.  The other tiles run
 alone, two to a cluster.  It applies when the longest range has 4 to 1024
-key blocks and all pairs fit in one wave (2 x items x pairs <= 148 SMs);
-with equal ranges (no mask) every tile is split.
+key blocks, some tiles are not split (uneven ranges) and all pairs fit in
+one wave (2 x items x pairs <= 148 SMs).
 
 Every shape below satisfies that (the comment gives tiles per head, the
 blocks of the longest range and the cluster pairs per head), covering fp16 /
@@ -63,15 +63,6 @@ def test_unequal_lengths_and_odd_light_count():
 def test_window():
     # causal with window_left 700: ranges of up to 7 blocks (the first tiles fewer)
     check_full(_w("bal_win", H=6, H_kv=6, L_q=1536, L_k=1536, window_left=700, seed=9940),
-               derived=True)
-
-
-@pytest.mark.parametrize("D", [64, 128])
-def test_equal_ranges(D):
-    # non-causal: every tile has the longest range, so every tile is split
-    # (8 tiles x 2 heads -> 16 pairs; D = 64 hands over through its own
-    # buffer, D = 128 through the receiver's K/V ring)
-    check_full(_w(f"bal_full_d{D}", H=2, H_kv=2, D=D, causal=False, seed=9945 + D),
                derived=True)
 
 

@@ -11,9 +11,10 @@ issued MMAs and TMEM is freed (the review of every wait and barrier on this
 path is in the design notes).  The test checks that the launch ends within
 the limit's order of magnitude, that fa_get_device_status reports
 FA_ERR_TIMEOUT once, and that the next, normal launch in the same context
-matches the oracle.  Both schedules that end differently are covered: the
-two-tile ping-pong (more query tiles than SMs) and the one-tile dual softmax
-with its cross-warpgroup merge barrier."""
+matches the oracle.  The schedules that end differently are covered: the
+two-tile ping-pong (more query tiles than SMs), the one-tile dual softmax
+with its cross-warpgroup merge barrier, and the balanced pair whose receiver
+gives up while its sender hands over its rows."""
 from __future__ import annotations
 
 import ctypes
@@ -64,6 +65,11 @@ CASES = [
     # a few tiles: one tile per CTA, keys split between two softmax warpgroups
     Workload(name="abort_dual", B=1, H=2, H_kv=2, L_q=1024, L_k=1024, D=64, dtype=F16,
              seed=6002),
+    # causal, a few tiles: the balanced schedule; CTA 0 is the receiver of the
+    # heaviest tile's pair (key blocks 0 .. 4), its sender hands over blocks
+    # 5 .. 7 while the receiver's wait runs out
+    Workload(name="abort_balanced", B=1, H=2, H_kv=2, L_q=1024, L_k=1024, D=64, dtype=F16,
+             causal=True, seed=6003),
 ]
 
 
