@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   // K/V stays hot in L2.
   int item, split, qpair;
   int bal_role = 0;   // balanced split pair: 1 receives the partner's slice, 2 sends its own
-  if (p.bal) {
+  if (kDual && p.bal) {   // (the host sets bal only with one tile per CTA)
     const int c = static_cast<int>(blockIdx.x) >> 1;
     item = c / p.bal_cpi;
     const uint32_t e = p.bal_desc[c - item * p.bal_cpi];
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     prefetch_tensormap(&p.tm_o);
   }
   tc_fence_before_sync();
-  if (p.bal)
+  if (kDual && p.bal)
     cluster_sync_all();   // both CTAs' barriers are initialised before any remote use
   else
     __syncthreads();
