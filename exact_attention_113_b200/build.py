@@ -45,12 +45,22 @@ def is_stale(path: str = LIB_PATH) -> bool:
     return any(os.path.getmtime(p) > t for p in DEPENDS)
 
 
-# The attention kernel launches 384 threads and re-splits its registers with
-# setmaxnreg (2 warpgroups x 224 + 1 x 56 = 384 x 168).  That split is only
-# valid when every instance is compiled at exactly this many registers.
-# kernels whose warpgroups re-split registers with setmaxnreg: the launch
-# allocation (registers per thread) each must be compiled at
+# The forward launches 384 threads and re-splits its registers with
+# setmaxnreg (2 warpgroups x 224 + 1 x 56 = 384 x 168); the backward 768
+# for D <= 64 (4 x 80 + 104 + 56 = 768 x 80) and 512 above (2 x 144 + 168 +
+# 56 = 512 x 128).  A split is only valid when every instance is compiled at
+# exactly its launch allocation (registers per thread).
 LAUNCH_REGS = {"fa_fwd_kernel": 168, "fa_bwd_kernel": 128}
+
+
+def launch_regs(name: str, tag: str) -> int:
+    """The launch allocation of one instance (its mangled name): the
+    backward's depends on its head dim, the first template argument."""
+    if tag == "fa_bwd_kernel":
+        m = re.search(r"fa_bwd_kernelILi(\d+)E", name)
+        if m and int(m.group(1)) <= 64:
+            return 80
+    return LAUNCH_REGS[tag]
 
 
 def check_register_counts(ptxas_log: str) -> dict:
@@ -73,7 +83,7 @@ def check_register_counts(ptxas_log: str) -> dict:
         if not any(tag in k for k in counts):
             raise RuntimeError(f"no register counts found for {tag}")
     bad = {k: v for k, v in counts.items()
-           for tag, want in LAUNCH_REGS.items() if tag in k and v != want}
+           for tag in LAUNCH_REGS if tag in k and v != launch_regs(k, tag)}
     if bad:
         raise RuntimeError(f"register counts differ from the launch allocation "
                            f"{LAUNCH_REGS}: {bad}; the setmaxnreg split would not match")

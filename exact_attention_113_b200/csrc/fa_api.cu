@@ -1003,6 +1003,13 @@ int launch_bwd(const BwdParams &prm, const void *out, const void *dout, const fl
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BG::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
+      // the warpgroups' setmaxnreg budgets add up to exactly the launch
+      // allocation the kernel was built with; any other count would leave
+      // the drain's increase waiting for registers that never come free
+      cudaFuncAttributes fa_attr{};
+      if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess ||
+          fa_attr.numRegs != static_cast<int>(BwdCfg<D>::kLaunchRegs))
+        return FA_ERR_CUDA;
       configured[dev] = true;
     }
   }
@@ -1012,7 +1019,7 @@ int launch_bwd(const BwdParams &prm, const void *out, const void *dout, const fl
       prm.dq_acc, prm.L_q, prm.L_q_pad, rows_pad);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(B) * prm.H_kv * prm.n_kblocks;
-  kern<<<grid, kBwdThreads, BG::kSmemBytes, stream>>>(prm);
+  kern<<<grid, BwdCfg<D>::kThreads, BG::kSmemBytes, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const size_t n = static_cast<size_t>(B) * H * prm.L_q * D;
   const unsigned cblocks = static_cast<unsigned>(std::min<size_t>((n / 4 + 255) / 256, 148 * 16));

@@ -24,15 +24,17 @@
 // TMA bulk reduce-add (the addition happens in L2, a tile at a time); the
 // other key blocks add theirs.
 //
-// Roles (512 threads): warpgroups 0 and 1 compute P and dS for query
-// columns [0, 64) and [64, 128) of every key row (thread = TMEM lane = key);
-// warp 8 issues the MMAs, warp 9 is the TMA producer; warpgroup 3 drains dQ
-// (thread = TMEM lane = query row).
+// Roles (768 threads): four warpgroups (0, 1, 4 and 5) compute P and dS,
+// each for 32 query columns of every key row (thread = TMEM lane = key), so
+// that four warps per SM sub-partition share the exponentials and the dS
+// math; warp 8 issues the MMAs, warp 9 is the TMA producer; warpgroup 3
+// drains dQ (thread = TMEM lane = query row).
 //
 // TMEM (512 columns): S^T [0,128) with P^T (two 16-bit values per column)
-// written over the first half of each warpgroup's columns; dP^T [128,256)
-// with dS^T likewise; dQ [128, 128+D) after dK has read dS^T (tcgen05 MMAs
-// of one thread run in order); dV [256, 256+D); dK [256+D, 256+2D).
+// written over the first half of each P/dS warpgroup's 32 columns; dP^T
+// [128,256) with dS^T likewise; dQ [128, 128+D) after dK has read dS^T
+// (tcgen05 MMAs of one thread run in order); dV [256, 256+D); dK
+// [256+D, 256+2D).
 //
 // Every wait is bounded (sm100.cuh); after a timeout each role leaves its
 // loop, the producer lets its copies land, and TMEM is freed.
@@ -66,15 +68,27 @@ struct BwdParams {
   long long mask_sb, mask_sh, mask_sq;
 };
 
-constexpr int kBwdThreads = 512;
-constexpr uint32_t kBwdLaunchRegs = 128;   // 65536 / 512
-// setmaxnreg split: P/dS warpgroups, dQ drain warpgroup, MMA/TMA warpgroup;
-// 2 * 144 + 168 + 56 = 4 * 128 (the launch allocation)
-constexpr uint32_t kBwdRegsPds = 144;
-constexpr uint32_t kBwdRegsDrain = 168;
-constexpr uint32_t kBwdRegsIssue = 56;
-static_assert(2 * kBwdRegsPds + kBwdRegsDrain + kBwdRegsIssue == 4 * kBwdLaunchRegs,
-              "register split must fit in the launch allocation");
+// Launch shape by head dim.  D <= 64 (dQ has TMEM columns of its own): the
+// P / dS math sets the step, so four P/dS warpgroups of 32 query columns
+// (768 threads, four warps per SM sub-partition); D > 64: the dQ drain ->
+// dP chain sets it, and two warpgroups of 64 columns (512 threads) draw less
+// power.  setmaxnreg split: P/dS warpgroups, dQ drain warpgroup, MMA/TMA
+// warpgroup, adding up to the launch allocation (registers per thread,
+// 65536 / threads in steps of 8; the host checks the built count).
+template <int D>
+struct BwdCfg {
+  static constexpr int kPdsGroups = D <= 64 ? 4 : 2;
+  static constexpr int kThreads = 256 + 128 * kPdsGroups;
+  static constexpr int kPdsCols = kBM / kPdsGroups;       // query columns per warpgroup
+  static constexpr uint32_t kLaunchRegs = D <= 64 ? 80 : 128;
+  static constexpr uint32_t kRegsPds = D <= 64 ? 80 : 144;
+  static constexpr uint32_t kRegsDrain = D <= 64 ? 104 : 168;
+  static constexpr uint32_t kRegsIssue = 56;
+  static_assert(kPdsGroups * kRegsPds + kRegsDrain + kRegsIssue ==
+                    (kThreads / 128) * kLaunchRegs,
+                "register split must fit in the launch allocation");
+  static_assert(kThreads * kLaunchRegs <= 65536, "launch allocation");
+};
 
 template <int D>
 struct BwdGeo {
@@ -159,9 +173,11 @@ __device__ __forceinline__ float bwd_mask_bias2(const BwdParams &p, long long id
 }
 
 template <int D, int DT, bool kMask>
-__global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
+    fa_bwd_kernel(const __grid_constant__ BwdParams p) {
   using G = Geo<D>;
   using BG = BwdGeo<D>;
+  using BC = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -197,8 +213,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     mbar_init(smem_u32(&bars->do_empty), 1);
     mbar_init(smem_u32(&bars->s_full), 1);
     mbar_init(smem_u32(&bars->dp_full), 1);
-    mbar_init(smem_u32(&bars->p_full), 256);
-    mbar_init(smem_u32(&bars->ds_full), 256);
+    mbar_init(smem_u32(&bars->p_full), 128 * BC::kPdsGroups);
+    mbar_init(smem_u32(&bars->ds_full), 128 * BC::kPdsGroups);
     mbar_init(smem_u32(&bars->dq_full), 1);
     mbar_init(smem_u32(&bars->dq_free), 128);
     mbar_init(smem_u32(&bars->mma_done), 1);
@@ -228,7 +244,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
 
   if (warp >= 8 && warp < 12) {
   // ===================================================== warpgroup 2
-  regs_dec<kBwdRegsIssue>();
+  regs_dec<BC::kRegsIssue>();
   if (warp == 9) {
     // =================================================== TMA producer
     const uint64_t pol_keep = policy_evict_last();
@@ -324,13 +340,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         }
         __syncwarp();
       };
-      // D_acc += X^T(TMEM, 16-bit, two warpgroups' halves) * B (MN-major tile)
+      // D_acc += X^T(TMEM, 16-bit, the P/dS warpgroups' packed columns) * B
+      // (MN-major tile); 16 queries = 8 packed columns, BC::kPdsCols per warpgroup
       auto issue_ts = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_tile, bool first) {
         const uint32_t blo = desc_lo(b_tile, G::kBoxBytes);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
-            const uint32_t a = a_base + (kk >> 2) * 64u + (kk & 3) * 8u;
+            constexpr int kSteps = BC::kPdsCols / 16;    // K steps per warpgroup
+            const uint32_t a = a_base + (kk / kSteps) * BC::kPdsCols + (kk % kSteps) * 8u;
             mma_ts(d_tmem, a, desc_join(blo + ((kk * 16 * G::kSwBytes) >> 4), kHi), kIdescKV,
                    (!first || kk > 0) ? 1u : 0u);
           }
@@ -411,46 +429,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     if (elect_one()) tc_commit(smem_u32(&bars->mma_done));
     __syncwarp();
   }
-  } else if (warp < 8) {
+  } else if (warp < 8 || warp >= 16) {
     // =================================================== P and dS
-    regs_inc<kBwdRegsPds>();
-    const int wg = warp >> 2;                      // query columns [64 wg, 64 wg + 64)
+    if constexpr (BC::kRegsPds > BC::kLaunchRegs) regs_inc<BC::kRegsPds>();
+    const int wg = warp >> 2;
+    const int pw = wg < 2 ? wg : wg - 2;           // query columns [kPdsCols pw, kPdsCols (pw + 1))
     const int r = tid & 127;                       // key row = TMEM lane
-    const int tc = tid;                            // 0..255: slot in the lse2 / delta buffer
+    const int tc = pw * 128 + r;                   // slot in the lse2 / delta buffer if < 256
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + 64u * wg;
-    const uint32_t tDP = tmem + lane_base + 128u + 64u * wg;
+    const uint32_t tS = tmem + lane_base + BC::kPdsCols * pw;
+    const uint32_t tDP = tmem + lane_base + 128u + BC::kPdsCols * pw;
     const int j = k0 + r;                          // key index of this row
     const float sl2 = p.scale_log2;
     bool ok = true;
-    // lse2 / delta of the next step, one value per thread
+    // lse2 / delta of the next step, one value per thread of the first two warpgroups
     auto fetch = [&](int n) -> float {
       const size_t base = static_cast<size_t>(bh_of(n)) * p.L_q_pad + q0_of(n) + (tc & 127);
       return tc < 128 ? p.lse2[base] : p.delta[base];
     };
-    float nxt = n_steps > 0 ? fetch(0) : 0.0f;
-    // Every warp of both warpgroups passes the two named barriers of every
-    // step, also after a timeout (then the step's work is skipped).
+    float nxt = (n_steps > 0 && tc < 256) ? fetch(0) : 0.0f;
+    // Every warp of the four warpgroups passes the two named barriers of
+    // every step, also after a timeout (then the step's work is skipped).
     for (int n = 0; n < n_steps; ++n) {
-      named_barrier_sync(1, 256);                  // the buffer of step n-1 is no longer read
-      s_vec[tc] = nxt;
-      named_barrier_sync(1, 256);
-      if (n + 1 < n_steps) nxt = fetch(n + 1);
+      named_barrier_sync(1, 128 * BC::kPdsGroups);  // the buffer of step n-1 is no longer read
+      if (tc < 256) s_vec[tc] = nxt;
+      named_barrier_sync(1, 128 * BC::kPdsGroups);
+      if (n + 1 < n_steps && tc < 256) nxt = fetch(n + 1);
       if (!ok) continue;
       const int q0 = q0_of(n);
-      const int qc = q0 + 64 * wg;                 // first query column of this thread
+      const int qc = q0 + BC::kPdsCols * pw;        // first query column of this thread
       const bool full = (k0 + kBN - 1 < p.L_k) && (p.wr < 0 || k0 + kBN - 1 <= q0 + p.wr) &&
                         (p.wl < 0 || k0 >= q0 + kBM - 1 - p.wl);
-      const float *lse2 = s_vec + 64 * wg;
-      const float *dlt = s_vec + 128 + 64 * wg;
+      const float *lse2 = s_vec + BC::kPdsCols * pw;
+      const float *dlt = s_vec + 128 + BC::kPdsCols * pw;
 
       // ---- P^T = 2^(s * scale * log2e - lse2), masked entries 0
       ok = mbar_wait_warp(smem_u32(&bars->s_full), n & 1, abort_flag);
       if (!ok) continue;
       tc_fence_after_sync();
-      float pr[64];
+      float pr[BC::kPdsCols];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < BC::kPdsCols / 32; ++h) {   // 32-column chunks
         uint32_t sr[32];
         tmem_ld_x32(tS + 32 * h, sr);
         tmem_wait_ld();
@@ -461,17 +480,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           const int bh = bh_of(n);
           const long long mrow = static_cast<long long>(bh / p.H) * p.mask_sb +
                                  static_cast<long long>(bh % p.H) * p.mask_sh + j;
-          float bias[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int i = qc + 32 * h + c;
-            bias[c] = (i < p.L_q && j < p.L_k)
-                          ? bwd_mask_bias2(p, mrow + static_cast<long long>(i) * p.mask_sq)
-                          : 0.0f;
+            const float bias = (i < p.L_q && j < p.L_k)
+                                   ? bwd_mask_bias2(p, mrow + static_cast<long long>(i) * p.mask_sq)
+                                   : 0.0f;
+            pr[32 * h + c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, bias - lse2[32 * h + c]));
           }
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            pr[32 * h + c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, bias[c] - lse2[32 * h + c]));
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
@@ -480,17 +496,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       }
       if (!full) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < BC::kPdsCols; ++c) {
           const int i = qc + c;
           const bool vis = (j < p.L_k) && (p.wr < 0 || j <= i + p.wr) && (p.wl < 0 || j >= i - p.wl);
           if (!vis) pr[c] = 0.0f;
         }
       }
       {
-        uint32_t pk[32];
+        uint32_t pk[BC::kPdsCols / 2];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) pk[u] = pack2<DT>(pr[2 * u], pr[2 * u + 1]);
-        tmem_st_x32(tS, pk);                       // over S^T columns already read
+        for (int u = 0; u < BC::kPdsCols / 2; ++u) pk[u] = pack2<DT>(pr[2 * u], pr[2 * u + 1]);
+        tmem_st_cols<BC::kPdsCols / 2>(tS, pk);    // over S^T columns already read
         tmem_wait_st();
       }
       tc_fence_before_sync();
@@ -505,25 +521,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         ok = mbar_wait_warp(smem_u32(&bars->dq_full), (n - 1) & 1, abort_flag);
         if (!ok) continue;
       }
-      uint8_t *ds_row = smem + BG::kOffDs + wg * BG::kDsBoxBytes + r * 128;
+      // this thread's queries in the box of 64 that holds them: its row of
+      // 128 bytes, from 16-byte unit u0 on; chunks of kCh columns
+      constexpr int kCh = BC::kPdsCols >= 64 ? 32 : 16;
+      const int q_first = BC::kPdsCols * pw;
+      uint8_t *ds_row = smem + BG::kOffDs + (q_first >> 6) * BG::kDsBoxBytes + r * 128;
+      const int u0 = (q_first & 63) >> 3;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t dp[32];
-        tmem_ld_x32(tDP + 32 * h, dp);
+      for (int h = 0; h < BC::kPdsCols / kCh; ++h) {
+        uint32_t dp[kCh];
+        tmem_ld_cols<kCh>(tDP + kCh * h, dp);
         tmem_wait_ld();
         reg_dep(dp);
-        uint32_t pk[16];
+        uint32_t pk[kCh / 2];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int c = 32 * h + 2 * u;
+        for (int u = 0; u < kCh / 2; ++u) {
+          const int c = kCh * h + 2 * u;
           const float d0 = pr[c] * (__uint_as_float(dp[2 * u]) - dlt[c]) * p.scale;
           const float d1 = pr[c + 1] * (__uint_as_float(dp[2 * u + 1]) - dlt[c + 1]) * p.scale;
           pk[u] = pack2<DT>(d0, d1);
         }
-        tmem_st_x16(tDP + 16 * h, pk);             // over dP^T columns already read
+        tmem_st_cols<kCh / 2>(tDP + (kCh / 2) * h, pk);   // over dP^T columns already read
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = 4 * h + u;              // 16-byte unit of the 128-byte row
+        for (int u = 0; u < kCh / 8; ++u) {
+          const int unit = u0 + (kCh / 8) * h + u;     // 16-byte unit of the 128-byte row
           *reinterpret_cast<uint4 *>(ds_row + ((unit ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
@@ -534,17 +555,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       mbar_arrive(smem_u32(&bars->ds_full));
     }
 
-    // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 dK (row j of this block)
+    // ---- epilogue (row j of this block): P/dS warpgroups 0 (and 2) write
+    // dV, 1 (and 3) dK; with four, each the 32-column chunks of one parity
     if (ok && n_steps > 0) {
       ok = mbar_wait_warp(smem_u32(&bars->mma_done), 0, abort_flag);
       if (ok) tc_fence_after_sync();
     }
     if (ok) {
-      const uint32_t tAcc = tmem + lane_base + 256u + (wg ? D : 0);
-      uint8_t *dst = static_cast<uint8_t *>(wg ? p.dk : p.dv) +
+      const int acc = pw & 1;                      // 0: dV, 1: dK
+      const uint32_t tAcc = tmem + lane_base + 256u + (acc ? D : 0);
+      uint8_t *dst = static_cast<uint8_t *>(acc ? p.dk : p.dv) +
                      (static_cast<size_t>(bh_kv) * p.L_k + j) * D * 2;
       for_o_chunks<D>([&](int c, auto wd) {   // 32-column chunks, 16-column tail
         constexpr int W = decltype(wd)::value;
+        if (((c >> 5) % (BC::kPdsGroups / 2)) != (pw >> 1)) return;
         uint32_t o[W];
         if (n_steps > 0) {
           tmem_ld_cols<W>(tAcc + c, o);
@@ -567,7 +591,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     }
   } else {
     // =================================================== dQ drain (warps 12-15)
-    regs_inc<kBwdRegsDrain>();
+    regs_inc<BC::kRegsDrain>();
     const int r = tid & 127;                       // query row within the block = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tDQ = tmem + lane_base + BG::kDqCol;

@@ -371,3 +371,27 @@ def test_test_library_exports_the_hook():
         pytest.skip("watchdog test library not built (build(testhooks=True))")
     t = ctypes.CDLL(fa_build.TESTHOOKS_PATH)
     assert hasattr(t, "fa_test_set_withhold") and hasattr(t, "fa_fwd")
+
+
+def test_register_check_follows_the_backward_launch_shape():
+    # the build refuses instances whose register count differs from the
+    # launch allocation their setmaxnreg split adds up to: 168 for the
+    # forward, 80 for the D <= 64 backward (768 threads), 128 above (512)
+    from exact_attention_113_b200 import build as fa_build
+
+    def log(entries):
+        return "\n".join(f"ptxas info    : Compiling entry function '{name}' for 'sm_100a'\n"
+                         f"ptxas info    : Used {regs} registers, used 3 barriers"
+                         for name, regs in entries)
+    fwd = ("_ZN2fa13fa_fwd_kernelILi128ELi0ELb0ELb0EEEvNS_9FwdParamsE", 168)
+    good = [fwd, ("_ZN2fa13fa_bwd_kernelILi64ELi0ELb0EEEvNS_9BwdParamsE", 80),
+            ("_ZN2fa13fa_bwd_kernelILi16ELi1ELb1EEEvNS_9BwdParamsE", 80),
+            ("_ZN2fa13fa_bwd_kernelILi128ELi0ELb0EEEvNS_9BwdParamsE", 128),
+            ("_ZN2fa13fa_bwd_kernelILi80ELi1ELb0EEEvNS_9BwdParamsE", 128)]
+    counts = fa_build.check_register_counts(log(good))
+    assert len(counts) == len(good)
+    for wrong in (("_ZN2fa13fa_bwd_kernelILi64ELi0ELb0EEEvNS_9BwdParamsE", 128),
+                  ("_ZN2fa13fa_bwd_kernelILi96ELi0ELb0EEEvNS_9BwdParamsE", 80),
+                  ("_ZN2fa13fa_fwd_kernelILi64ELi0ELb0ELb0EEEvNS_9FwdParamsE", 160)):
+        with pytest.raises(RuntimeError, match="launch allocation"):
+            fa_build.check_register_counts(log(good + [wrong]))
