@@ -442,10 +442,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     const int j = k0 + r;                          // key index of this row
     const float sl2 = p.scale_log2;
     bool ok = true;
-    // lse2 / delta of the next step, one value per thread of the first two warpgroups
+    // the math on packed fp32 pairs where it is the step's limit (four
+    // warpgroups); with two, the scalar form keeps the registers unspilled
+    constexpr bool kPacked = BC::kPdsGroups == 4;
+    // lse2 / delta of the next step, one value per thread of the first two
+    // warpgroups (packed: -delta * scale, the dS form below)
     auto fetch = [&](int n) -> float {
       const size_t base = static_cast<size_t>(bh_of(n)) * p.L_q_pad + q0_of(n) + (tc & 127);
-      return tc < 128 ? p.lse2[base] : p.delta[base];
+      if (tc < 128) return p.lse2[base];
+      return kPacked ? -p.delta[base] * p.scale : p.delta[base];
     };
     float nxt = (n_steps > 0 && tc < 256) ? fetch(0) : 0.0f;
     // Every warp of the four warpgroups passes the two named barriers of
@@ -487,6 +492,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
                                    ? bwd_mask_bias2(p, mrow + static_cast<long long>(i) * p.mask_sq)
                                    : 0.0f;
             pr[32 * h + c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, bias - lse2[32 * h + c]));
+          }
+        } else if constexpr (kPacked) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                make_float2(sl2, sl2), make_float2(-lse2[32 * h + c], -lse2[32 * h + c + 1]));
+            pr[32 * h + c] = ex2(x.x);
+            pr[32 * h + c + 1] = ex2(x.y);
           }
         } else {
 #pragma unroll
@@ -537,9 +551,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
         for (int u = 0; u < kCh / 2; ++u) {
           const int c = kCh * h + 2 * u;
-          const float d0 = pr[c] * (__uint_as_float(dp[2 * u]) - dlt[c]) * p.scale;
-          const float d1 = pr[c + 1] * (__uint_as_float(dp[2 * u + 1]) - dlt[c + 1]) * p.scale;
-          pk[u] = pack2<DT>(d0, d1);
+          if constexpr (kPacked) {
+            // P * (dP * scale + (-delta * scale))
+            const float2 g = __ffma2_rn(
+                make_float2(__uint_as_float(dp[2 * u]), __uint_as_float(dp[2 * u + 1])),
+                make_float2(p.scale, p.scale), make_float2(dlt[c], dlt[c + 1]));
+            const float2 dd = __fmul2_rn(make_float2(pr[c], pr[c + 1]), g);
+            pk[u] = pack2<DT>(dd.x, dd.y);
+          } else {
+            const float d0 = pr[c] * (__uint_as_float(dp[2 * u]) - dlt[c]) * p.scale;
+            const float d1 = pr[c + 1] * (__uint_as_float(dp[2 * u + 1]) - dlt[c + 1]) * p.scale;
+            pk[u] = pack2<DT>(d0, d1);
+          }
         }
         tmem_st_cols<kCh / 2>(tDP + (kCh / 2) * h, pk);   // over dP^T columns already read
 #pragma unroll
