@@ -24,17 +24,21 @@
 // TMA bulk reduce-add (the addition happens in L2, a tile at a time); the
 // other key blocks add theirs.
 //
-// Roles (768 threads): four warpgroups (0, 1, 4 and 5) compute P and dS,
-// each for 32 query columns of every key row (thread = TMEM lane = key), so
-// that four warps per SM sub-partition share the exponentials and the dS
-// math; warp 8 issues the MMAs, warp 9 is the TMA producer; warpgroup 3
-// drains dQ (thread = TMEM lane = query row).
+// Roles: P/dS warpgroups compute P and dS for a share of the query columns
+// of every key row (thread = TMEM lane = key): for D <= 64 four of them
+// (warpgroups 0, 1, 4 and 5; 32 columns each, 768 threads), so that four
+// warps per SM sub-partition share the exponentials and the dS math; for
+// D > 64 two (warpgroups 0 and 1; 64 columns each, 512 threads).  Warp 8
+// issues the MMAs, warp 9 is the TMA producer; warpgroup 3 drains dQ
+// (thread = TMEM lane = query row).
 //
-// TMEM (512 columns): S^T [0,128) with P^T (two 16-bit values per column)
-// written over the first half of each P/dS warpgroup's 32 columns; dP^T
-// [128,256) with dS^T likewise; dQ [128, 128+D) after dK has read dS^T
-// (tcgen05 MMAs of one thread run in order); dV [256, 256+D); dK
-// [256+D, 256+2D).
+// TMEM (512 columns): S^T [0,128); dP^T [128,256) with dS^T (two 16-bit
+// values per column) written over the first half of each P/dS warpgroup's
+// columns; dV [256, 256+D); dK [256+D, 256+2D).  D > 64: P^T over S^T
+// likewise, and dQ [128, 128+D) after dK has read dS^T (tcgen05 MMAs of
+// one thread run in order).  D <= 64: dQ [384, 384+D) of its own; D = 16
+// also P^T [448, 512), so that S^T of the next step is computed while P of
+// this one is.
 //
 // Every wait is bounded (sm100.cuh); after a timeout each role leaves its
 // loop, the producer lets its copies land, and TMEM is freed.
@@ -84,6 +88,12 @@ struct BwdCfg {
   static constexpr uint32_t kRegsPds = D <= 64 ? 80 : 144;
   static constexpr uint32_t kRegsDrain = D <= 64 ? 104 : 168;
   static constexpr uint32_t kRegsIssue = 56;
+  // D = 16: P^T goes to TMEM columns [448, 512), free there (S^T, dP^T,
+  // dV, dK and dQ take [0, 384 + D)), so S^T of the next step can be
+  // computed while P of this one is: once every P/dS thread holds S^T(n).
+  // (+9 % at D = 16; at D = 32 and 64 the earlier S MMA cost 1-5 %.)
+  static constexpr bool kEarlyS = D <= 16;
+  static constexpr uint32_t kPCol = 448;
   static_assert(kPdsGroups * kRegsPds + kRegsDrain + kRegsIssue ==
                     (kThreads / 128) * kLaunchRegs,
                 "register split must fit in the launch allocation");
@@ -142,6 +152,8 @@ struct BwdBars {
   uint64_t ds_full;
   uint64_t dq_full;
   uint64_t dq_free;
+  uint64_t s_free;        // early S^T: every P/dS thread holds S^T of the step
+  uint64_t p_free;        // early S^T: dV of the step has read P^T
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -217,6 +229,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_init(smem_u32(&bars->ds_full), 128 * BC::kPdsGroups);
     mbar_init(smem_u32(&bars->dq_full), 1);
     mbar_init(smem_u32(&bars->dq_free), 128);
+    mbar_init(smem_u32(&bars->s_free), 128 * BC::kPdsGroups);
+    mbar_init(smem_u32(&bars->p_free), 1);
     mbar_init(smem_u32(&bars->mma_done), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -342,13 +356,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       };
       // D_acc += X^T(TMEM, 16-bit, the P/dS warpgroups' packed columns) * B
       // (MN-major tile); 16 queries = 8 packed columns, BC::kPdsCols per warpgroup
-      auto issue_ts = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_tile, bool first) {
+      // (wg_stride: TMEM columns between two warpgroups' packed values)
+      auto issue_ts = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_tile, bool first,
+                          uint32_t wg_stride) {
         const uint32_t blo = desc_lo(b_tile, G::kBoxBytes);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
             constexpr int kSteps = BC::kPdsCols / 16;    // K steps per warpgroup
-            const uint32_t a = a_base + (kk / kSteps) * BC::kPdsCols + (kk % kSteps) * 8u;
+            const uint32_t a = a_base + (kk / kSteps) * wg_stride + (kk % kSteps) * 8u;
             mma_ts(d_tmem, a, desc_join(blo + ((kk * 16 * G::kSwBytes) >> 4), kHi), kIdescKV,
                    (!first || kk > 0) ? 1u : 0u);
           }
@@ -378,12 +394,26 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       }
       for (int n = 0; n < n_steps && ok; ++n) {
         const int st = n & 1;
+        if (BC::kEarlyS && n + 1 < n_steps) {
+          // S^T(n+1) as soon as every P/dS thread holds S^T(n)
+          const int st1 = (n + 1) & 1;
+          ok = mbar_wait_warp(smem_u32(&bars->s_free), n & 1, abort_flag) &&
+               mbar_wait_warp(smem_u32(&bars->q_full[st1]), ((n + 1) >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_kmajor(tS, sK, sQ + st1 * G::kTileBytes, smem_u32(&bars->s_full));
+        }
         ok = mbar_wait_warp(smem_u32(&bars->p_full), n & 1, abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
-        issue_ts(tDV, tS, do_tile(n), n == 0);
+        if constexpr (BC::kEarlyS) {
+          issue_ts(tDV, tmem + BC::kPCol, do_tile(n), n == 0, BC::kPdsCols / 2);
+          commit(smem_u32(&bars->p_free));
+        } else {
+          issue_ts(tDV, tS, do_tile(n), n == 0, BC::kPdsCols);
+        }
         if constexpr (BG::kDoStages == 1) commit(smem_u32(&bars->do_empty));
-        if (n + 1 < n_steps) {
+        if (!BC::kEarlyS && n + 1 < n_steps) {
           const int st1 = (n + 1) & 1;
           ok = mbar_wait_warp(smem_u32(&bars->q_full[st1]), ((n + 1) >> 1) & 1, abort_flag);
           if (!ok) break;
@@ -393,7 +423,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         ok = mbar_wait_warp(smem_u32(&bars->ds_full), n & 1, abort_flag);
         if (!ok) break;
         tc_fence_after_sync();
-        issue_ts(tDK, tDP, sQ + st * G::kTileBytes, n == 0);
+        issue_ts(tDK, tDP, sQ + st * G::kTileBytes, n == 0, BC::kPdsCols);
         if (BG::kDqOwn && n > 0) {
           // dQ has its own columns: only dQ(n) waits for the drain of dQ(n-1)
           ok = mbar_wait_warp(smem_u32(&bars->dq_free), (n - 1) & 1, abort_flag);
@@ -479,6 +509,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tmem_ld_x32(tS + 32 * h, sr);
         tmem_wait_ld();
         reg_dep(sr);
+        if constexpr (BC::kEarlyS) {
+          // S^T(n) is in registers (one chunk): S^T(n+1) may overwrite it
+          static_assert(!BC::kEarlyS || BC::kPdsCols == 32, "one S chunk per thread");
+          tc_fence_before_sync();
+          mbar_arrive(smem_u32(&bars->s_free));
+        }
         if constexpr (kMask) {
           // this row's mask entries for the 32 query columns (one key per
           // lane: each load is 32 consecutive elements across the warp)
@@ -516,11 +552,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
           if (!vis) pr[c] = 0.0f;
         }
       }
+      if (BC::kEarlyS && n > 0) {
+        // dV(n-1) has read P^T(n-1) from the columns this store reuses
+        ok = mbar_wait_warp(smem_u32(&bars->p_free), (n - 1) & 1, abort_flag);
+        if (!ok) continue;
+      }
       {
         uint32_t pk[BC::kPdsCols / 2];
 #pragma unroll
         for (int u = 0; u < BC::kPdsCols / 2; ++u) pk[u] = pack2<DT>(pr[2 * u], pr[2 * u + 1]);
-        tmem_st_cols<BC::kPdsCols / 2>(tS, pk);    // over S^T columns already read
+        // early S^T: P^T's own columns; else over S^T columns already read
+        tmem_st_cols<BC::kPdsCols / 2>(
+            BC::kEarlyS ? tmem + lane_base + BC::kPCol + (BC::kPdsCols / 2) * pw : tS, pk);
         tmem_wait_st();
       }
       tc_fence_before_sync();
