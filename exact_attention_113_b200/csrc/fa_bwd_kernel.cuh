@@ -472,15 +472,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     const int j = k0 + r;                          // key index of this row
     const float sl2 = p.scale_log2;
     bool ok = true;
-    // the math on packed fp32 pairs where it is the step's limit (four
-    // warpgroups); with two, the scalar form keeps the registers unspilled
+    // dS on packed fp32 pairs (every layout); P's exponent argument too
+    // where the P/dS math sets the step (four warpgroups; with two the
+    // scalar form spills less)
     constexpr bool kPacked = BC::kPdsGroups == 4;
-    // lse2 / delta of the next step, one value per thread of the first two
-    // warpgroups (packed: -delta * scale, the dS form below)
+    // lse2 / -delta * scale (the dS form below) of the next step, one value
+    // per thread of the first two warpgroups
     auto fetch = [&](int n) -> float {
       const size_t base = static_cast<size_t>(bh_of(n)) * p.L_q_pad + q0_of(n) + (tc & 127);
       if (tc < 128) return p.lse2[base];
-      return kPacked ? -p.delta[base] * p.scale : p.delta[base];
+      return -p.delta[base] * p.scale;
     };
     float nxt = (n_steps > 0 && tc < 256) ? fetch(0) : 0.0f;
     // Every warp of the four warpgroups passes the two named barriers of
@@ -594,18 +595,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 #pragma unroll
         for (int u = 0; u < kCh / 2; ++u) {
           const int c = kCh * h + 2 * u;
-          if constexpr (kPacked) {
-            // P * (dP * scale + (-delta * scale))
-            const float2 g = __ffma2_rn(
-                make_float2(__uint_as_float(dp[2 * u]), __uint_as_float(dp[2 * u + 1])),
-                make_float2(p.scale, p.scale), make_float2(dlt[c], dlt[c + 1]));
-            const float2 dd = __fmul2_rn(make_float2(pr[c], pr[c + 1]), g);
-            pk[u] = pack2<DT>(dd.x, dd.y);
-          } else {
-            const float d0 = pr[c] * (__uint_as_float(dp[2 * u]) - dlt[c]) * p.scale;
-            const float d1 = pr[c + 1] * (__uint_as_float(dp[2 * u + 1]) - dlt[c + 1]) * p.scale;
-            pk[u] = pack2<DT>(d0, d1);
-          }
+          // P * (dP * scale + (-delta * scale))
+          const float2 g = __ffma2_rn(
+              make_float2(__uint_as_float(dp[2 * u]), __uint_as_float(dp[2 * u + 1])),
+              make_float2(p.scale, p.scale), make_float2(dlt[c], dlt[c + 1]));
+          const float2 dd = __fmul2_rn(make_float2(pr[c], pr[c + 1]), g);
+          pk[u] = pack2<DT>(dd.x, dd.y);
         }
         tmem_st_cols<kCh / 2>(tDP + (kCh / 2) * h, pk);   // over dP^T columns already read
 #pragma unroll
