@@ -134,6 +134,16 @@ def test_gqa(H, H_kv):
                  seed=6400 + H + H_kv))
 
 
+@pytest.mark.parametrize("D", [16, 32, 48])
+@pytest.mark.parametrize("dtype", [F16, BF16])
+def test_small_head_dims_over_many_steps(D, dtype):
+    # the four-warpgroup layout (D <= 64) and, at D = 16, P^T in its own
+    # TMEM columns with S^T of the next step started early: GQA groups of
+    # three heads, a causal window, several query blocks per key block
+    check_bwd(_w(B=2, H=6, H_kv=2, L_q=520, L_k=520, D=D, causal=True, window_left=300,
+                 dtype=dtype, seed=6450 + D + dtype))
+
+
 def test_fully_masked_rows():
     # rows 200.. see no key: lse = -inf, their dq is 0, they add nothing
     w = _w(L_q=500, L_k=200, D=64, causal=True, window_left=0, seed=6500)
